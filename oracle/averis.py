@@ -1,0 +1,144 @@
+"""Averis mean-residual split, its quantized operands and the reference
+products.  TEST INFRASTRUCTURE ONLY (see ``oracle/__init__``).
+
+From "The Curse and Blessing of Mean Bias in FP4-Quantized LLM Training":
+
+  * column mean over the l tokens, mu_X = (1/l) 1^T X, X in R^{l x m}
+    (Lighthouse review, section 二 2.1 "核心 Insight");
+  * forward:  Y_hat = 1 (mu_bar_X W_bar) + X_bar_R W_bar,
+              mu_bar_X = Q_4(mu_X),  X_bar_R = Q_4(X - 1 mu_X)
+    (Lighthouse review, section 二 "Averis 方法", forward equation;
+    gist.science technical summary, section 2 "Il Metodo Proposto: Averis",
+    which writes the same residual as X - 1 mu_X^T in column convention);
+  * backward (dgrad): dL/dX_hat = 1 (mu_bar_D W_bar^T) + D_bar_R W_bar^T,
+    the same split of the output gradient D (same section, backward
+    equation);
+  * cost: only reductions and elementwise subtractions (same section,
+    "计算开销"; arXiv abstract).
+
+Readings where the pages are silent:
+  * fixed fp32 order of the mean: rows cut into 256-token chunks; each chunk
+    partial starts at +0.0 and adds its rows in ascending order; the column
+    sum starts at +0.0 and adds the chunk partials in ascending chunk order;
+    mu = fl(S / l) (IEEE division);
+  * W_bar in the two equations is one symbol but two quantizations, one per
+    contraction axis: along m for the forward (stored [n, m/2]) and along n
+    for dgrad (stored [m, n/2]); weights are always rounded to nearest even;
+  * stochastic rounding (when selected) applies to the split operands X_R,
+    mu_X, D_R, mu_D and to the vanilla operands, each with its own stream tag.
+"""
+
+import numpy as np
+
+from .nvfp4 import NVFP4, nvfp4_quantize, nvfp4_dequantize
+
+CHUNK = 256
+
+# Philox stream tags (third counter word) per quantized operand.
+TAGS = {
+    "x_r": 1, "mu_x": 2, "d_r": 3, "mu_d": 4,
+    "w_fwd": 5, "w_dgrad": 6, "vanilla_x": 7, "vanilla_d": 8,
+}
+
+
+def _as_f32(X):
+    """Widen the input (fp32, or bf16 held as torch/uint16/float) to fp32
+    exactly."""
+    X = np.asarray(X)
+    if X.dtype == np.float32:
+        return X
+    if X.dtype == np.uint16:           # raw bf16 bit patterns
+        return (X.astype(np.uint32) << 16).view(np.float32)
+    return X.astype(np.float32)
+
+
+def column_mean(X):
+    """mu_j in the fixed order (256-row chunks, then chunks in order)."""
+    X = _as_f32(X)
+    l, m = X.shape
+    S = np.zeros(m, dtype=np.float32)
+    for c0 in range(0, l, CHUNK):
+        p = np.zeros(m, dtype=np.float32)
+        for i in range(c0, min(c0 + CHUNK, l)):
+            p = p + X[i]                # one fp32 add per column, row by row
+        S = S + p
+    return (S / np.float32(l)).astype(np.float32)
+
+
+def mean_residual_split(X, mu):
+    """X_R = fl(X - 1 mu), elementwise."""
+    return (_as_f32(X) - np.asarray(mu, dtype=np.float32)[None, :]).astype(np.float32)
+
+
+def column_mean_and_residual_amax(X):
+    """(mu, X_R, max|X_R|) with the amax taken directly from X_R."""
+    mu = column_mean(X)
+    XR = mean_residual_split(X, mu)
+    A = np.float32(np.max(np.abs(XR))) if XR.size else np.float32(0.0)
+    return mu, XR, A
+
+
+def _check_finite(X):
+    if not np.all(np.isfinite(X)):
+        raise ValueError("non-finite input")
+
+
+def averis_split_quant(X, rounding="sr", seed=0, offset=0, grad=False):
+    """(mu, X_R, mu_bar, X_bar_R) for activations (grad=False) or output
+    gradients (grad=True, which only changes the stream tags)."""
+    X = _as_f32(X)
+    _check_finite(X)
+    mu, XR, A = column_mean_and_residual_amax(X)
+    _check_finite(mu)
+    t_r, t_mu = (TAGS["d_r"], TAGS["mu_d"]) if grad else (TAGS["x_r"], TAGS["mu_x"])
+    xr_q = nvfp4_quantize(XR, rounding, seed, offset, t_r, amax=A)
+    mu_q = nvfp4_quantize(mu[None, :], rounding, seed, offset, t_mu)
+    return mu, XR, mu_q, xr_q
+
+
+def vanilla_quant(X, rounding="sr", seed=0, offset=0, grad=False):
+    """Q_4(X) with no split (the comparison path)."""
+    X = _as_f32(X)
+    _check_finite(X)
+    tag = TAGS["vanilla_d"] if grad else TAGS["vanilla_x"]
+    return nvfp4_quantize(X, rounding, seed, offset, tag)
+
+
+def quant_weight(W):
+    """(W_bar_fwd [n, m/2], W_bar_dgrad [m, n/2]) from W [m, n], RNE."""
+    W = _as_f32(W)
+    _check_finite(W)
+    w_fwd = nvfp4_quantize(np.ascontiguousarray(W.T), "rne", tag=TAGS["w_fwd"])
+    w_dgrad = nvfp4_quantize(W, "rne", tag=TAGS["w_dgrad"])
+    return w_fwd, w_dgrad
+
+
+def bias_row(mu_q: NVFP4, w_q: NVFP4):
+    """The rank-one row mu_bar W_bar (fp64), one value per output column."""
+    return (nvfp4_dequantize(mu_q) @ nvfp4_dequantize(w_q).T)[0]
+
+
+def gemm_reference(a_q: NVFP4, b_q: NVFP4, bias=None, rows=None):
+    """fp64 product deq(A) deq(B)^T (+ bias broadcast to every row).
+
+    ``rows`` restricts the product to a subset of output rows."""
+    A = nvfp4_dequantize(a_q)
+    if rows is not None:
+        A = A[np.asarray(rows)]
+    Y = A @ nvfp4_dequantize(b_q).T
+    if bias is not None:
+        Y = Y + np.asarray(bias, dtype=np.float64)[None, :]
+    return Y
+
+
+def averis_linear_reference(X, w_q: NVFP4, rounding="sr", seed=0, offset=0, grad=False):
+    """Forward (grad=False, w_q = W_bar_fwd) or dgrad (grad=True,
+    w_q = W_bar_dgrad) of the Averis linear: fp64 Y_hat plus the operands."""
+    mu, XR, mu_q, xr_q = averis_split_quant(X, rounding, seed, offset, grad)
+    b = bias_row(mu_q, w_q)
+    return gemm_reference(xr_q, w_q, b), dict(mu=mu, xr=XR, mu_q=mu_q, xr_q=xr_q, bias=b)
+
+
+def vanilla_linear_reference(X, w_q: NVFP4, rounding="sr", seed=0, offset=0, grad=False):
+    x_q = vanilla_quant(X, rounding, seed, offset, grad)
+    return gemm_reference(x_q, w_q), dict(x_q=x_q)
