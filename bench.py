@@ -1,0 +1,432 @@
+"""Benchmark of the Averis split NVFP4 linear layer (forward + dgrad).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl averis|reference]
+
+One step = one forward and one dgrad pass of the Qwen3-0.6B fused-QKV
+projection (X bf16 [8192, 1024], W [1024, 4096], dY bf16 [8192, 4096],
+Philox stochastic rounding): column reduce, split quantizer (+ mean quantizer
+and rank-one row) and tcgen05 FP4 GEMM for each pass, six kernel launches.
+The weight quantization is done once before timing (it runs once per weight
+update, not per linear) and is reported on its own.
+
+Metric: useful FLOPs 2*(2 l m n) per step / device time, TFLOP/s.  Device
+time: CUDA events around K replays of a CUDA graph of the step, inputs
+rotating over enough copies that they exceed the 126 MB L2; max over ranks.
+Under torchrun each rank runs its own replica (weak scaling, no collective in
+the data path: the layer needs none).  Prints one JSON line on rank 0.
+
+--impl reference times the CPU oracle (the plain restatement of the method
+that the tests compare against) on a bounded row sample of the same workload.
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L, M, N = 8192, 1024, 4096
+WORKLOAD = "Qwen3-0.6B fused QKV projection, forward + dgrad: X bf16 [8192, 1024], W [1024, 4096], dY bf16 [8192, 4096], stochastic rounding"
+METRIC = "Averis fwd+dgrad linear TFLOP/s (Qwen3-0.6B shapes); split-quant HBM GB/s"
+FLOPS_PER_STEP = 2 * (2 * L * M * N)
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="averis", choices=["averis", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-sample-rows", type=int, default=1024)
+    p.add_argument("--copies", type=int, default=4, help="input copies rotated between steps")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) != 6:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[2:]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline
+# ---------------------------------------------------------------------------
+def oracle_step(x, d, w_fwd_q, w_dgrad_q):
+    """One forward + dgrad of the Averis linear in the oracle."""
+    import oracle
+    oracle.averis_linear_reference(x, w_fwd_q, "sr", seed=1, offset=0)
+    oracle.averis_linear_reference(d, w_dgrad_q, "sr", seed=2, offset=0, grad=True)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_operands(rows):
+    import oracle
+    from quantized_gemm_column_b200 import inputs
+    X, W, D = inputs.workload1()
+    x = inputs.bf16_as_f32(X)[:rows]
+    d = inputs.bf16_as_f32(D)[:rows]
+    w_fwd_q, w_dgrad_q = oracle.quant_weight(inputs.bf16_as_f32(W))
+    return x, d, w_fwd_q, w_dgrad_q
+
+
+def cpu_baseline(rows, steps=1):
+    x, d, wf, wd = oracle_operands(rows)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle_step(x, d, wf, wd)
+    dt = (time.perf_counter() - t0) / steps
+    flops = 2 * (2 * rows * M * N)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"first {rows} of {L} tokens of X and dY (column mean, split, NVFP4 SR "
+                      f"quantization and fp64 product of the sample), {dt:.1f} s per fwd+dgrad"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    rows = 128
+    x, d, wf, wd = oracle_operands(rows)
+    for _ in range(args.warmup):
+        oracle_step(x, d, wf, wd)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(x, d, wf, wd)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = 2 * (2 * rows * M * N) / dt / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 product of e2m1 x e4m3 operands",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample_rows": rows},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"first {rows} of {L} tokens per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from quantized_gemm_column_b200 import api, inputs
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    api.load()
+
+    # inputs: `copies` replicas of (X, dY) so the rotating working set exceeds L2
+    X0, W0, D0 = inputs.workload1(seed_tag=rank)
+    copies = max(1, args.copies)
+    Xs = [X0.to(dev) for _ in range(copies)]
+    Ds = [D0.to(dev) for _ in range(copies)]
+    Wd = W0.to(dev)
+    w_fwd, w_dgrad = api.NVFP4Tensor(N, M, dev), api.NVFP4Tensor(M, N, dev)
+    ws = api.workspace(L, N, N, dev)
+    Y = torch.empty((L, N), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((L, M), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.Stream(dev)
+
+    def step(i, s=None):
+        api.averis_linear_fwd(Xs[i % copies], w_fwd, "sr", 1 + i, 0, Y, ws, stream=s)
+        api.averis_linear_dgrad(Ds[i % copies], w_dgrad, "sr", 1 + i, 0, dX, ws, stream=s)
+
+    def vanilla_step(i, s=None):
+        api.nvfp4_linear_fwd(Xs[i % copies], w_fwd, "sr", 1 + i, 0, Y, ws, stream=s)
+        api.nvfp4_linear_dgrad(Ds[i % copies], w_dgrad, "sr", 1 + i, 0, dX, ws, stream=s)
+
+    with torch.cuda.stream(stream):
+        # weight quantization (once per weight update), timed alone
+        api.averis_quant_weight(Wd, w_fwd, w_dgrad, ws, stream=stream)
+        torch.cuda._sleep(20_000_000)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(10):
+            api.averis_quant_weight(Wd, w_fwd, w_dgrad, ws, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        wq_us = e0.elapsed_time(e1) * 1e3 / 10
+        for i in range(2):
+            step(i, stream)
+            vanilla_step(i, stream)
+        torch.cuda.synchronize(dev)
+    st = api.averis_check_status(ws, stream)
+    if st:
+        raise RuntimeError(f"device status {st} during warm-up")
+
+    # CUDA graphs: one per input copy for the Averis step and the vanilla step
+    graphs, vgraphs, launch = [], [], "cuda-graph"
+    try:
+        for i in range(copies):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step(i, stream)
+            graphs.append(g)
+            vg = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(vg, stream=stream):
+                vanilla_step(i, stream)
+            vgraphs.append(vg)
+    except Exception as exc:   # capture unsupported: time eager launches instead
+        graphs, vgraphs, launch = [], [], f"eager ({type(exc).__name__})"
+        torch.cuda.synchronize(dev)
+
+    def replay(i, vanilla=False):
+        if graphs:
+            (vgraphs if vanilla else graphs)[i % copies].replay()
+        else:
+            (vanilla_step if vanilla else step)(i, stream)
+
+    def timed(n, vanilla=False):
+        with torch.cuda.stream(stream):
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize(dev)
+            torch.cuda._sleep(5_000_000)            # let the host run ahead of the device
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for i in range(n):
+                replay(i, vanilla)
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            if world > 1:
+                dist.barrier()
+            return a.elapsed_time(b)                # ms
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            replay(i)
+            replay(i, True)
+        torch.cuda.synchronize(dev)
+
+    with ClockSampler(local_rank) as clk:
+        ms = timed(args.steps)
+        ms_van = timed(args.steps, vanilla=True)
+    clocks = clk.summary()
+    st = api.averis_check_status(ws, stream)
+    if st:
+        raise RuntimeError(f"device status {st} in the timed region")
+
+    ms_t = torch.tensor([ms, ms_van], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms, ms_van = float(ms_t[0]), float(ms_t[1])
+    step_ms = ms / args.steps
+    value = FLOPS_PER_STEP * world / (step_ms * 1e-3) / 1e12
+
+    # per-kernel-group timing (same stream, events around n launches each)
+    xr = api.NVFP4Tensor(L, M, dev)
+    dr = api.NVFP4Tensor(L, N, dev)
+    muq, dmuq = api.NVFP4Tensor(1, M, dev), api.NVFP4Tensor(1, N, dev)
+
+    def avg_us(fn, n=20):
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                fn(i)
+            torch.cuda.synchronize(dev)
+            torch.cuda._sleep(5_000_000)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for i in range(n):
+                fn(i)
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) * 1e3 / n
+
+    sq_x = avg_us(lambda i: api.averis_split_quant(Xs[i % copies], "sr", 1, 0, False, None, muq, xr, None, ws, stream))
+    sq_d = avg_us(lambda i: api.averis_split_quant(Ds[i % copies], "sr", 1, 0, True, None, dmuq, dr, None, ws, stream))
+    g_f = avg_us(lambda i: api.nvfp4_gemm(xr, w_fwd, None, Y, ws, stream))
+    g_d = avg_us(lambda i: api.nvfp4_gemm(dr, w_dgrad, None, dX, ws, stream))
+    gemm_tflops = 2 * L * M * N * 2 / ((g_f + g_d) * 1e-6) / 1e12
+
+    # split-quant algorithmic bytes: read the input twice (reduce, quantize),
+    # write codes (1/2 byte per element) and scales (1/16 byte per element)
+    def sq_bytes(rows, K):
+        return rows * K * (2 * 2 + 0.5 + 1.0 / 16)
+    sq_gbs = (sq_bytes(L, M) + sq_bytes(L, N)) / ((sq_x + sq_d) * 1e-6) / 1e9
+
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        pass
+    bf16_peak = peaks.get("bf16_tflops", 1590.0)
+    fp4_peak = 4.0 * bf16_peak             # nominal dense FP4 : BF16 ratio 9 : 2.25
+    hbm_peak = peaks.get("hbm_gbs", 6650.0)
+    peak_src = "measured" if peaks else "fallback"
+
+    # dominant kernel group by time share of the step
+    gemm_share = (g_f + g_d) / (step_ms * 1e3)
+    if gemm_share >= 0.5:
+        roof = {"bound": "tensor", "kernel": "gemm_nvfp4_kernel (fwd + dgrad)",
+                "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
+                "frac": gemm_tflops / fp4_peak, "traffic": None,
+                "peak_source": f"{peak_src} bf16 x 4 (nominal FP4:BF16 ratio)"}
+    else:
+        roof = {"bound": "hbm", "kernel": "colreduce_kernel + quant_kernel (split-quant, X and dY)",
+                "achieved": sq_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": sq_gbs / hbm_peak,
+                "traffic": None, "peak_source": f"{peak_src} HBM copy"}
+
+    # end to end through the public API with host buffers
+    Xh = X0.pin_memory()
+    Dh = D0.pin_memory()
+    Yh = torch.empty((L, N), dtype=torch.bfloat16).pin_memory()
+    dXh = torch.empty((L, M), dtype=torch.bfloat16).pin_memory()
+    Xe, De = Xs[0], Ds[0]
+
+    def e2e_step(i):
+        Xe.copy_(Xh, non_blocking=True)
+        De.copy_(Dh, non_blocking=True)
+        api.averis_linear_fwd(Xe, w_fwd, "sr", 1 + i, 0, Y, ws, stream=stream)
+        api.averis_linear_dgrad(De, w_dgrad, "sr", 1 + i, 0, dX, ws, stream=stream)
+        Yh.copy_(Y, non_blocking=True)
+        dXh.copy_(dX, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    with torch.cuda.stream(stream):
+        for i in range(2):
+            e2e_step(i)
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+    e2e_ms = torch.tensor([a.elapsed_time(b) / e2e_steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_val = FLOPS_PER_STEP * world / (float(e2e_ms) * 1e-3) / 1e12
+    h2d = (X0.numel() + D0.numel()) * 2
+    d2h = (Y.numel() + dX.numel()) * 2
+
+    if rank != 0:
+        return
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        cpu = cpu_baseline(args.cpu_sample_rows)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e2m1 x e2m1 (e4m3 block scales) -> fp32 accumulate",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "l": L, "m": M, "n": N, "rounding": "philox-sr",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single gpu",
+                   "launch": launch,
+                   "l2": f"inputs rotate over {copies} copies of (X, dY) = "
+                         f"{copies * (L * M + L * N) * 2 / 2**20:.0f} MiB > 126 MB L2"},
+        "split_quant_gbs": sq_gbs,
+        "split_quant_us": {"X": sq_x, "dY": sq_d},
+        "gemm_us": {"fwd": g_f, "dgrad": g_d}, "gemm_tflops": gemm_tflops,
+        "gemm_frac_fp4_peak": gemm_tflops / fp4_peak,
+        "vanilla_ms_per_step": ms_van / args.steps,
+        "averis_overhead_vs_vanilla": (ms / ms_van) - 1.0,
+        "weight_quant_us": wq_us,
+        "roofline": roof,
+        "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
+                   "reasons": clocks["reasons"]},
+        "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 6 * args.steps,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    for g in graphs + vgraphs:
+        del g
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_gpu(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

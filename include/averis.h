@@ -1,0 +1,211 @@
+/*
+ * averis.h -- C ABI of libaveris: the Averis mean-residual split NVFP4
+ * linear layer (forward and dgrad) on NVIDIA B200 (sm_100a).
+ *
+ * Source of the method: "The Curse and Blessing of Mean Bias in
+ * FP4-Quantized LLM Training" (Cao, Huang et al.).  Passages cited below:
+ *   [R2.1]  Lighthouse review page, section 二 2.1 "核心 Insight": column mean
+ *           mu_X = (1/l) 1^T X of X in R^{l x m} (l tokens, m features).
+ *   [RAv]   same page, section 二 "Averis 方法": forward
+ *           Y_hat = 1 (mu_bar_X W_bar) + X_bar_R W_bar with mu_bar_X = Q_4(mu_X),
+ *           X_bar_R = Q_4(X - 1 mu_X); backward
+ *           dL/dX_hat = 1 (mu_bar_D W_bar^T) + D_bar_R W_bar^T; cost: two
+ *           reductions and two subtractions.
+ *   [R3.1]  same page, section 三 3.1: W4A4G4, E2M1 NVFP4, stochastic
+ *           rounding by default; vanilla FP4 as the comparison.
+ *   [Abs]   arXiv abstract page: mean-residual splitting with reductions and
+ *           elementwise subtractions before FP4 quantization; 2.20%
+ *           end-to-end overhead over vanilla NVFP4.
+ *   [GS2]   gist.science technical summary, section 2 "Il Metodo Proposto:
+ *           Averis": X_R = X - 1 mu_X^T, mean and residual quantized
+ *           separately, forward and backward recombined.
+ *
+ * Readings where the pages are silent (the same readings the CPU oracle
+ * follows): 16-element blocks along the contraction axis with unsigned E4M3
+ * block scales and one FP32 per-tensor decode scale g_dec = amax / 2688;
+ * the fixed fp32 order of the mean (256-row chunks summed row by row, then
+ * chunk partials in chunk order, mu = S / l); Philox4x32-10 random bits,
+ * 16 per element, for stochastic rounding; weights always round to nearest
+ * even.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers to caller-owned memory; the
+ *     library never allocates and never frees.  Row-major, contiguous.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and never synchronize, except averis_check_status.
+ *   - Validation happens on the host before any launch; a rejected call
+ *     launches nothing and returns a non-zero avr_status.  Launch failures
+ *     return AVR_ERR_CUDA.
+ *   - Conditions found on the device (a bounded wait that expired, a
+ *     non-finite mean or amax) are latched in the workspace status word and
+ *     returned by averis_check_status.  Outputs of such a call are undefined.
+ *   - `ws` is a device workspace of at least averis_workspace_size(l, K, N)
+ *     bytes (256-byte aligned).  It must be zero-filled before its first use
+ *     (averis_workspace_init); every call that completes leaves it reusable.
+ *     One workspace must not be used by two calls that may run concurrently.
+ *   - Shape rules: K (the contraction size) > 0 and K % 64 == 0; N % 64 == 0;
+ *     l (tokens / rows) >= 0, any value (l = 0 is a no-op returning AVR_OK, and
+ *     the tensor pointers may then be NULL);
+ *     every pointer 16-byte aligned; l, K, N < 2^31.
+ */
+#ifndef AVERIS_H_
+#define AVERIS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* avr_stream; /* same type as cudaStream_t */
+
+typedef enum {
+  AVR_OK = 0,
+  AVR_ERR_INVALID_ARG = 1,         /* null pointer, unknown enum value */
+  AVR_ERR_UNSUPPORTED_SHAPE = 2,   /* K % 64, N % 64, sizes out of range */
+  AVR_ERR_MISALIGNED = 3,          /* a pointer not 16-byte aligned */
+  AVR_ERR_WORKSPACE_TOO_SMALL = 4,
+  AVR_ERR_CUDA = 5,                /* a CUDA runtime/driver call failed */
+  AVR_ERR_DEVICE_TIMEOUT = 6,      /* a device-side bounded wait expired */
+  AVR_ERR_NONFINITE = 7,           /* the input held NaN/Inf (mean or amax not finite) */
+  AVR_ERR_NO_DEVICE = 8            /* current device is not an sm_100 GPU */
+} avr_status;
+
+typedef enum { AVR_F32 = 0, AVR_BF16 = 1 } avr_dtype;
+typedef enum { AVR_RNE = 0, AVR_SR = 1 } avr_round;
+
+/* An NVFP4 tensor T [rows, K] quantized along K ([R3.1] "E2M1 NVFP4").
+ *   codes  : rows * K/2 bytes; element 2k of a row in the low nibble of
+ *            byte k, element 2k+1 in the high nibble; E2M1 code = sign<<3 |
+ *            magnitude index into {0, .5, 1, 1.5, 2, 3, 4, 6}.
+ *   scales : avr_nvfp4_scales_bytes(rows, K) bytes of unsigned E4M3 block
+ *            scales in the tcgen05 block-scaling layout: 512-byte atoms of
+ *            128 rows x 4 scales, atom (r/128, c/4) at index
+ *            (r/128) * (K/64) + c/4, and inside an atom the scale of (r, c)
+ *            at byte 16*(r%32) + 4*((r%128)/32) + c%4.  Rows past `rows` up
+ *            to the next multiple of 128 are zero.
+ *   g_dec  : one fp32 per-tensor decode scale.
+ * value(r, k) = e2m1(code) * e4m3(scale(r, k/16)) * g_dec. */
+typedef struct {
+  uint8_t* codes;
+  uint8_t* scales;
+  float* g_dec;
+  int64_t rows;
+  int64_t K;
+} avr_nvfp4;
+
+/* Bytes of the scale array of an NVFP4 tensor [rows, K]. */
+size_t avr_nvfp4_scales_bytes(int64_t rows, int64_t K);
+
+/* Workspace bytes that cover every call below for l rows, contraction K and
+ * N output columns (N may be 0 for calls without a GEMM). */
+size_t averis_workspace_size(int64_t l, int64_t K, int64_t N);
+
+/* Zero-fill a workspace before its first use (stream ordered). */
+avr_status averis_workspace_init(void* ws, size_t ws_bytes, avr_stream stream);
+
+/* Synchronize `stream`, return the first device-side error latched in the
+ * workspace status word since the last check (AVR_OK if none) and clear it. */
+avr_status averis_check_status(void* ws, avr_stream stream);
+
+/* Static description of a status code. */
+const char* averis_status_string(avr_status status);
+
+/* -------------------------------------------------------------------------
+ * Split quantization [R2.1], [RAv], [GS2]
+ * ------------------------------------------------------------------------- */
+
+/* Mean-residual split and quantization of X [l, K] (K = the feature axis).
+ *   mu      [K] fp32 out : column mean in the fixed order (nullable).
+ *   mu_q    out          : Q_4(mu) as a 1 x K NVFP4 tensor (nullable).
+ *   xr_q    out          : Q_4(X - 1 mu), l x K.
+ *   xr_debug [l, K] fp32 : X_R itself (nullable; for tests).
+ *   grad = 0 for activations X (random-stream tags 1 and 2), 1 for output
+ *   gradients D (tags 3 and 4).  rm selects RNE or Philox SR; the stream of
+ *   element e (row-major index) is keyed by `seed` and counted from
+ *   `offset` + e/8.  Launches 2 kernels (column reduce, split-quantize). */
+avr_status averis_split_quant(const void* X, avr_dtype xt, int64_t l, int64_t K, avr_round rm,
+                              uint64_t seed, uint64_t offset, int grad, float* mu,
+                              const avr_nvfp4* mu_q, const avr_nvfp4* xr_q, float* xr_debug,
+                              void* ws, size_t ws_bytes, avr_stream stream);
+
+/* Vanilla NVFP4 quantization of X [rows, K] (no split; [R3.1] "Vanilla FP4").
+ * grad selects stream tag 7 (0) or 8 (1). */
+avr_status nvfp4_quant(const void* X, avr_dtype xt, int64_t rows, int64_t K, avr_round rm,
+                       uint64_t seed, uint64_t offset, int grad, const avr_nvfp4* out,
+                       void* ws, size_t ws_bytes, avr_stream stream);
+
+/* Both quantizations of a weight W [m, n] (W_bar in both equations of [RAv]):
+ *   w_fwd   : Q_4(W^T), n x m (blocks along m, the forward contraction);
+ *   w_dgrad : Q_4(W),   m x n (blocks along n, the dgrad contraction).
+ * Round to nearest even; one tensor scale (amax of W) for both.  Needs
+ * m % 64 == 0 and n % 64 == 0. */
+avr_status averis_quant_weight(const void* W, avr_dtype wt, int64_t m, int64_t n,
+                               const avr_nvfp4* w_fwd, const avr_nvfp4* w_dgrad, void* ws,
+                               size_t ws_bytes, avr_stream stream);
+
+/* The rank-one row mu_bar W_bar of [RAv]: bias[j] = sum_k value(mu_q)[k] *
+ * value(w_q)[j, k] in fp32, j < w_q->rows.  mu_q is 1 x K, w_q is N x K. */
+avr_status averis_bias_row(const avr_nvfp4* mu_q, const avr_nvfp4* w_q, float* bias, void* ws,
+                           size_t ws_bytes, avr_stream stream);
+
+/* Block-scaled FP4 GEMM on the tcgen05 tensor cores:
+ *   Y[i, j] = g_dec(a) g_dec(b) sum_k e2m1(a)e4m3(sa) e2m1(b)e4m3(sb) + bias[j]
+ * with A = a [M, K], B = b [N, K] (both K-major), bias [N] fp32 nullable,
+ * Y [M, N] in yt (row-major). */
+avr_status nvfp4_gemm(const avr_nvfp4* a, const avr_nvfp4* b, const float* bias, void* Y,
+                      avr_dtype yt, void* ws, size_t ws_bytes, avr_stream stream);
+
+/* -------------------------------------------------------------------------
+ * The linear layer [RAv]
+ * ------------------------------------------------------------------------- */
+
+/* Forward: Y [l, n] = 1 (Q_4(mu_X) W_bar) + Q_4(X - 1 mu_X) W_bar for
+ * X [l, m] and w_fwd = Q_4(W^T) [n, m].  save_xr / save_mu (nullable)
+ * receive the quantized operands for a later weight-gradient pass; when
+ * NULL they live in the workspace.  Three launches: column reduce,
+ * split-quantize (+ mean quantize + rank-one row), GEMM. */
+avr_status averis_linear_fwd(const void* X, avr_dtype xt, int64_t l, int64_t m, int64_t n,
+                             const avr_nvfp4* w_fwd, avr_round rm, uint64_t seed,
+                             uint64_t offset, void* Y, avr_dtype yt, const avr_nvfp4* save_xr,
+                             const avr_nvfp4* save_mu, void* ws, size_t ws_bytes,
+                             avr_stream stream);
+
+/* Dgrad: dX [l, m] = 1 (Q_4(mu_D) W_bar^T) + Q_4(D - 1 mu_D) W_bar^T for
+ * D [l, n] and w_dgrad = Q_4(W) [m, n]. */
+avr_status averis_linear_dgrad(const void* D, avr_dtype dt, int64_t l, int64_t m, int64_t n,
+                               const avr_nvfp4* w_dgrad, avr_round rm, uint64_t seed,
+                               uint64_t offset, void* dX, avr_dtype xt, void* ws,
+                               size_t ws_bytes, avr_stream stream);
+
+/* Vanilla NVFP4 forward / dgrad ([R3.1], [Abs] "vanilla NVFP4"): Y = Q_4(X)
+ * W_bar, dX = Q_4(D) W_bar^T, the same three launches without the split. */
+avr_status nvfp4_linear_fwd(const void* X, avr_dtype xt, int64_t l, int64_t m, int64_t n,
+                            const avr_nvfp4* w_fwd, avr_round rm, uint64_t seed, uint64_t offset,
+                            void* Y, avr_dtype yt, void* ws, size_t ws_bytes, avr_stream stream);
+avr_status nvfp4_linear_dgrad(const void* D, avr_dtype dt, int64_t l, int64_t m, int64_t n,
+                              const avr_nvfp4* w_dgrad, avr_round rm, uint64_t seed,
+                              uint64_t offset, void* dX, avr_dtype xt, void* ws, size_t ws_bytes,
+                              avr_stream stream);
+
+/* -------------------------------------------------------------------------
+ * Diagnostics (used by the tests to pin the number formats on the device)
+ * ------------------------------------------------------------------------- */
+
+/* For n fp32 inputs: e4m3[i] = E4M3 RNE-satfinite code of |in[i]| and
+ * e2m1[i] = E2M1 RNE-satfinite code of in[i], exactly as the quantizer
+ * computes them.  Either output may be NULL. */
+avr_status averis_probe_convert(const float* in, uint8_t* e4m3, uint8_t* e2m1, int64_t n,
+                                avr_stream stream);
+
+/* out[4*i .. 4*i+3] = Philox4x32-10 words of counter (lo32(offset+i),
+ * hi32(offset+i), tag, 0) under key (lo32(seed), hi32(seed)), i < n. */
+avr_status averis_probe_philox(uint64_t seed, uint64_t offset, uint32_t tag, int64_t n,
+                               uint32_t* out, avr_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AVERIS_H_ */

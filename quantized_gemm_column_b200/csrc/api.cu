@@ -1,0 +1,428 @@
+// The C ABI of libaveris (declared in include/averis.h): host-side
+// validation, workspace layout, tensor maps and the launch chains.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "internal.h"
+
+namespace avr {
+
+static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t scales_bytes(int64_t rows, int64_t K) {
+  const int64_t rows_pad = (rows + 127) / 128 * 128;
+  return static_cast<size_t>(rows_pad) * static_cast<size_t>(K / 16);
+}
+
+WsLayout ws_layout(int64_t l, int64_t K, int64_t N) {
+  WsLayout w;
+  size_t off = round_up(w.slots + 2 * sizeof(float) * kMaxColTiles, 256);
+  const size_t C = static_cast<size_t>((l + kChunkRows - 1) / kChunkRows);
+  w.partials = off;  off = round_up(off + 3 * C * static_cast<size_t>(K) * sizeof(float), 256);
+  w.mu = off;        off = round_up(off + static_cast<size_t>(K) * sizeof(float), 256);
+  w.mu_codes = off;  off = round_up(off + static_cast<size_t>(K) / 2, 256);
+  w.mu_scales = off; off = round_up(off + scales_bytes(1, K), 256);
+  w.mu_gdec = off;   off += 256;
+  w.xr_gdec = off;   off += 256;
+  w.bias = off;      off = round_up(off + static_cast<size_t>(N) * sizeof(float), 256);
+  w.xr_codes = off;  off = round_up(off + static_cast<size_t>(l) * static_cast<size_t>(K) / 2, 256);
+  w.xr_scales = off; off = round_up(off + scales_bytes(l, K), 256);
+  w.total = off;
+  return w;
+}
+
+// ---------------------------------------------------------------------------
+// driver entry point for tensor maps (no link-time dependency on libcuda)
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_tensor_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes,
+                        uint64_t rows, uint64_t cols, uint32_t box_rows, uint32_t box_cols,
+                        CUtensorMapSwizzle swizzle) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem_bytes)};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+cudaError_t set_max_dynamic_smem(const void* func, size_t bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<int, const void*>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> g(mu);
+  if (done.count({dev, func})) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e == cudaSuccess) done.insert({dev, func});
+  return e;
+}
+
+// ---------------------------------------------------------------------------
+// validation helpers
+// ---------------------------------------------------------------------------
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool dtype_ok(avr_dtype t) { return t == AVR_F32 || t == AVR_BF16; }
+static bool round_ok(avr_round r) { return r == AVR_RNE || r == AVR_SR; }
+constexpr int64_t kMaxDim = (int64_t{1} << 31) - 1;
+static bool k_ok(int64_t K) { return K > 0 && K % 64 == 0 && K <= int64_t{kColTile} * kMaxColTiles; }
+static bool l_ok(int64_t l) { return l >= 0 && l <= kMaxDim; }
+static bool n_ok(int64_t N) { return N > 0 && N % 64 == 0 && N <= kMaxDim; }
+
+static avr_status device_ok() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return AVR_ERR_NO_DEVICE;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return AVR_ERR_NO_DEVICE;
+  return major == 10 ? AVR_OK : AVR_ERR_NO_DEVICE;
+}
+
+static avr_status check_nvfp4(const avr_nvfp4* t, int64_t rows, int64_t K) {
+  if (!t || !t->codes || !t->scales || !t->g_dec) return AVR_ERR_INVALID_ARG;
+  if (t->rows != rows || t->K != K) return AVR_ERR_INVALID_ARG;
+  if (!aligned16(t->codes) || !aligned16(t->scales) || (reinterpret_cast<uintptr_t>(t->g_dec) & 3u))
+    return AVR_ERR_MISALIGNED;
+  return AVR_OK;
+}
+
+static avr_status cuda_status(cudaError_t e) { return e == cudaSuccess ? AVR_OK : AVR_ERR_CUDA; }
+
+#define AVR_TRY(expr)                  \
+  do {                                 \
+    avr_status st_ = (expr);           \
+    if (st_ != AVR_OK) return st_;     \
+  } while (0)
+
+struct Ws {
+  char* base;
+  WsLayout lay;
+  uint32_t* status() const { return reinterpret_cast<uint32_t*>(base + lay.status); }
+  float* slot_xr() const { return reinterpret_cast<float*>(base + lay.slots); }
+  float* slot_mu() const { return slot_xr() + kMaxColTiles; }
+  template <typename T>
+  T* at(size_t off) const { return reinterpret_cast<T*>(base + off); }
+};
+
+static avr_status make_ws(void* ws, size_t ws_bytes, int64_t l, int64_t K, int64_t N, Ws* out) {
+  if (!ws) return AVR_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return AVR_ERR_MISALIGNED;
+  out->base = static_cast<char*>(ws);
+  out->lay = ws_layout(l, K, N);
+  if (ws_bytes < out->lay.total) return AVR_ERR_WORKSPACE_TOO_SMALL;
+  return AVR_OK;
+}
+
+static int n_tiles(int64_t K) { return static_cast<int>((K + kColTile - 1) / kColTile); }
+
+// K1 + K2 (+ mean quantizer and rank-one row when mu_q / w are given)
+static avr_status split_chain(const void* X, avr_dtype xt, int64_t l, int64_t K, int split,
+                              avr_round rm, uint64_t seed, uint64_t offset, uint32_t tag,
+                              uint32_t tag_mu, float* mu_buf, const avr_nvfp4* mu_q,
+                              const avr_nvfp4* xr_q, float* xr_debug, const avr_nvfp4* w,
+                              float* bias, const Ws& ws, cudaStream_t s) {
+  ColReduceArgs ca;
+  ca.X = X;
+  ca.xt = xt;
+  ca.l = l;
+  ca.K = K;
+  ca.split = split;
+  ca.mu_out = mu_buf;
+  ca.ws = ws.base;
+  ca.lay = &ws.lay;
+  AVR_TRY(cuda_status(launch_colreduce(ca, s, true)));
+  QuantArgs qa = {};
+  qa.X = X;
+  qa.xt = xt;
+  qa.rows = l;
+  qa.K = K;
+  qa.mu = split ? mu_buf : nullptr;
+  qa.n_tiles = n_tiles(K);
+  qa.slot_xr = ws.slot_xr();
+  qa.codes = xr_q->codes;
+  qa.scales = xr_q->scales;
+  qa.g_dec = xr_q->g_dec;
+  qa.xr_debug = xr_debug;
+  qa.seed = seed;
+  qa.offset = offset;
+  qa.tag = tag;
+  qa.sr = rm == AVR_SR;
+  qa.status = ws.status();
+  qa.slot_mu = ws.slot_mu();
+  qa.tag_mu = tag_mu;
+  if (mu_q) {
+    qa.mu_codes = mu_q->codes;
+    qa.mu_scales = mu_q->scales;
+    qa.mu_gdec = mu_q->g_dec;
+  }
+  if (w) {
+    qa.w_codes = w->codes;
+    qa.w_scales = w->scales;
+    qa.w_gdec = w->g_dec;
+    qa.n_out = w->rows;
+    qa.bias = bias;
+  }
+  return cuda_status(launch_quant(qa, s, true));
+}
+
+static avr_status gemm(const avr_nvfp4* a, const avr_nvfp4* b, const float* bias, void* Y,
+                       avr_dtype yt, uint32_t* status, cudaStream_t s) {
+  GemmArgs g;
+  g.a_codes = a->codes;
+  g.a_scales = a->scales;
+  g.a_gdec = a->g_dec;
+  g.b_codes = b->codes;
+  g.b_scales = b->scales;
+  g.b_gdec = b->g_dec;
+  g.M = a->rows;
+  g.N = b->rows;
+  g.K = a->K;
+  g.bias = bias;
+  g.Y = Y;
+  g.yt = yt;
+  g.status = status;
+  return cuda_status(launch_gemm(g, s, true));
+}
+
+}  // namespace avr
+
+using namespace avr;
+
+extern "C" {
+
+size_t avr_nvfp4_scales_bytes(int64_t rows, int64_t K) {
+  if (rows < 0 || K <= 0 || K % 16) return 0;
+  return scales_bytes(rows, K);
+}
+
+size_t averis_workspace_size(int64_t l, int64_t K, int64_t N) {
+  if (l < 0 || K <= 0 || N < 0) return 0;
+  return ws_layout(l, K, N).total;
+}
+
+avr_status averis_workspace_init(void* ws, size_t ws_bytes, avr_stream stream) {
+  if (!ws) return AVR_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, stream));
+}
+
+avr_status averis_check_status(void* ws, avr_stream stream) {
+  if (!ws) return AVR_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return AVR_ERR_CUDA;
+  uint32_t st = 0;
+  if (cudaMemcpy(&st, ws, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return AVR_ERR_CUDA;
+  if (st != 0 && cudaMemset(ws, 0, sizeof(st)) != cudaSuccess) return AVR_ERR_CUDA;
+  return static_cast<avr_status>(st);
+}
+
+const char* averis_status_string(avr_status s) {
+  switch (s) {
+    case AVR_OK: return "ok";
+    case AVR_ERR_INVALID_ARG: return "invalid argument";
+    case AVR_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (need K % 64 == 0, N % 64 == 0, sizes < 2^31)";
+    case AVR_ERR_MISALIGNED: return "misaligned pointer (need 16-byte alignment, 256 for the workspace)";
+    case AVR_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case AVR_ERR_CUDA: return "CUDA error";
+    case AVR_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case AVR_ERR_NONFINITE: return "non-finite input (mean or amax is NaN/Inf)";
+    case AVR_ERR_NO_DEVICE: return "no sm_100 device is current";
+  }
+  return "unknown status";
+}
+
+avr_status averis_split_quant(const void* X, avr_dtype xt, int64_t l, int64_t K, avr_round rm,
+                              uint64_t seed, uint64_t offset, int grad, float* mu,
+                              const avr_nvfp4* mu_q, const avr_nvfp4* xr_q, float* xr_debug,
+                              void* ws, size_t ws_bytes, avr_stream stream) {
+  if (!dtype_ok(xt) || !round_ok(rm)) return AVR_ERR_INVALID_ARG;
+  if (!k_ok(K) || !l_ok(l)) return AVR_ERR_UNSUPPORTED_SHAPE;
+  if (l == 0) return AVR_OK;   // no tokens: nothing is read or written
+  if (!X) return AVR_ERR_INVALID_ARG;
+  AVR_TRY(check_nvfp4(xr_q, l, K));
+  if (mu_q) AVR_TRY(check_nvfp4(mu_q, 1, K));
+  if (!aligned16(X) || !aligned16(mu) || !aligned16(xr_debug)) return AVR_ERR_MISALIGNED;
+  Ws w;
+  AVR_TRY(make_ws(ws, ws_bytes, l, K, 0, &w));
+  AVR_TRY(device_ok());
+  float* mu_buf = mu ? mu : w.at<float>(w.lay.mu);
+  return split_chain(X, xt, l, K, 1, rm, seed, offset, grad ? 3u : 1u, grad ? 4u : 2u, mu_buf, mu_q,
+                     xr_q, xr_debug, nullptr, nullptr, w, stream);
+}
+
+avr_status nvfp4_quant(const void* X, avr_dtype xt, int64_t rows, int64_t K, avr_round rm,
+                       uint64_t seed, uint64_t offset, int grad, const avr_nvfp4* out, void* ws,
+                       size_t ws_bytes, avr_stream stream) {
+  if (!dtype_ok(xt) || !round_ok(rm)) return AVR_ERR_INVALID_ARG;
+  if (!k_ok(K) || !l_ok(rows)) return AVR_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0) return AVR_OK;
+  if (!X) return AVR_ERR_INVALID_ARG;
+  AVR_TRY(check_nvfp4(out, rows, K));
+  if (!aligned16(X)) return AVR_ERR_MISALIGNED;
+  Ws w;
+  AVR_TRY(make_ws(ws, ws_bytes, rows, K, 0, &w));
+  AVR_TRY(device_ok());
+  return split_chain(X, xt, rows, K, 0, rm, seed, offset, grad ? 8u : 7u, 0u, nullptr, nullptr, out,
+                     nullptr, nullptr, nullptr, w, stream);
+}
+
+avr_status averis_quant_weight(const void* W, avr_dtype wt, int64_t m, int64_t n,
+                               const avr_nvfp4* w_fwd, const avr_nvfp4* w_dgrad, void* ws,
+                               size_t ws_bytes, avr_stream stream) {
+  if (!W || !dtype_ok(wt)) return AVR_ERR_INVALID_ARG;
+  if (!k_ok(m) || !k_ok(n) || !n_ok(m) || !n_ok(n)) return AVR_ERR_UNSUPPORTED_SHAPE;
+  AVR_TRY(check_nvfp4(w_fwd, n, m));
+  AVR_TRY(check_nvfp4(w_dgrad, m, n));
+  if (!aligned16(W)) return AVR_ERR_MISALIGNED;
+  Ws w;
+  AVR_TRY(make_ws(ws, ws_bytes, m, n, 0, &w));
+  AVR_TRY(device_ok());
+  // amax of W, then W_bar_dgrad = Q_4(W) along n and W_bar_fwd = Q_4(W^T) along m
+  AVR_TRY(split_chain(W, wt, m, n, 0, AVR_RNE, 0, 0, 6u, 0u, nullptr, nullptr, w_dgrad, nullptr,
+                      nullptr, nullptr, w, stream));
+  QuantTransposedArgs t;
+  t.W = W;
+  t.wt = wt;
+  t.m = m;
+  t.n = n;
+  t.n_tiles = n_tiles(n);
+  t.slot_amax = w.slot_xr();
+  t.codes = w_fwd->codes;
+  t.scales = w_fwd->scales;
+  t.g_dec = w_fwd->g_dec;
+  return cuda_status(launch_quant_transposed(t, stream));
+}
+
+avr_status averis_bias_row(const avr_nvfp4* mu_q, const avr_nvfp4* w_q, float* bias, void* ws,
+                           size_t ws_bytes, avr_stream stream) {
+  if (!mu_q || !w_q || !bias) return AVR_ERR_INVALID_ARG;
+  if (!k_ok(mu_q->K) || !n_ok(w_q->rows)) return AVR_ERR_UNSUPPORTED_SHAPE;
+  AVR_TRY(check_nvfp4(mu_q, 1, mu_q->K));
+  AVR_TRY(check_nvfp4(w_q, w_q->rows, mu_q->K));
+  if (!aligned16(bias)) return AVR_ERR_MISALIGNED;
+  Ws w;
+  AVR_TRY(make_ws(ws, ws_bytes, 0, mu_q->K, 0, &w));
+  AVR_TRY(device_ok());
+  BiasArgs b;
+  b.mu_codes = mu_q->codes;
+  b.mu_scales = mu_q->scales;
+  b.mu_gdec = mu_q->g_dec;
+  b.w_codes = w_q->codes;
+  b.w_scales = w_q->scales;
+  b.w_gdec = w_q->g_dec;
+  b.K = mu_q->K;
+  b.n_out = w_q->rows;
+  b.bias = bias;
+  return cuda_status(launch_bias(b, stream));
+}
+
+avr_status nvfp4_gemm(const avr_nvfp4* a, const avr_nvfp4* b, const float* bias, void* Y,
+                      avr_dtype yt, void* ws, size_t ws_bytes, avr_stream stream) {
+  if (!a || !b || !dtype_ok(yt)) return AVR_ERR_INVALID_ARG;
+  if (!k_ok(a->K) || !l_ok(a->rows) || !n_ok(b->rows)) return AVR_ERR_UNSUPPORTED_SHAPE;
+  if (a->rows == 0) return AVR_OK;
+  if (!Y) return AVR_ERR_INVALID_ARG;
+  AVR_TRY(check_nvfp4(a, a->rows, a->K));
+  AVR_TRY(check_nvfp4(b, b->rows, a->K));
+  if (!aligned16(Y) || !aligned16(bias)) return AVR_ERR_MISALIGNED;
+  Ws w;
+  AVR_TRY(make_ws(ws, ws_bytes, 0, a->K, 0, &w));
+  AVR_TRY(device_ok());
+  return gemm(a, b, bias, Y, yt, w.status(), stream);
+}
+
+static avr_status linear(const void* X, avr_dtype xt, int64_t l, int64_t K, int64_t N,
+                         const avr_nvfp4* wq, int split, avr_round rm, uint64_t seed,
+                         uint64_t offset, uint32_t tag, uint32_t tag_mu, void* Y, avr_dtype yt,
+                         const avr_nvfp4* save_xr, const avr_nvfp4* save_mu, void* ws,
+                         size_t ws_bytes, avr_stream stream) {
+  if (!dtype_ok(xt) || !dtype_ok(yt) || !round_ok(rm)) return AVR_ERR_INVALID_ARG;
+  if (!k_ok(K) || !n_ok(N) || !l_ok(l)) return AVR_ERR_UNSUPPORTED_SHAPE;
+  if (l == 0) return AVR_OK;
+  if (!X || !Y) return AVR_ERR_INVALID_ARG;
+  AVR_TRY(check_nvfp4(wq, N, K));
+  if (save_xr) AVR_TRY(check_nvfp4(save_xr, l, K));
+  if (save_mu) AVR_TRY(check_nvfp4(save_mu, 1, K));
+  if (!aligned16(X) || !aligned16(Y)) return AVR_ERR_MISALIGNED;
+  Ws w;
+  AVR_TRY(make_ws(ws, ws_bytes, l, K, N, &w));
+  AVR_TRY(device_ok());
+  avr_nvfp4 xr_ws = {w.at<uint8_t>(w.lay.xr_codes), w.at<uint8_t>(w.lay.xr_scales),
+                     w.at<float>(w.lay.xr_gdec), l, K};
+  avr_nvfp4 mu_ws = {w.at<uint8_t>(w.lay.mu_codes), w.at<uint8_t>(w.lay.mu_scales),
+                     w.at<float>(w.lay.mu_gdec), 1, K};
+  const avr_nvfp4* xr = save_xr ? save_xr : &xr_ws;
+  const avr_nvfp4* muq = save_mu ? save_mu : &mu_ws;
+  float* bias = split ? w.at<float>(w.lay.bias) : nullptr;
+  AVR_TRY(split_chain(X, xt, l, K, split, rm, seed, offset, tag, tag_mu, w.at<float>(w.lay.mu),
+                      split ? muq : nullptr, xr, nullptr, split ? wq : nullptr, bias, w, stream));
+  return gemm(xr, wq, bias, Y, yt, w.status(), stream);
+}
+
+avr_status averis_linear_fwd(const void* X, avr_dtype xt, int64_t l, int64_t m, int64_t n,
+                             const avr_nvfp4* w_fwd, avr_round rm, uint64_t seed, uint64_t offset,
+                             void* Y, avr_dtype yt, const avr_nvfp4* save_xr,
+                             const avr_nvfp4* save_mu, void* ws, size_t ws_bytes,
+                             avr_stream stream) {
+  return linear(X, xt, l, m, n, w_fwd, 1, rm, seed, offset, 1u, 2u, Y, yt, save_xr, save_mu, ws,
+                ws_bytes, stream);
+}
+
+avr_status averis_linear_dgrad(const void* D, avr_dtype dt, int64_t l, int64_t m, int64_t n,
+                               const avr_nvfp4* w_dgrad, avr_round rm, uint64_t seed,
+                               uint64_t offset, void* dX, avr_dtype xt, void* ws, size_t ws_bytes,
+                               avr_stream stream) {
+  return linear(D, dt, l, n, m, w_dgrad, 1, rm, seed, offset, 3u, 4u, dX, xt, nullptr, nullptr, ws,
+                ws_bytes, stream);
+}
+
+avr_status nvfp4_linear_fwd(const void* X, avr_dtype xt, int64_t l, int64_t m, int64_t n,
+                            const avr_nvfp4* w_fwd, avr_round rm, uint64_t seed, uint64_t offset,
+                            void* Y, avr_dtype yt, void* ws, size_t ws_bytes, avr_stream stream) {
+  return linear(X, xt, l, m, n, w_fwd, 0, rm, seed, offset, 7u, 0u, Y, yt, nullptr, nullptr, ws,
+                ws_bytes, stream);
+}
+
+avr_status nvfp4_linear_dgrad(const void* D, avr_dtype dt, int64_t l, int64_t m, int64_t n,
+                              const avr_nvfp4* w_dgrad, avr_round rm, uint64_t seed,
+                              uint64_t offset, void* dX, avr_dtype xt, void* ws, size_t ws_bytes,
+                              avr_stream stream) {
+  return linear(D, dt, l, n, m, w_dgrad, 0, rm, seed, offset, 8u, 0u, dX, xt, nullptr, nullptr, ws,
+                ws_bytes, stream);
+}
+
+avr_status averis_probe_convert(const float* in, uint8_t* e4m3, uint8_t* e2m1, int64_t n,
+                                avr_stream stream) {
+  if (!in || n < 0) return AVR_ERR_INVALID_ARG;
+  if (n == 0) return AVR_OK;
+  AVR_TRY(device_ok());
+  return cuda_status(launch_probe_convert(in, e4m3, e2m1, n, stream));
+}
+
+avr_status averis_probe_philox(uint64_t seed, uint64_t offset, uint32_t tag, int64_t n,
+                               uint32_t* out, avr_stream stream) {
+  if (!out || n < 0) return AVR_ERR_INVALID_ARG;
+  if (!aligned16(out)) return AVR_ERR_MISALIGNED;
+  if (n == 0) return AVR_OK;
+  AVR_TRY(device_ok());
+  return cuda_status(launch_probe_philox(seed, offset, tag, n, out, stream));
+}
+
+}  // extern "C"

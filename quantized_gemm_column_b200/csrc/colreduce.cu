@@ -1,0 +1,183 @@
+// K1: deterministic column reduce -- the "reduce" of the Averis split.
+//
+// mu_X = (1/l) 1^T X (Lighthouse review of "The Curse and Blessing of Mean
+// Bias in FP4-Quantized LLM Training", section 二 2.1), computed in a fixed
+// fp32 order so that every run and the CPU oracle give the same bits:
+//   p[c][j] = (((+0 + x[256c][j]) + x[256c+1][j]) + ...)    rows of chunk c in order
+//   S[j]    = (((+0 + p[0][j]) + p[1][j]) + ...)              chunks in order
+//   mu[j]   = S[j] / l                                        IEEE division
+// The same pass keeps the column max and min, so the last CTA of a column tile
+// can also give max_i |fl(x_ij - mu_j)| = max(fl(colmax - mu), fl(mu - colmin))
+// (rounded subtraction is monotone), the amax the residual's tensor scale
+// needs, without a third pass over X.
+//
+// Grid (column tiles of 128, chunks of 256 rows).  One TMA copy brings the
+// 256 x 128 tile into shared memory; thread j then runs the sequential sum of
+// column j over the chunk.  Partials go to the workspace; the CTA that takes
+// the last ticket of its column tile (atomicInc wraps the ticket back to 0)
+// sums the partials in chunk order and writes mu and the tile's amax slots.
+#include "device.cuh"
+#include "internal.h"
+
+namespace avr {
+
+struct ColReduceParams {
+  int64_t l, K;
+  int C;                  // chunks
+  int split;
+  float* part;            // [3][C][K]: sum, max, min
+  uint32_t* tickets;      // [T]
+  float* slot_xr;         // [T] max |X_R| (split) or max |X| (vanilla)
+  float* slot_mu;         // [T] max |mu|
+  float* mu_out;          // [K]
+  uint32_t* status;
+};
+
+template <bool kBf16>
+__global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_constant__ CUtensorMap map,
+                                                             const ColReduceParams p) {
+  extern __shared__ __align__(1024) uint8_t tile[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t s_last, s_ok;
+  __shared__ float s_red[2][kColTile / 32];
+
+  const int tid = threadIdx.x;
+  const int t = blockIdx.x;
+  const int c = blockIdx.y;
+  const int64_t col = static_cast<int64_t>(t) * kColTile + tid;
+  const int64_t row0 = static_cast<int64_t>(c) * kChunkRows;
+  const int rows = static_cast<int>(min64(kChunkRows, p.l - row0));
+  constexpr uint32_t kElem = kBf16 ? 2u : 4u;
+  constexpr uint32_t kTileBytes = kChunkRows * kColTile * kElem;
+
+  if (tid == 0) {
+    prefetch_tensormap(&map);
+    mbar_init(&bar, 1);
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  pdl_wait_prior_grid();
+  pdl_allow_next_grid();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bar, kTileBytes);
+    tma_load_2d(tile, &map, &bar, t * kColTile, static_cast<int32_t>(row0));
+    s_ok = mbar_wait(&bar, 0, p.status) ? 1u : 0u;
+    if (!s_ok) mbar_wait(&bar, 0, nullptr);   // a second bounded wait for the copy in flight
+  }
+  __syncthreads();
+  if (!s_ok) return;
+
+  // Sequential fp32 sum of this column over the chunk, plus max and min.
+  if (col < p.K) {
+    float s = 0.0f, mx = -INFINITY, mn = INFINITY;
+    if (kBf16) {
+      const uint16_t* v = reinterpret_cast<const uint16_t*>(tile) + tid;
+#pragma unroll 8
+      for (int i = 0; i < rows; ++i) {
+        const float x = __uint_as_float(static_cast<uint32_t>(v[i * kColTile]) << 16);
+        s = __fadd_rn(s, x);
+        mx = fmaxf(mx, x);
+        mn = fminf(mn, x);
+      }
+    } else {
+      const float* v = reinterpret_cast<const float*>(tile) + tid;
+#pragma unroll 8
+      for (int i = 0; i < rows; ++i) {
+        const float x = v[i * kColTile];
+        s = __fadd_rn(s, x);
+        mx = fmaxf(mx, x);
+        mn = fminf(mn, x);
+      }
+    }
+    const int64_t o = static_cast<int64_t>(c) * p.K + col;
+    const int64_t plane = static_cast<int64_t>(p.C) * p.K;
+    p.part[o] = s;
+    p.part[plane + o] = mx;
+    p.part[2 * plane + o] = mn;
+  }
+
+  // Last CTA of this column tile finalizes it.
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicInc(&p.tickets[t], static_cast<uint32_t>(p.C - 1)) ==
+                          static_cast<uint32_t>(p.C - 1));
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  float a_xr = 0.0f, a_mu = 0.0f;
+  if (col < p.K) {
+    const int64_t plane = static_cast<int64_t>(p.C) * p.K;
+    float S = 0.0f, cmax = -INFINITY, cmin = INFINITY;
+    for (int cc = 0; cc < p.C; ++cc) {
+      const int64_t o = static_cast<int64_t>(cc) * p.K + col;
+      S = __fadd_rn(S, __ldcg(&p.part[o]));
+      cmax = fmaxf(cmax, __ldcg(&p.part[plane + o]));
+      cmin = fminf(cmin, __ldcg(&p.part[2 * plane + o]));
+    }
+    if (!isfinite(S)) raise_status(p.status, AVR_ERR_NONFINITE);
+    if (p.split) {
+      const float mu = __fdiv_rn(S, static_cast<float>(p.l));
+      if (!isfinite(mu)) raise_status(p.status, AVR_ERR_NONFINITE);
+      a_xr = fmaxf(__fsub_rn(cmax, mu), __fsub_rn(mu, cmin));
+      a_mu = fabsf(mu);
+      p.mu_out[col] = mu;
+    } else {
+      a_xr = fmaxf(cmax, -cmin);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a_xr = fmaxf(a_xr, __shfl_xor_sync(0xFFFFFFFFu, a_xr, o));
+    a_mu = fmaxf(a_mu, __shfl_xor_sync(0xFFFFFFFFu, a_mu, o));
+  }
+  if ((tid & 31) == 0) {
+    s_red[0][tid >> 5] = a_xr;
+    s_red[1][tid >> 5] = a_mu;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float x = s_red[0][0], m = s_red[1][0];
+#pragma unroll
+    for (int w = 1; w < kColTile / 32; ++w) {
+      x = fmaxf(x, s_red[0][w]);
+      m = fmaxf(m, s_red[1][w]);
+    }
+    p.slot_xr[t] = x;
+    p.slot_mu[t] = m;
+  }
+}
+
+cudaError_t launch_colreduce(const ColReduceArgs& a, cudaStream_t s, bool pdl) {
+  const bool bf16 = a.xt == AVR_BF16;
+  const int elem = bf16 ? 2 : 4;
+  CUtensorMap map;
+  if (!make_tensor_map_2d(&map, a.X, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                          elem, static_cast<uint64_t>(a.l), static_cast<uint64_t>(a.K), kChunkRows,
+                          kColTile, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  ColReduceParams p;
+  p.l = a.l;
+  p.K = a.K;
+  p.C = static_cast<int>((a.l + kChunkRows - 1) / kChunkRows);
+  p.split = a.split;
+  p.part = reinterpret_cast<float*>(a.ws + a.lay->partials);
+  p.tickets = reinterpret_cast<uint32_t*>(a.ws + a.lay->tickets);
+  p.slot_xr = reinterpret_cast<float*>(a.ws + a.lay->slots);
+  p.slot_mu = p.slot_xr + kMaxColTiles;
+  p.mu_out = a.mu_out;
+  p.status = reinterpret_cast<uint32_t*>(a.ws + a.lay->status);
+  const int T = static_cast<int>((a.K + kColTile - 1) / kColTile);
+  const size_t smem = static_cast<size_t>(kChunkRows) * kColTile * elem;
+  dim3 grid(T, p.C);
+  if (bf16) {
+    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(colreduce_kernel<true>), smem);
+    if (e != cudaSuccess) return e;
+    return launch_ex(colreduce_kernel<true>, grid, dim3(kColTile), smem, s, pdl, map, p);
+  }
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(colreduce_kernel<false>), smem);
+  if (e != cudaSuccess) return e;
+  return launch_ex(colreduce_kernel<false>, grid, dim3(kColTile), smem, s, pdl, map, p);
+}
+
+}  // namespace avr

@@ -1,0 +1,155 @@
+// Host-side interface between the C ABI (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/averis.h"
+
+namespace avr {
+
+constexpr int kChunkRows = 256;      // rows per partial of the fixed-order mean
+constexpr int kColTile = 128;        // columns per column-reduce CTA
+constexpr int kMaxColTiles = 4096;   // K <= 524288
+constexpr int kStripCols = 256;      // columns per warp in the quantizer
+
+// Workspace layout (byte offsets, 256-aligned).  The status word and the
+// per-column-tile tickets sit at fixed offsets whatever the sizes, so a
+// workspace can be reused across shapes; everything after them is scratch
+// that each call writes before it reads.
+struct WsLayout {
+  size_t status = 0;
+  size_t tickets = 256;
+  size_t slots = 256 + 4 * kMaxColTiles;           // float[2][kMaxColTiles]
+  size_t partials = 0;                              // float[3][C][K]
+  size_t mu = 0;                                    // float[K]
+  size_t mu_codes = 0, mu_scales = 0, mu_gdec = 0;  // Q_4(mu), 1 x K
+  size_t xr_gdec = 0;
+  size_t bias = 0;                                  // float[N]
+  size_t xr_codes = 0, xr_scales = 0;               // Q_4(X_R), l x K
+  size_t total = 0;
+};
+WsLayout ws_layout(int64_t l, int64_t K, int64_t N);
+
+size_t scales_bytes(int64_t rows, int64_t K);
+
+// ---------------- K1: fixed-order column reduce ----------------
+struct ColReduceArgs {
+  const void* X;
+  avr_dtype xt;
+  int64_t l, K;
+  int split;              // 1: mean + residual amax; 0: amax of X only (vanilla)
+  float* mu_out;          // [K], written when split (nullable otherwise)
+  char* ws;               // workspace base
+  const WsLayout* lay;
+};
+cudaError_t launch_colreduce(const ColReduceArgs& a, cudaStream_t s, bool pdl);
+
+// ---------------- K2: split quantizer (+ mean quantizer, rank-one row) ----------------
+struct QuantArgs {
+  const void* X;
+  avr_dtype xt;
+  int64_t rows, K;
+  const float* mu;          // [K] subtracted from every row; NULL = vanilla
+  int n_tiles;              // column tiles whose amax slots hold max |X_R|
+  const float* slot_xr;     // [n_tiles]
+  uint8_t* codes;
+  uint8_t* scales;
+  float* g_dec;
+  float* xr_debug;          // nullable
+  uint64_t seed, offset;
+  uint32_t tag;
+  int sr;
+  uint32_t* status;
+  // mean quantization and rank-one row (run by extra CTAs when mu != NULL)
+  const float* slot_mu;     // [n_tiles] max |mu| per tile
+  uint32_t tag_mu;
+  uint8_t* mu_codes;        // nullable: where Q_4(mu) is stored
+  uint8_t* mu_scales;
+  float* mu_gdec;
+  const uint8_t* w_codes;   // nullable: no rank-one row
+  const uint8_t* w_scales;
+  const float* w_gdec;
+  int64_t n_out;            // rows of w = entries of bias
+  float* bias;
+};
+cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s, bool pdl);
+
+// Q_4 of T = W^T for W [m, n] (T [n, m], blocks along m), round to nearest even.
+struct QuantTransposedArgs {
+  const void* W;
+  avr_dtype wt;
+  int64_t m, n;
+  int n_tiles;
+  const float* slot_amax;
+  uint8_t* codes;
+  uint8_t* scales;
+  float* g_dec;
+};
+cudaError_t launch_quant_transposed(const QuantTransposedArgs& a, cudaStream_t s);
+
+// rank-one row only
+struct BiasArgs {
+  const uint8_t* mu_codes;
+  const uint8_t* mu_scales;
+  const float* mu_gdec;
+  const uint8_t* w_codes;
+  const uint8_t* w_scales;
+  const float* w_gdec;
+  int64_t K, n_out;
+  float* bias;
+};
+cudaError_t launch_bias(const BiasArgs& a, cudaStream_t s);
+
+// ---------------- K3: tcgen05 block-scaled FP4 GEMM ----------------
+struct GemmArgs {
+  const uint8_t* a_codes;
+  const uint8_t* a_scales;
+  const float* a_gdec;
+  const uint8_t* b_codes;
+  const uint8_t* b_scales;
+  const float* b_gdec;
+  int64_t M, N, K;
+  const float* bias;   // nullable
+  void* Y;
+  avr_dtype yt;
+  uint32_t* status;
+};
+cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, bool pdl);
+
+// ---------------- diagnostics ----------------
+cudaError_t launch_probe_convert(const float* in, uint8_t* e4m3, uint8_t* e2m1, int64_t n,
+                                 cudaStream_t s);
+cudaError_t launch_probe_philox(uint64_t seed, uint64_t offset, uint32_t tag, int64_t n,
+                                uint32_t* out, cudaStream_t s);
+
+// ---------------- tensor maps ----------------
+// 2-D row-major tensor [rows, cols] of elem_bytes-sized elements.
+bool make_tensor_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                        int elem_bytes, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                        uint32_t box_cols, CUtensorMapSwizzle swizzle);
+
+// cudaFuncAttributeMaxDynamicSharedMemorySize for the current device (set
+// once per device and function).
+cudaError_t set_max_dynamic_smem(const void* func, size_t bytes);
+
+// launch with the programmatic-stream-serialization attribute when pdl
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t s, bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+}  // namespace avr

@@ -1,0 +1,140 @@
+"""The tcgen05 block-scaled FP4 GEMM against the oracle's fp64 product."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import nvfp4 as F
+from nvfp4_io import from_oracle, gemm_tolerance, check_bf16_output
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def api():
+    from quantized_gemm_column_b200 import api as a
+    a.load()
+    return a
+
+
+def _rand_q(rng, rows, K, scale_lo=0x28, scale_hi=0x48, g_dec=1.0):
+    codes = rng.integers(0, 16, (rows, K), dtype=np.uint8)
+    sc = rng.integers(scale_lo, scale_hi, (rows, K // 16)).astype(np.uint8)
+    return F.NVFP4(F.pack_codes(codes), sc, np.float32(g_dec), rows, K)
+
+
+def _gemm(api, a_q, b_q, bias=None, out=torch.float32):
+    a, b = from_oracle(a_q, api), from_oracle(b_q, api)
+    Y = torch.empty((a_q.rows, b_q.rows), dtype=out, device="cuda")
+    ws = api.workspace(0, a_q.K)
+    bd = None if bias is None else torch.from_numpy(np.asarray(bias, np.float32)).cuda()
+    api.nvfp4_gemm(a, b, bd, Y, ws)
+    assert api.averis_check_status(ws) == 0
+    return Y.float().cpu().numpy().astype(np.float64)
+
+
+def test_scale_layout_probe_A(api):
+    """A has every code 1.0 and random E4M3 scales; row j of B is 1.0 on the
+    16-block (j mod 4) of a 64-wide K and 0 elsewhere, with scale 1.  Then
+    Y[r, j] = 16 * scale_A[r, j mod 4] exactly: each output names one scale
+    of A, so a wrong tensor-memory scale layout cannot pass."""
+    rng = np.random.default_rng(0)
+    M, K, N = 256, 64, 64
+    a = F.NVFP4(F.pack_codes(np.full((M, K), 2, np.uint8)),
+                rng.integers(0x20, 0x58, (M, K // 16)).astype(np.uint8), np.float32(1.0), M, K)
+    bc = np.zeros((N, K), np.uint8)
+    for j in range(N):
+        bc[j, 16 * (j % 4):16 * (j % 4) + 16] = 2
+    b = F.NVFP4(F.pack_codes(bc), np.full((N, K // 16), 0x38, np.uint8), np.float32(1.0), N, K)
+    Y = _gemm(api, a, b)
+    want = 16.0 * oracle.e4m3_value(a.scales).astype(np.float64)[:, np.arange(N) % 4]
+    assert np.array_equal(Y, want)
+
+
+def test_scale_layout_probe_B(api):
+    """The same with the roles swapped: Y[i, j] = 16 * scale_B[j, i mod 4]
+    for N = 256 (two 128-row scale atoms of B)."""
+    rng = np.random.default_rng(1)
+    M, K, N = 128, 64, 256
+    ac = np.zeros((M, K), np.uint8)
+    for i in range(M):
+        ac[i, 16 * (i % 4):16 * (i % 4) + 16] = 2
+    a = F.NVFP4(F.pack_codes(ac), np.full((M, K // 16), 0x38, np.uint8), np.float32(1.0), M, K)
+    b = F.NVFP4(F.pack_codes(np.full((N, K), 2, np.uint8)),
+                rng.integers(0x20, 0x58, (N, K // 16)).astype(np.uint8), np.float32(1.0), N, K)
+    Y = _gemm(api, a, b)
+    want = 16.0 * oracle.e4m3_value(b.scales).astype(np.float64)[:, np.arange(M) % 4].T
+    assert np.array_equal(Y, want)
+
+
+def test_nibble_order_probe(api):
+    """Row j of B is one-hot at element j: Y[r, j] = value of A's element
+    (r, j), so a swapped nibble order shows at every odd j."""
+    rng = np.random.default_rng(2)
+    M, K = 128, 64
+    ac = rng.integers(0, 16, (M, K)).astype(np.uint8)
+    a = F.NVFP4(F.pack_codes(ac), np.full((M, K // 16), 0x38, np.uint8), np.float32(1.0), M, K)
+    bc = np.zeros((K, K), np.uint8)
+    bc[np.arange(K), np.arange(K)] = 2
+    b = F.NVFP4(F.pack_codes(bc), np.full((K, K // 16), 0x38, np.uint8), np.float32(1.0), K, K)
+    Y = _gemm(api, a, b)
+    assert np.array_equal(Y, oracle.e2m1_value(ac).astype(np.float64))
+
+
+def test_k_stage_and_kblock_order(api):
+    """One-hot 64-element k-blocks across several 256-element stages: row j of
+    B selects k-block j, so Y[:, j] = 64 * scale_A[:, 4j..4j+3] mean... each
+    k-block of A holds a distinct constant, which pins the k advance inside a
+    stage and across stages (K = 640 has a partial last stage)."""
+    rng = np.random.default_rng(3)
+    M, K = 128, 640
+    nkb = K // 64
+    ac = np.zeros((M, K), np.uint8)
+    for kb in range(nkb):
+        ac[:, 64 * kb:64 * kb + 64] = rng.integers(1, 8, (M, 1))
+    a = F.NVFP4(F.pack_codes(ac), np.full((M, K // 16), 0x38, np.uint8), np.float32(1.0), M, K)
+    N = 64
+    bc = np.zeros((N, K), np.uint8)
+    for j in range(N):
+        kb = j % nkb
+        bc[j, 64 * kb:64 * kb + 64] = 2
+    b = F.NVFP4(F.pack_codes(bc), np.full((N, K // 16), 0x38, np.uint8), np.float32(1.0), N, K)
+    Y = _gemm(api, a, b)
+    assert np.array_equal(Y, oracle.gemm_reference(a, b))
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 128, 64), (256, 256, 256), (300, 192, 320),
+                                   (1024, 512, 1024), (129, 64, 2048)])
+def test_random_gemm_fp32_out(api, M, N, K):
+    rng = np.random.default_rng(M + N + K)
+    a = _rand_q(rng, M, K, g_dec=0.013)
+    b = _rand_q(rng, N, K, g_dec=0.002)
+    bias = rng.standard_normal(N)
+    Y = _gemm(api, a, b, bias)
+    ref = oracle.gemm_reference(a, b, bias)
+    rel = np.linalg.norm(Y - ref) / np.linalg.norm(ref)
+    assert rel <= 1e-5, rel
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 256, 256), (300, 192, 320), (2048, 1024, 4096)])
+def test_random_gemm_bf16_out(api, M, N, K):
+    rng = np.random.default_rng(M * 7 + N + K)
+    a = _rand_q(rng, M, K, g_dec=0.01)
+    b = _rand_q(rng, N, K, g_dec=0.003)
+    bias = rng.standard_normal(N) * 0.1
+    Y = _gemm(api, a, b, bias, out=torch.bfloat16)
+    ref = oracle.gemm_reference(a, b, bias)
+    check_bf16_output(Y, ref, gemm_tolerance(a, b, bias, K))
+
+
+def test_quantized_operands_from_oracle(api):
+    """Operands produced by the oracle's quantizer (realistic scale mix)."""
+    rng = np.random.default_rng(4)
+    X = (rng.standard_normal((512, 1024)) * 2 + 1).astype(np.float32)
+    W = rng.standard_normal((768, 1024)).astype(np.float32)
+    a = oracle.nvfp4_quantize(X, "sr", seed=3, tag=1)
+    b = oracle.nvfp4_quantize(W, "rne")
+    Y = _gemm(api, a, b)
+    ref = oracle.gemm_reference(a, b)
+    assert np.linalg.norm(Y - ref) / np.linalg.norm(ref) <= 1e-5

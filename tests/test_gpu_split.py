@@ -1,0 +1,159 @@
+"""Column reduce and split quantizer on the GPU, bit-exact against the
+oracle (mu, X_R, codes, scales, decode scales)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_gemm_column_b200 import inputs
+from nvfp4_io import assert_nvfp4_equal
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def api():
+    from quantized_gemm_column_b200 import api as a
+    a.load()
+    return a
+
+
+def _x(l, K, dtype, seed=0, mean_scale=1.0):
+    rng = inputs.rng_for(50, seed)
+    X = inputs.spiked_activations(rng, l, K, rank=2, s=(8.0, 4.0), n_hot=max(1, K // 100),
+                                  mean_scale=mean_scale)
+    if dtype == "bf16":
+        t = inputs.to_bf16(X)
+        return t.cuda(), inputs.bf16_as_f32(t)
+    x = inputs.to_f32(X)
+    return torch.from_numpy(x).cuda(), x
+
+
+def _split(api, Xd, rm, seed=7, offset=0, grad=False):
+    l, K = Xd.shape
+    mu = torch.empty(K, dtype=torch.float32, device="cuda")
+    mu_q = api.NVFP4Tensor(1, K)
+    xr_q = api.NVFP4Tensor(l, K)
+    xr = torch.empty((l, K), dtype=torch.float32, device="cuda")
+    ws = api.workspace(l, K)
+    api.averis_split_quant(Xd, rm, seed, offset, grad, mu, mu_q, xr_q, xr, ws)
+    assert api.averis_check_status(ws) == 0
+    return mu, mu_q, xr_q, xr
+
+
+SHAPES = [(256, 128, "f32"), (300, 192, "bf16"), (1024, 1024, "bf16"), (4133, 640, "bf16"),
+          (512, 6144, "bf16"), (64, 64, "f32"), (1, 256, "bf16")]
+
+
+@pytest.mark.parametrize("l,K,dt", SHAPES)
+@pytest.mark.parametrize("rm", ["rne", "sr"])
+def test_split_quant_bit_exact(api, l, K, dt, rm):
+    Xd, x = _x(l, K, dt, seed=l + K)
+    mu, mu_q, xr_q, xr = _split(api, Xd, rm, seed=1234 + l, offset=99)
+    rmu, rxr, rmu_q, rxr_q = oracle.averis_split_quant(x, rm, seed=1234 + l, offset=99)
+    assert np.array_equal(mu.cpu().numpy().view(np.uint32), rmu.view(np.uint32))
+    assert np.array_equal(xr.cpu().numpy().view(np.uint32), rxr.view(np.uint32))
+    assert_nvfp4_equal(xr_q, rxr_q, "X_bar_R")
+    assert_nvfp4_equal(mu_q, rmu_q, "mu_bar")
+
+
+def test_grad_tags(api):
+    Xd, x = _x(512, 256, "bf16", seed=3)
+    _, mu_q, xr_q, _ = _split(api, Xd, "sr", seed=5, grad=True)
+    _, _, rmu_q, rxr_q = oracle.averis_split_quant(x, "sr", seed=5, grad=True)
+    assert_nvfp4_equal(xr_q, rxr_q, "D_bar_R")
+    assert_nvfp4_equal(mu_q, rmu_q, "mu_bar_D")
+
+
+def test_order_pins_on_device(api):
+    """The oracle's order pins hold on the device: [2^24, 1, ..., 1] keeps
+    2^24 inside a chunk and across chunks."""
+    X = np.zeros((1024, 64), dtype=np.float32)
+    X[0, 0] = 2.0 ** 24
+    X[1:256, 0] = 1.0
+    X[0, 1] = 2.0 ** 24
+    X[256, 1] = X[512, 1] = X[768, 1] = 1.0
+    mu, _, _, _ = _split(api, torch.from_numpy(X).cuda(), "rne")
+    m = mu.cpu().numpy()
+    assert m[0] == np.float32(2.0 ** 24 / 1024) and m[1] == np.float32(2.0 ** 24 / 1024)
+
+
+def test_constant_columns(api):
+    rng = np.random.default_rng(1)
+    c = inputs.bf16_as_f32(inputs.to_bf16(rng.standard_normal(128) * 10))
+    X = np.repeat(c[None, :], 2048, axis=0)
+    mu, _, xr_q, xr = _split(api, torch.from_numpy(X).to(torch.bfloat16).cuda(), "sr")
+    assert np.array_equal(mu.cpu().numpy(), c)
+    assert not xr.cpu().numpy().any()
+    assert not xr_q.codes.cpu().numpy().any() and xr_q.g_dec.item() == 1.0
+
+
+@pytest.mark.parametrize("rm", ["rne", "sr"])
+def test_vanilla_quant_bit_exact(api, rm):
+    Xd, x = _x(700, 384, "bf16", seed=9)
+    q = api.NVFP4Tensor(700, 384)
+    ws = api.workspace(700, 384)
+    api.nvfp4_quant(Xd, rm, 77, 3, False, q, ws)
+    assert api.averis_check_status(ws) == 0
+    assert_nvfp4_equal(q, oracle.vanilla_quant(x, rm, 77, 3), "Q_4(X)")
+
+
+@pytest.mark.parametrize("m,n,dt", [(128, 256, "f32"), (1024, 4096, "bf16"), (192, 320, "bf16")])
+def test_weight_quant_bit_exact(api, m, n, dt):
+    rng = inputs.rng_for(51, m + n)
+    W = inputs.weight(rng, m, n)
+    if dt == "bf16":
+        Wt = inputs.to_bf16(W)
+        w = inputs.bf16_as_f32(Wt)
+        Wd = Wt.cuda()
+    else:
+        w = inputs.to_f32(W)
+        Wd = torch.from_numpy(w).cuda()
+    w_fwd, w_dgrad = api.NVFP4Tensor(n, m), api.NVFP4Tensor(m, n)
+    ws = api.workspace(m, n)
+    api.averis_quant_weight(Wd, w_fwd, w_dgrad, ws)
+    assert api.averis_check_status(ws) == 0
+    r_fwd, r_dgrad = oracle.quant_weight(w)
+    assert_nvfp4_equal(w_fwd, r_fwd, "W_bar fwd")
+    assert_nvfp4_equal(w_dgrad, r_dgrad, "W_bar dgrad")
+
+
+def test_nonfinite_input_sets_status(api):
+    X = torch.ones((256, 64), dtype=torch.bfloat16, device="cuda")
+    X[17, 5] = float("nan")
+    mu = torch.empty(64, dtype=torch.float32, device="cuda")
+    xr_q = api.NVFP4Tensor(256, 64)
+    ws = api.workspace(256, 64)
+    api.averis_split_quant(X, "rne", 0, 0, False, mu, None, xr_q, None, ws)
+    assert api.averis_check_status(ws) == api.AVR_ERR_NONFINITE
+    assert api.averis_check_status(ws) == 0       # cleared by the read
+
+
+def test_empty_input_is_a_no_op(api):
+    X = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    mu = torch.full((128,), 3.0, device="cuda")
+    xr_q = api.NVFP4Tensor(0, 128)
+    ws = api.workspace(0, 128)
+    api.averis_split_quant(X, "sr", 0, 0, False, mu, None, xr_q, None, ws)
+    assert api.averis_check_status(ws) == 0
+    assert torch.all(mu == 3.0)
+
+
+def test_repeat_calls_reuse_workspace(api):
+    """Tickets wrap back to zero, so one workspace serves many calls and
+    shapes in a row with identical results."""
+    ws = api.workspace(4096, 1024)
+    Xd, x = _x(1024, 512, "bf16", seed=21)
+    outs = []
+    for _ in range(3):
+        mu = torch.empty(512, device="cuda")
+        q = api.NVFP4Tensor(1024, 512)
+        api.averis_split_quant(Xd, "sr", 1, 0, False, mu, None, q, None, ws)
+        outs.append((mu.cpu().numpy(), q.codes.cpu().numpy()))
+        Yd, _ = _x(4096, 1024, "bf16", seed=22)
+        api.averis_split_quant(Yd, "rne", 1, 0, False, torch.empty(1024, device="cuda"), None,
+                               api.NVFP4Tensor(4096, 1024), None, ws)
+    assert api.averis_check_status(ws) == 0
+    for o in outs[1:]:
+        assert np.array_equal(o[0], outs[0][0]) and np.array_equal(o[1], outs[0][1])
