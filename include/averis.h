@@ -130,6 +130,34 @@ avr_status averis_split_quant(const void* X, avr_dtype xt, int64_t l, int64_t K,
                               const avr_nvfp4* mu_q, const avr_nvfp4* xr_q, float* xr_debug,
                               void* ws, size_t ws_bytes, avr_stream stream);
 
+/* averis_split_quant for callers that cannot allocate.  The paper has no
+ * counterpart to this entry point; it exists for the library's users.
+ *
+ * Some callers have no device memory to give the library: a plugin that
+ * receives only its input and output pointers from a framework that owns
+ * every allocation, or latency-critical code that must not call
+ * cudaMalloc/cudaFree (they synchronize the device).  This call takes no
+ * workspace: the column reduce's scratch lives in a fixed 4 MiB array inside
+ * the library, which every GPU that loads the library holds until the
+ * process exits.  It computes exactly what averis_split_quant computes, with
+ * the same arguments except `ws`/`ws_bytes`.
+ *   Limit: 3 * ceil(l/256) * K * 4 bytes of chunk partials plus K * 4 bytes
+ *   for the mean and 48.25 KiB of bookkeeping must fit in 4 MiB, so K can be
+ *   at most 10624 for l = 8192 and at most 2688 for l = 32768; larger sizes
+ *   return AVR_ERR_WORKSPACE_TOO_SMALL without launching anything.
+ *   device_status: nullable device pointer to a uint32 the caller has set to
+ *   0; the first device-side error of the call (AVR_ERR_NONFINITE,
+ *   AVR_ERR_DEVICE_TIMEOUT) is stored there.
+ *   The first call on each device looks up the array's device address (with
+ *   that device current) and keeps it; make that first call before any
+ *   stream capture.  Every call shares the array, so calls that may overlap
+ *   on the GPU (other streams, other threads) race: issue them in one stream
+ *   order.  Each call clears the parts of the array that must start at zero. */
+avr_status averis_split_quant_noalloc(const void* X, avr_dtype xt, int64_t l, int64_t K,
+                                      avr_round rm, uint64_t seed, uint64_t offset, int grad,
+                                      float* mu, const avr_nvfp4* mu_q, const avr_nvfp4* xr_q,
+                                      float* xr_debug, uint32_t* device_status, avr_stream stream);
+
 /* Vanilla NVFP4 quantization of X [rows, K] (no split; [R3.1] "Vanilla FP4").
  * grad selects stream tag 7 (0) or 8 (1). */
 avr_status nvfp4_quant(const void* X, avr_dtype xt, int64_t rows, int64_t K, avr_round rm,

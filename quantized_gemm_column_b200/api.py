@@ -254,3 +254,23 @@ def averis_probe_convert(x, e4m3, e2m1, stream=None):
 def averis_probe_philox(seed, offset, tag, n, out, stream=None):
     _check(load().averis_probe_philox(seed, offset, tag, n, _ptr(out), _stream(stream)),
            "averis_probe_philox")
+
+
+# ---------------------------------------------------------------------------
+# split quantization without a caller workspace
+# ---------------------------------------------------------------------------
+_SIGS["averis_split_quant_noalloc"] = (
+    _c_int, [_c_ptr, _c_int, _c_i64, _c_i64, _c_int, _c_u64, _c_u64, _c_int, _c_ptr,
+             ctypes.POINTER(avr_nvfp4), ctypes.POINTER(avr_nvfp4), _c_ptr, _c_ptr, _c_ptr])
+
+
+def averis_split_quant_noalloc(X, rm, seed, offset, grad, mu, mu_q, xr_q, xr_debug,
+                               device_status=None, stream=None):
+    """averis_split_quant without a workspace, for callers that cannot
+    allocate device memory; its scratch is a fixed 4 MiB array inside the
+    library (see include/averis.h for the size limit and the rules)."""
+    l, K = X.shape
+    _check(load().averis_split_quant_noalloc(_ptr(X), _dtype(X), l, K, _round(rm), seed, offset,
+                                             int(grad), _ptr(mu), _s(mu_q), _s(xr_q), _ptr(xr_debug),
+                                             _ptr(device_status), _stream(stream)),
+           "averis_split_quant_noalloc")
