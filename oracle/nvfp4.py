@@ -76,12 +76,16 @@ def e2m1_rne(y):
 
 
 def e2m1_sr(y, r16):
-    """Stochastic rounding of fp32 values to E2M1 with 16 random bits each.
+    """Stochastic rounding of fp32 values to E2M1 with a 16-bit random value
+    each (add-and-carry):
 
-    a = min(|y|, 6); lo = largest grid value <= a; h = the next grid value;
-    p = (a - lo) / (h - lo), exact in fp32 (a - lo is exact because lo = 0 or
-    lo <= a < 2 lo, and h - lo is a power of two); round up iff
-    float(r16) < p * 65536.  The sign is kept, also on zero.
+    a = min(|y|, 6); lo <= a < h are its grid neighbours; F = floor of the
+    position of a in [lo, h) scaled to 16 bits, floor((a - lo) / (h - lo) *
+    65536) (exact in fp32: a - lo is exact because lo = 0 or lo <= a < 2 lo,
+    h - lo and 65536 are powers of two); round up iff F + r16 >= 65536, i.e.
+    the random value added to the 16 bits below the kept precision carries.
+    The sign is kept, also on zero.  P(up) = F / 65536, so the rounding is
+    unbiased to within 2^-16 of a grid step.
     """
     y = _f32(y)
     a = np.minimum(np.abs(y), E2M1_MAX)
@@ -89,8 +93,8 @@ def e2m1_sr(y, r16):
     lo = E2M1_GRID[idx]
     hi = E2M1_GRID[np.minimum(idx + 1, 7)]
     step = np.where(idx == 7, np.float32(1.0), hi - lo).astype(np.float32)
-    p = ((a - lo) / step).astype(np.float32)
-    up = np.asarray(r16, dtype=np.uint32).astype(np.float32) < p * np.float32(65536.0)
+    F = np.floor(((a - lo) / step).astype(np.float32) * np.float32(65536.0)).astype(np.int64)
+    up = (F + np.asarray(r16, dtype=np.int64)) >= 65536
     code = (idx + (up & (idx < 7))).astype(np.uint8)
     sign = np.signbit(y).astype(np.uint8) << 3
     return (code | sign).astype(np.uint8)

@@ -48,6 +48,32 @@ def test_conversions_match_oracle(api):
     assert bad2.size == 0, f"E2M1: {bad2.size} differ, e.g. x={x[bad2[:4]]} gpu={g2[bad2[:4]]} ref={r2[bad2[:4]]}"
 
 
+def test_stochastic_conversion_matches_oracle(api):
+    """Every (sign, exponent, top-12-mantissa-bit) class in [2^-20, 8) x 3
+    random words (zero, all ones, random), four values per word: the device's
+    stochastic rounding gives the oracle's codes."""
+    from oracle.philox import group_values16
+    rng = np.random.default_rng(12)
+    sign = np.arange(2, dtype=np.uint32)[:, None, None]
+    exp = np.arange(107, 130, dtype=np.uint32)[None, :, None]          # 2^-20 .. 8
+    top = np.arange(4096, dtype=np.uint32)[None, None, :]
+    base = ((sign << 31) | (exp << 23) | (top << 11)).ravel()
+    vals = np.concatenate([base | 0, base | 1, base | rng.integers(0, 2048, base.size, dtype=np.uint32)])
+    vals = rng.permutation(vals).view(np.float32)
+    vals = vals[: vals.size // 4 * 4].reshape(-1, 4)
+    for words in (np.zeros(len(vals), np.uint32), np.full(len(vals), 0xFFFFFFFF, np.uint32),
+                  rng.integers(0, 2 ** 32, len(vals), dtype=np.uint64).astype(np.uint32)):
+        xd = torch.from_numpy(np.ascontiguousarray(vals)).cuda()
+        wd = torch.from_numpy(words.view(np.int32)).cuda()
+        out = torch.empty(len(vals), dtype=torch.int16, device="cuda")
+        api.averis_probe_convert_sr(xd, wd, out)
+        got = out.cpu().numpy().view(np.uint16).astype(np.uint32)
+        got = np.stack([(got >> (4 * k)) & 0xF for k in range(4)], axis=1)
+        ref = oracle.e2m1_sr(vals, group_values16(words))
+        bad = np.argwhere(got != ref)
+        assert bad.size == 0, f"{len(bad)} codes differ, e.g. x={vals[tuple(bad[0])]} got={got[tuple(bad[0])]} ref={ref[tuple(bad[0])]}"
+
+
 @pytest.mark.parametrize("seed,offset,tag", [(0, 0, 1), (0xDEADBEEF12345678, (1 << 32) - 5, 4)])
 def test_philox_matches_oracle(api, seed, offset, tag):
     n = 1 << 18

@@ -30,24 +30,27 @@ def test_uniformity_chi_square():
 def test_stream_mapping_properties():
     seed, tag = 0xDEADBEEF12345678, 3
     a = random_bits16(seed, 100, tag, 4096)
-    # advancing the counter offset by one equals skipping 8 elements
-    b = random_bits16(seed, 101, tag, 4096 - 8)
-    assert np.array_equal(a[8:], b)
+    # advancing the counter offset by one equals skipping 16 elements
+    b = random_bits16(seed, 101, tag, 4096 - 16)
+    assert np.array_equal(a[16:], b)
     # starting inside the stream gives the same bits as slicing it
-    c = random_bits16(seed, 100, tag, 100, start=37)
-    assert np.array_equal(a[37:137], c)
-    # 8 consecutive elements use all 128 bits of one call exactly once
+    c = random_bits16(seed, 100, tag, 100, start=36)
+    assert np.array_equal(a[36:136], c)
+    # the 16 elements of one call: each group of 4 rebuilds its output word
+    # from W (elements 0, 1 = W and its bit reversal) and V (elements 2, 3)
     w = philox4x32_10(np.uint64(100), np.uint64(0), np.uint64(tag), np.uint64(0),
                       np.uint64(seed & 0xFFFFFFFF), np.uint64(seed >> 32))
-    halves = sorted(int(x) >> s & 0xFFFF for x in w for s in (0, 16))
-    assert sorted(a[:8].tolist()) == halves
+    for k in range(4):
+        W, Wr, V, Vr = (int(x) for x in a[4 * k:4 * k + 4])
+        assert int(w[k]) == ((V >> 8) << 24) | ((W >> 8) << 16) | ((V & 0xFF) << 8) | (W & 0xFF)
+        assert Wr == int(f"{W:016b}"[::-1], 2) and Vr == int(f"{V:016b}"[::-1], 2)
     # tag, seed and offset each select a different stream
     assert not np.array_equal(a, random_bits16(seed, 100, tag + 1, 4096))
     assert not np.array_equal(a, random_bits16(seed + 1, 100, tag, 4096))
-    assert not np.array_equal(a[:8], a[8:16])
+    assert not np.array_equal(a[:16], a[16:32])
     # 64-bit counter: the high word of the offset is used
-    hi = random_bits16(seed, 100 + (1 << 32), tag, 8)
-    assert not np.array_equal(a[:8], hi)
+    hi = random_bits16(seed, 100 + (1 << 32), tag, 16)
+    assert not np.array_equal(a[:16], hi)
 
 
 def test_sr_is_unbiased_over_seeds():
