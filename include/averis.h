@@ -227,6 +227,12 @@ avr_status nvfp4_linear_dgrad(const void* D, avr_dtype dt, int64_t l, int64_t m,
 avr_status averis_probe_convert(const float* in, uint8_t* e4m3, uint8_t* e2m1, int64_t n,
                                 avr_stream stream);
 
+/* For n groups of four fp32 values in[4i .. 4i+3] and one 32-bit random word
+ * rbits[i] each: out[i] = the four E2M1 codes (element 4i in bits 0..3) that
+ * the quantizer's stochastic rounding gives them. */
+avr_status averis_probe_convert_sr(const float* in, const uint32_t* rbits, uint16_t* out, int64_t n,
+                                   avr_stream stream);
+
 /* out[4*i .. 4*i+3] = Philox4x32-10 words of counter (lo32(offset+i),
  * hi32(offset+i), tag, 0) under key (lo32(seed), hi32(seed)), i < n. */
 avr_status averis_probe_philox(uint64_t seed, uint64_t offset, uint32_t tag, int64_t n,

@@ -78,6 +78,7 @@ _SIGS = {
                                     _c_int, _c_u64, _c_u64, _c_ptr, _c_int, _c_ptr, _c_size, _c_ptr]),
     "averis_probe_convert": (_c_int, [_c_ptr, _c_ptr, _c_ptr, _c_i64, _c_ptr]),
     "averis_probe_philox": (_c_int, [_c_u64, _c_u64, _c_u32, _c_i64, _c_ptr, _c_ptr]),
+    "averis_probe_convert_sr": (_c_int, [_c_ptr, _c_ptr, _c_ptr, _c_i64, _c_ptr]),
 }
 
 
@@ -249,6 +250,11 @@ def nvfp4_linear_dgrad(D, w_dgrad, rm, seed, offset, dX, ws, stream=None):
 def averis_probe_convert(x, e4m3, e2m1, stream=None):
     _check(load().averis_probe_convert(_ptr(x), _ptr(e4m3), _ptr(e2m1), x.numel(), _stream(stream)),
            "averis_probe_convert")
+
+
+def averis_probe_convert_sr(x, rbits, out, stream=None):
+    _check(load().averis_probe_convert_sr(_ptr(x), _ptr(rbits), _ptr(out), rbits.numel(), _stream(stream)),
+           "averis_probe_convert_sr")
 
 
 def averis_probe_philox(seed, offset, tag, n, out, stream=None):

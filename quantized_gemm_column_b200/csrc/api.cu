@@ -2,8 +2,10 @@
 // validation, workspace layout, tensor maps and the launch chains.
 #include <cudaTypedefs.h>
 
+#include <map>
 #include <mutex>
 #include <set>
+#include <tuple>
 #include <utility>
 
 #include "internal.h"
@@ -76,6 +78,27 @@ cudaError_t set_max_dynamic_smem(const void* func, size_t bytes) {
   e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
   if (e == cudaSuccess) done.insert({dev, func});
   return e;
+}
+
+int blocks_per_sm(const void* func, int threads, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, const void*, int, size_t>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  std::lock_guard<std::mutex> g(mu);
+  auto key = std::make_tuple(dev, func, threads, smem);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  int n = 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, func, threads, smem) != cudaSuccess || n < 1) n = 1;
+  cache[key] = n;
+  return n;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
 }
 
 // ---------------------------------------------------------------------------
@@ -414,6 +437,16 @@ avr_status averis_probe_convert(const float* in, uint8_t* e4m3, uint8_t* e2m1, i
   if (n == 0) return AVR_OK;
   AVR_TRY(device_ok());
   return cuda_status(launch_probe_convert(in, e4m3, e2m1, n, stream));
+}
+
+avr_status averis_probe_convert_sr(const float* in, const uint32_t* rbits, uint16_t* out, int64_t n,
+                                   avr_stream stream) {
+  if (!in || !rbits || !out || n < 0) return AVR_ERR_INVALID_ARG;
+  if (!aligned16(in) || (reinterpret_cast<uintptr_t>(rbits) & 3u) || (reinterpret_cast<uintptr_t>(out) & 1u))
+    return AVR_ERR_MISALIGNED;
+  if (n == 0) return AVR_OK;
+  AVR_TRY(device_ok());
+  return cuda_status(launch_probe_convert_sr(in, rbits, out, n, stream));
 }
 
 avr_status averis_probe_philox(uint64_t seed, uint64_t offset, uint32_t tag, int64_t n,

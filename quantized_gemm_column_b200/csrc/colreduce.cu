@@ -105,16 +105,36 @@ __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_consta
   if (!s_last) return;
   __threadfence();
 
+  // Each thread folds its column's chunk partials in chunk order; the loads
+  // of a batch of kBatch chunks (three planes) are all issued before the
+  // first add, so the fold waits for one L2 round trip per batch.
   float a_xr = 0.0f, a_mu = 0.0f;
+  float S = 0.0f, cmax = -INFINITY, cmin = INFINITY;
   if (col < p.K) {
+    constexpr int kBatch = 16;
     const int64_t plane = static_cast<int64_t>(p.C) * p.K;
-    float S = 0.0f, cmax = -INFINITY, cmin = INFINITY;
-    for (int cc = 0; cc < p.C; ++cc) {
-      const int64_t o = static_cast<int64_t>(cc) * p.K + col;
-      S = __fadd_rn(S, __ldcg(&p.part[o]));
-      cmax = fmaxf(cmax, __ldcg(&p.part[plane + o]));
-      cmin = fminf(cmin, __ldcg(&p.part[2 * plane + o]));
+    for (int c0 = 0; c0 < p.C; c0 += kBatch) {
+      float ps[kBatch], px[kBatch], pn[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        if (c0 + u < p.C) {
+          const int64_t o = static_cast<int64_t>(c0 + u) * p.K + col;
+          ps[u] = __ldcg(&p.part[o]);
+          px[u] = __ldcg(&p.part[plane + o]);
+          pn[u] = __ldcg(&p.part[2 * plane + o]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        if (c0 + u < p.C) {
+          S = __fadd_rn(S, ps[u]);
+          cmax = fmaxf(cmax, px[u]);
+          cmin = fminf(cmin, pn[u]);
+        }
+      }
     }
+  }
+  if (col < p.K) {
     if (!isfinite(S)) raise_status(p.status, AVR_ERR_NONFINITE);
     if (p.split) {
       const float mu = __fdiv_rn(S, static_cast<float>(p.l));

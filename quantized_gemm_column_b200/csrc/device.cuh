@@ -60,6 +60,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -108,6 +112,38 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// TMA tensor store shared -> global (bulk-group completion) and its waits.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_group_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Named barrier over `count` threads; returns the OR of `pred` over them.
+__device__ __forceinline__ bool named_barrier_or(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r) : "r"(pred ? 1u : 0u), "r"(id), "r"(count) : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void named_barrier(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -201,6 +237,7 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
 }
 constexpr uint32_t kLayoutSwizzleNone = 0;
 constexpr uint32_t kLayoutSwizzle128B = 2;
+constexpr uint32_t kLayoutSwizzle64B = 4;
 
 // ---------------------------------------------------------------------------
 // Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11)
@@ -217,8 +254,9 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
   return c;
 }
 
-// The 128 random bits shared by the 8 elements e with floor(e/8) = blk:
-// counter (lo32(offset+blk), hi32(offset+blk), tag, 0), key (lo32(seed), hi32(seed)).
+// The 128 random bits of the 16 elements e with floor(e/16) = blk (word k
+// for elements 16 blk + 4k .. 16 blk + 4k + 3): counter (lo32(offset+blk),
+// hi32(offset+blk), tag, 0), key (lo32(seed), hi32(seed)).
 __device__ __forceinline__ uint4 philox_block(uint64_t seed, uint64_t offset, uint32_t tag,
                                               uint64_t blk) {
   const uint64_t g = offset + blk;
@@ -271,31 +309,20 @@ __device__ __forceinline__ uint32_t e2m1x2_rn(float lo, float hi) {
   return r;
 }
 
-// Stochastic rounding of y to an E2M1 code with 16 random bits r16.
-// Definition: a = min(|y|, 6), lo = largest grid value <= a, h = next one,
-// round up iff r16 < (a - lo) / (h - lo) * 65536.  Integer form used here:
-//   a in [1, 6]:  a = 2^e (1 + f/2^23), e in {0,1,2}; the lower neighbour
-//                 keeps f's top bit, the step is 2^(e-1), and
-//                 (a - lo)/(h - lo) * 65536 = (f mod 2^22) / 64, so
-//                 round up iff (r16 << 6) < (f mod 2^22); code = 2 + 2e + top bit.
-//   a in [.5, 1): (a - .5)/.5 * 65536 = f / 128: round up iff (r16 << 7) < f;
-//                 code 1.
-//   a in [0, .5): (a - 0)/.5 * 65536 = a * 2^17 (exact): code 0.
-__device__ __forceinline__ uint32_t e2m1_sr(float y, uint32_t r16) {
-  const uint32_t sign = (__float_as_uint(y) >> 28) & 8u;
-  const float a = fminf(fabsf(y), 6.0f);
-  const uint32_t b = __float_as_uint(a);
-  uint32_t code;
-  if (a >= 1.0f) {
-    const uint32_t e = (b >> 23) - 127u;
-    const uint32_t base = 2u + 2u * e + ((b >> 22) & 1u);
-    code = base + (((r16 << 6) < (b & 0x3FFFFFu)) ? 1u : 0u);
-  } else if (a >= 0.5f) {
-    code = 1u + (((r16 << 7) < (b & 0x7FFFFFu)) ? 1u : 0u);
-  } else {
-    code = (static_cast<float>(r16) < a * 131072.0f) ? 1u : 0u;
-  }
-  return code | sign;
+// Stochastic rounding of four fp32 values to E2M1 codes (element 0 in bits
+// 0..3 of the result) with one 32-bit random word, by the hardware convert.
+// For each element the fraction of |y| inside its E2M1 interval, truncated to
+// 16 bits, is added to a 16-bit random value and a carry rounds up (|y| > 6
+// saturates to 6; the sign is kept).  The random values the instruction takes
+// from the word (bytes b0..b3): W = b2:b0 for element 0, bitrev16(W) for
+// element 1, V = b3:b1 for element 2 and bitrev16(V) for element 3.  The
+// instruction puts its first operand in the top nibble, so the elements are
+// passed in reverse order.
+__device__ __forceinline__ uint32_t e2m1x4_sr(float e0, float e1, float e2, float e3, uint32_t rbits) {
+  uint16_t r;
+  asm("cvt.rs.satfinite.e2m1x4.f32 %0, {%1, %2, %3, %4}, %5;"
+      : "=h"(r) : "f"(e3), "f"(e2), "f"(e1), "f"(e0), "r"(rbits));
+  return static_cast<uint32_t>(r);
 }
 
 // E2M1 code -> value.  Codes 2..7 are normal: 2^((c>>1) - 1) * (1 + (c&1)/2).

@@ -8,91 +8,127 @@
 // added to every output row:
 //   Y[i, j] = g_dec(A) g_dec(B) * acc[i, j] + bias[j].
 //
-// CTA tile 128 x BN, K staged 256 elements (128 bytes per row) at a time.
-//   warp 0     : TMA producer -- 2-D tensor copies of the A and B code tiles
-//                (128-byte swizzle) and 1-D bulk copies of the matching
-//                512-byte scale atoms, all completing on the stage's mbarrier;
-//   warp 1     : allocates tensor memory; one thread copies the scale atoms
-//                shared -> tensor memory (tcgen05.cp 32x128b, replicated to the
-//                four lane quarters) and issues the
-//                tcgen05.mma.kind::mxf4nvf4.block_scale.block16 instructions
-//                (M 128, N BN, K 64 each), then commits to free the stage;
-//   warps 2..5 : epilogue -- tcgen05.ld of the fp32 accumulator (each warp its
-//                32-lane quarter), scale, add the bias, convert, store.
-// Two CTAs share an SM, so one CTA's epilogue overlaps the other's mainloop.
+// Persistent kernel, one CTA per SM, output tiles handed out round-robin;
+// K staged 256 elements (128 bytes per row, 128-byte swizzle) at a time.
+//   warp 0     : allocates tensor memory; one thread copies the scale atoms
+//                shared -> tensor memory (tcgen05.cp 32x128b, replicated into
+//                the four lane quarters) and issues
+//                tcgen05.mma.kind::mxf4nvf4.block_scale.block16 (M 128, K 64);
+//   warps 1..4 : producers, one TMA operation each per stage -- the A code
+//                tile, the B code tile, and A's and B's 512-byte scale atoms
+//                (2-D copies over the atom array, out-of-range atoms read as
+//                zero).  A thread issues one bulk copy at a time, so the
+//                four copies of a stage go out from four warps;
+//   warps 5..  : epilogue -- tcgen05.ld of the accumulator (each warp one
+//                32-lane quarter and a run of columns), alpha * acc + bias,
+//                convert, write a 128-byte-swizzled staging tile, TMA-store it.
 #include "device.cuh"
 #include "internal.h"
 
 namespace avr {
 
-template <int BN>
+// Two tile shapes:
+//  BN = 256 (bf16 output): MMAs of M 128 x N 256, the shape that reaches the
+//    tensor cores' rate; 3 stages; one accumulator of 256 columns (the scale
+//    buffers take the rest of tensor memory), drained by 8 epilogue warps into
+//    a 64 KB staging tile.
+//  BN = 128 (fp32 output): 4 stages; two accumulators, so the epilogue
+//    overlaps the next tile's mainloop.
+template <int BN, bool kBf16Out>
 struct GemmCfg {
-  static constexpr int kBM = 128;
-  static constexpr int kStages = 3;
+  static constexpr int kBM = 128, kBN = BN;
   static constexpr int kStageK = 256;                      // fp4 elements per stage
+  static constexpr int kRowBytes = kStageK / 2;            // 128 bytes per row
+  static constexpr int kStages = BN == 256 ? 3 : 4;
   static constexpr int kKbPerStage = kStageK / 64;         // MMAs per stage
-  static constexpr int kABytes = kBM * 128;
-  static constexpr int kBBytes = BN * 128;
-  static constexpr int kSfaBytes = kKbPerStage * 512;
-  static constexpr int kSfbBytes = (BN / 128) * kKbPerStage * 512;
+  static constexpr int kAccBufs = BN == 256 ? 1 : 2;
+  static constexpr int kEpiWarps = BN / 32;                // 8 or 4
+  static constexpr int kFirstEpiWarp = 5;
+  static constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
+  static constexpr uint32_t kSwizzle = kLayoutSwizzle128B;
+  static constexpr uint32_t kSbo = 8 * kRowBytes;          // 8-row swizzle atom
+  static constexpr int kABytes = kBM * kRowBytes;
+  static constexpr int kBBytes = kBN * kRowBytes;
+  static constexpr int kSfaBytes = kKbPerStage * 512;      // one 128-row group
+  static constexpr int kSfbBytes = (kBN / 128) * kKbPerStage * 512;
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
-  static constexpr int kBarOffset = kStages * kStageBytes;
-  static constexpr int kSmemBytes = kBarOffset + 256 + 1024;   // + barriers + alignment slack
-  static constexpr int kTmemCols = BN <= 128 ? 256 : 512;
-  static constexpr int kSfaCol = BN;                           // 2 buffers x 16 columns
-  static constexpr int kSfbCol = BN + 2 * kKbPerStage * 4;     // 2 buffers x 4 k-blocks x BN/32
-  static constexpr int kSfbColsPerKb = BN / 32;
-  static_assert(kSfbCol + 2 * kKbPerStage * kSfbColsPerKb <= kTmemCols, "tensor memory budget");
+  static constexpr int kOutElem = kBf16Out ? 2 : 4;
+  static constexpr int kBoxCols = 128 / kOutElem;          // columns per 128-byte swizzled store box
+  static constexpr int kBoxes = kBN / kBoxCols;
+  static constexpr int kStageOutBytes = kBM * kBN * kOutElem;
+  static constexpr int kOutOffset = kStages * kStageBytes;
+  static constexpr int kBarOffset = kOutOffset + kStageOutBytes;
+  // dynamic shared memory starts 1024-aligned when a kernel has no static
+  // shared memory; the kernel checks it and refuses to run otherwise
+  static constexpr int kSmemBytes = kBarOffset + 128;
+  static constexpr int kAccCols = kBN;
+  static constexpr int kSfaCols = kKbPerStage * 4;
+  static constexpr int kSfbCols = kKbPerStage * (kBN / 32);
+  static constexpr int kSfCol = kAccBufs * kAccCols;         // 2 scale buffers after the accumulators
+  static constexpr int kTmemCols = 512;
+  static_assert(kSfCol + 2 * (kSfaCols + kSfbCols) <= kTmemCols, "tensor memory budget");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   // instruction descriptor: E2M1 A and B (format 1), UE4M3 scales, K-major
   // operands, N >> 3 at bit 17, M >> 4 at bit 24
-  static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
+  static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kBN >> 3) << 17) |
                                      (static_cast<uint32_t>(kBM >> 4) << 24);
 };
 
 struct GemmParams {
   int64_t M, N, K;
+  int tiles_n, num_tiles;
   const uint8_t* sfa;
   const uint8_t* sfb;
   const float* gdec_a;
   const float* gdec_b;
   const float* bias;
-  void* Y;
   uint32_t* status;
 };
 
 template <int BN, bool kBf16Out>
-__global__ void __launch_bounds__(192, 1) gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a,
-                                                            const __grid_constant__ CUtensorMap map_b,
-                                                            const GemmParams p) {
-  using Cfg = GemmCfg<BN>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+__global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
+    gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                      const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
+                      const __grid_constant__ CUtensorMap map_y, const GemmParams p) {
+  using Cfg = GemmCfg<BN, kBf16Out>;
+  constexpr int kEpiThreads = 32 * Cfg::kEpiWarps;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {            // the swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) raise_status(p.status, AVR_ERR_MISALIGNED);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint8_t* sA = smem;
   uint8_t* sB = sA + Cfg::kStages * Cfg::kABytes;
   uint8_t* sSfa = sB + Cfg::kStages * Cfg::kBBytes;
   uint8_t* sSfb = sSfa + Cfg::kStages * Cfg::kSfaBytes;
+  uint8_t* sOut = smem + Cfg::kOutOffset;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOffset);
   uint64_t* empty = full + Cfg::kStages;
-  uint64_t* acc_bar = empty + Cfg::kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_bar + 1);
+  uint64_t* acc_full = empty + Cfg::kStages;   // [kAccBufs]
+  uint64_t* acc_empty = acc_full + 2;          // [kAccBufs]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * BN;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * Cfg::kBM;
-  const int n_stages = static_cast<int>((p.K + Cfg::kStageK - 1) / Cfg::kStageK);
-  const uint32_t kb64 = static_cast<uint32_t>(p.K / 64);
+  const int n_kst = static_cast<int>((p.K + Cfg::kStageK - 1) / Cfg::kStageK);
 
   if (threadIdx.x == 0) {
     prefetch_tensormap(&map_a);
     prefetch_tensormap(&map_b);
+    prefetch_tensormap(&map_sfa);
+    prefetch_tensormap(&map_sfb);
+    prefetch_tensormap(&map_y);
     for (int s = 0; s < Cfg::kStages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 4);                  // one arrival per producer warp
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_bar, 1);
+    for (int b = 0; b < Cfg::kAccBufs; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], Cfg::kEpiWarps);   // one arrival per epilogue warp
+    }
     fence_mbarrier_init();
   }
-  if (warp == 1) {
+  if (warp == 0) {
     tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
   }
@@ -103,156 +139,228 @@ __global__ void __launch_bounds__(192, 1) gemm_nvfp4_kernel(const __grid_constan
   pdl_wait_prior_grid();
   pdl_allow_next_grid();
 
-  if (warp == 0) {
+  if (warp >= 1 && warp <= 4) {
     if (lane == 0) {
-      // ---------------- producer ----------------
-      for (int ks = 0; ks < n_stages; ++ks) {
-        const int st = ks % Cfg::kStages;
-        if (ks >= Cfg::kStages &&
-            !mbar_wait(&empty[st], static_cast<uint32_t>((ks / Cfg::kStages) - 1) & 1u, p.status))
-          break;
-        const int nkb = static_cast<int>(min64(Cfg::kKbPerStage, (p.K - static_cast<int64_t>(ks) * Cfg::kStageK) / 64));
-        const uint32_t sf_bytes = static_cast<uint32_t>(nkb) * 512u;
-        mbar_arrive_expect_tx(&full[st], Cfg::kABytes + Cfg::kBBytes + sf_bytes * (1 + BN / 128));
-        tma_load_2d(sA + st * Cfg::kABytes, &map_a, &full[st], ks * 128, static_cast<int32_t>(m0));
-        tma_load_2d(sB + st * Cfg::kBBytes, &map_b, &full[st], ks * 128, static_cast<int32_t>(n0));
-        const uint64_t a_atom = (static_cast<uint64_t>(m0 / 128) * kb64 + static_cast<uint64_t>(ks) * Cfg::kKbPerStage) * 512u;
-        bulk_load(sSfa + st * Cfg::kSfaBytes, p.sfa + a_atom, sf_bytes, &full[st]);
-#pragma unroll
-        for (int g = 0; g < BN / 128; ++g) {
-          const uint64_t b_atom = (static_cast<uint64_t>(n0 / 128 + g) * kb64 + static_cast<uint64_t>(ks) * Cfg::kKbPerStage) * 512u;
-          bulk_load(sSfb + st * Cfg::kSfbBytes + g * Cfg::kKbPerStage * 512, p.sfb + b_atom, sf_bytes, &full[st]);
+      // ---------------- producers: warp 1 A, 2 B, 3 A's scales, 4 B's scales ----------------
+      const int role = warp - 1;
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        const int32_t m0 = (tile / p.tiles_n) * Cfg::kBM;
+        const int32_t n0 = (tile % p.tiles_n) * Cfg::kBN;
+        for (int ks = 0; ks < n_kst; ++ks, ++it) {
+          const int st = it % Cfg::kStages;
+          if (it >= Cfg::kStages &&
+              !mbar_wait(&empty[st], static_cast<uint32_t>((it / Cfg::kStages) - 1) & 1u, p.status)) {
+            ok = false;
+            break;
+          }
+          if (role == 0) {
+            mbar_arrive_expect_tx(&full[st], Cfg::kABytes);
+            tma_load_2d(sA + st * Cfg::kABytes, &map_a, &full[st], ks * Cfg::kRowBytes, m0);
+          } else if (role == 1) {
+            mbar_arrive_expect_tx(&full[st], Cfg::kBBytes);
+            tma_load_2d(sB + st * Cfg::kBBytes, &map_b, &full[st], ks * Cfg::kRowBytes, n0);
+          } else if (role == 2) {
+            // 4 atoms (2 KB) of the tile's 128-row group, as 256 eight-byte elements
+            mbar_arrive_expect_tx(&full[st], Cfg::kSfaBytes);
+            tma_load_2d(sSfa + st * Cfg::kSfaBytes, &map_sfa, &full[st], ks * 256, m0 / 128);
+          } else {
+            mbar_arrive_expect_tx(&full[st], Cfg::kSfbBytes);
+            tma_load_2d(sSfb + st * Cfg::kSfbBytes, &map_sfb, &full[st], ks * 256, n0 / 128);
+          }
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 0) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      for (int ks = 0; ks < n_stages; ++ks) {
-        const int st = ks % Cfg::kStages;
-        if (!mbar_wait(&full[st], static_cast<uint32_t>(ks / Cfg::kStages) & 1u, p.status)) break;
+      int it = 0, tcount = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tcount) {
+        const int ab = tcount % Cfg::kAccBufs;
+        const int use = tcount / Cfg::kAccBufs;
+        if (use >= 1 && !mbar_wait(&acc_empty[ab], static_cast<uint32_t>(use - 1) & 1u, p.status)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const int nkb = static_cast<int>(min64(Cfg::kKbPerStage, (p.K - static_cast<int64_t>(ks) * Cfg::kStageK) / 64));
-        const uint32_t buf = static_cast<uint32_t>(ks & 1);
-        const uint32_t sfa_t = tmem + Cfg::kSfaCol + buf * (Cfg::kKbPerStage * 4);
-        const uint32_t sfb_t = tmem + Cfg::kSfbCol + buf * (Cfg::kKbPerStage * Cfg::kSfbColsPerKb);
-        for (int kb = 0; kb < nkb; ++kb) {
-          tc_cp_32x128b_warpx4(sfa_t + 4 * kb,
-                               smem_desc(smem_u32(sSfa + st * Cfg::kSfaBytes + kb * 512), 0, 128, kLayoutSwizzleNone));
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(ab * Cfg::kAccCols);
+        for (int ks = 0; ks < n_kst; ++ks, ++it) {
+          const int st = it % Cfg::kStages;
+          if (!mbar_wait(&full[st], static_cast<uint32_t>(it / Cfg::kStages) & 1u, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nkb = static_cast<int>(min64(Cfg::kKbPerStage, (p.K - static_cast<int64_t>(ks) * Cfg::kStageK) / 64));
+          const uint32_t buf = static_cast<uint32_t>(it & 1);
+          const uint32_t sfa_t = tmem + Cfg::kSfCol + buf * (Cfg::kSfaCols + Cfg::kSfbCols);
+          const uint32_t sfb_t = sfa_t + Cfg::kSfaCols;
+          for (int kb = 0; kb < nkb; ++kb) {
+            tc_cp_32x128b_warpx4(sfa_t + 4 * kb,
+                                 smem_desc(smem_u32(sSfa + st * Cfg::kSfaBytes + kb * 512), 0, 128, kLayoutSwizzleNone));
 #pragma unroll
-          for (int g = 0; g < BN / 128; ++g)
-            tc_cp_32x128b_warpx4(sfb_t + Cfg::kSfbColsPerKb * kb + 4 * g,
-                                 smem_desc(smem_u32(sSfb + st * Cfg::kSfbBytes + g * Cfg::kKbPerStage * 512 + kb * 512),
-                                           0, 128, kLayoutSwizzleNone));
+            for (int g = 0; g < Cfg::kBN / 128; ++g)
+              tc_cp_32x128b_warpx4(sfb_t + (Cfg::kBN / 32) * kb + 4 * g,
+                                   smem_desc(smem_u32(sSfb + st * Cfg::kSfbBytes + g * Cfg::kKbPerStage * 512 + kb * 512),
+                                             0, 128, kLayoutSwizzleNone));
+          }
+          const uint32_t a_base = smem_u32(sA + st * Cfg::kABytes);
+          const uint32_t b_base = smem_u32(sB + st * Cfg::kBBytes);
+          for (int kb = 0; kb < nkb; ++kb) {
+            const uint64_t adesc = smem_desc(a_base + kb * 32, 16, Cfg::kSbo, Cfg::kSwizzle);
+            const uint64_t bdesc = smem_desc(b_base + kb * 32, 16, Cfg::kSbo, Cfg::kSwizzle);
+            mma_nvf4(d_tmem, adesc, bdesc, Cfg::kIdesc, sfa_t + 4 * kb, sfb_t + (Cfg::kBN / 32) * kb,
+                     (ks > 0 || kb > 0) ? 1u : 0u);
+          }
+          tc_commit(&empty[st]);
         }
-        const uint32_t a_base = smem_u32(sA + st * Cfg::kABytes);
-        const uint32_t b_base = smem_u32(sB + st * Cfg::kBBytes);
-        for (int kb = 0; kb < nkb; ++kb) {
-          const uint64_t adesc = smem_desc(a_base + kb * 32, 16, 1024, kLayoutSwizzle128B);
-          const uint64_t bdesc = smem_desc(b_base + kb * 32, 16, 1024, kLayoutSwizzle128B);
-          mma_nvf4(tmem, adesc, bdesc, Cfg::kIdesc, sfa_t + 4 * kb, sfb_t + Cfg::kSfbColsPerKb * kb,
-                   (ks > 0 || kb > 0) ? 1u : 0u);
-        }
-        tc_commit(&empty[st]);
+        tc_commit(&acc_full[ab]);
       }
-      tc_commit(acc_bar);
     }
   } else {
     // ---------------- epilogue ----------------
-    const int q = warp & 3;
-    const int64_t row = m0 + 32 * q + lane;
-    // warp-uniform, so that the .sync.aligned tensor-memory loads below are
-    // executed by all 32 lanes or by none
-    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_bar, 0u, p.status) ? 1 : 0) != 0;
-    tc_fence_after();
-    if (ok) {
-      const float alpha = __ldg(p.gdec_a) * __ldg(p.gdec_b);
+    const int ew = warp - Cfg::kFirstEpiWarp;  // epilogue warp index
+    const int q = warp & 3;                    // lane quarter of tensor memory this warp may read
+    const int h = ew / 4;                      // which 128-column half (BN = 256)
+    const int r = 32 * q + lane;               // row of the tile
+    const bool leader = (ew == 0 && lane == 0);
+    const float alpha = __ldg(p.gdec_a) * __ldg(p.gdec_b);
+    int tcount = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+      const int ab = tcount % Cfg::kAccBufs;
+      const int64_t m0 = static_cast<int64_t>(tile / p.tiles_n) * Cfg::kBM;
+      const int64_t n0 = static_cast<int64_t>(tile % p.tiles_n) * Cfg::kBN;
+      const bool ok = mbar_wait(&acc_full[ab], static_cast<uint32_t>(tcount / Cfg::kAccBufs) & 1u, p.status);
+      // all epilogue threads agree, so the .sync.aligned loads below run in
+      // every lane of every warp or in none
+      if (named_barrier_or(1, kEpiThreads, !ok)) break;
+      tc_fence_after();
+      // the previous tile's store must have read the staging tile
+      if (leader) bulk_wait_group_read<0>();
+      named_barrier(1, kEpiThreads);
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        const int64_t col = n0 + 32 * c;
-        if (col >= p.N) break;
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(32 * c), r);
+      for (int c = 0; c < 4; ++c) {
+        const int cc = 4 * h + c;              // 32-column chunk of the tile
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) +
+                               static_cast<uint32_t>(ab * Cfg::kAccCols + 32 * cc), v);
         tmem_ld_wait();
         float b[32];
-        if (p.bias) {
+        const int64_t col = n0 + 32 * cc;
+        if (p.bias != nullptr && col < p.N) {
           const float4* bp = reinterpret_cast<const float4*>(p.bias + col);
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const float4 t = __ldg(bp + v);
-            b[4 * v] = t.x; b[4 * v + 1] = t.y; b[4 * v + 2] = t.z; b[4 * v + 3] = t.w;
+          for (int u = 0; u < 8; ++u) {
+            const float4 t = __ldg(bp + u);
+            b[4 * u] = t.x; b[4 * u + 1] = t.y; b[4 * u + 2] = t.z; b[4 * u + 3] = t.w;
           }
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j) b[j] = 0.0f;
         }
-        if (row < p.M) {
-          if (kBf16Out) {
-            uint32_t w[16];
+        if (kBf16Out) {
+          // 32 bf16 = 64 bytes = four 16-byte pieces of row r in box cc/2
+          uint8_t* box = sOut + (cc >> 1) * (Cfg::kBM * 128);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float y0 = fmaf(alpha, __uint_as_float(r[2 * j]), b[2 * j]);
-              const float y1 = fmaf(alpha, __uint_as_float(r[2 * j + 1]), b[2 * j + 1]);
-              const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
-              w[j] = *reinterpret_cast<const uint32_t*>(&h);
+          for (int u = 0; u < 4; ++u) {
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int j = 8 * u + 2 * k;
+              const __nv_bfloat162 pr = __floats2bfloat162_rn(fmaf(alpha, __uint_as_float(v[j]), b[j]),
+                                                              fmaf(alpha, __uint_as_float(v[j + 1]), b[j + 1]));
+              w[k] = *reinterpret_cast<const uint32_t*>(&pr);
             }
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Y) + row * p.N + col);
+            const int piece = ((cc & 1) * 4 + u) ^ (r & 7);
+            *reinterpret_cast<uint4*>(box + r * 128 + piece * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        } else {
+          // 32 fp32 = 128 bytes = one full row of box cc
+          uint8_t* box = sOut + cc * (Cfg::kBM * 128);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-          } else {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.Y) + row * p.N + col);
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(fmaf(alpha, __uint_as_float(r[4 * v]), b[4 * v]),
-                                   fmaf(alpha, __uint_as_float(r[4 * v + 1]), b[4 * v + 1]),
-                                   fmaf(alpha, __uint_as_float(r[4 * v + 2]), b[4 * v + 2]),
-                                   fmaf(alpha, __uint_as_float(r[4 * v + 3]), b[4 * v + 3]));
+          for (int u = 0; u < 8; ++u) {
+            const int j = 4 * u;
+            const float4 f = make_float4(fmaf(alpha, __uint_as_float(v[j]), b[j]),
+                                         fmaf(alpha, __uint_as_float(v[j + 1]), b[j + 1]),
+                                         fmaf(alpha, __uint_as_float(v[j + 2]), b[j + 2]),
+                                         fmaf(alpha, __uint_as_float(v[j + 3]), b[j + 3]));
+            *reinterpret_cast<float4*>(box + r * 128 + ((u ^ (r & 7)) * 16)) = f;
           }
         }
       }
+      // accumulator drained: hand it back to the MMA warp
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      // staging tile complete and visible to the TMA engine: store it
+      fence_proxy_async_smem();
+      named_barrier(1, kEpiThreads);
+      if (leader) {
+#pragma unroll
+        for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+          if (n0 + bx * Cfg::kBoxCols < p.N)
+            tma_store_2d(&map_y, sOut + bx * (Cfg::kBM * 128), static_cast<int32_t>(n0 + bx * Cfg::kBoxCols),
+                         static_cast<int32_t>(m0));
+        bulk_commit_group();
+      }
     }
+    if (leader) bulk_wait_group_all();
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::kTmemCols);
   }
 }
 
 template <int BN, bool kBf16Out>
-static cudaError_t launch_gemm_t(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParams& p,
-                                 cudaStream_t s, bool pdl) {
-  using Cfg = GemmCfg<BN>;
-  auto kern = gemm_nvfp4_kernel<BN, kBf16Out>;
-  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes);
-  if (e != cudaSuccess) return e;
-  dim3 grid(static_cast<unsigned>((p.N + BN - 1) / BN), static_cast<unsigned>((p.M + Cfg::kBM - 1) / Cfg::kBM));
-  return launch_ex(kern, grid, dim3(192), Cfg::kSmemBytes, s, pdl, ma, mb, p);
-}
-
-cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, bool pdl) {
-  constexpr int BN = 128;
-  CUtensorMap ma, mb;
+static cudaError_t launch_gemm_t(const GemmArgs& a, cudaStream_t s, bool pdl) {
+  using Cfg = GemmCfg<BN, kBf16Out>;
+  constexpr CUtensorMapSwizzle kOpSwizzle = CU_TENSOR_MAP_SWIZZLE_128B;
+  CUtensorMap ma, mb, msa, msb, my;
   if (!make_tensor_map_2d(&ma, a.a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(a.M),
-                          static_cast<uint64_t>(a.K / 2), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+                          static_cast<uint64_t>(a.K / 2), Cfg::kBM, Cfg::kRowBytes, kOpSwizzle))
     return cudaErrorInvalidValue;
   if (!make_tensor_map_2d(&mb, a.b_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(a.N),
-                          static_cast<uint64_t>(a.K / 2), BN, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+                          static_cast<uint64_t>(a.K / 2), Cfg::kBN, Cfg::kRowBytes, kOpSwizzle))
+    return cudaErrorInvalidValue;
+  // scale atoms as a [row groups, K/64 * 64] array of 8-byte elements; a box of
+  // 256 elements is the 4 atoms (2 KB) of one stage of one 128-row group
+  const uint64_t sf_cols = static_cast<uint64_t>(a.K / 64) * 64;
+  if (!make_tensor_map_2d(&msa, a.a_scales, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, static_cast<uint64_t>((a.M + 127) / 128),
+                          sf_cols, 1, 256, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  if (!make_tensor_map_2d(&msb, a.b_scales, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, static_cast<uint64_t>((a.N + 127) / 128),
+                          sf_cols, Cfg::kBN / 128, 256, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  if (!make_tensor_map_2d(&my, a.Y, kBf16Out ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                          Cfg::kOutElem, static_cast<uint64_t>(a.M), static_cast<uint64_t>(a.N), Cfg::kBM,
+                          Cfg::kBoxCols, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   GemmParams p;
   p.M = a.M;
   p.N = a.N;
   p.K = a.K;
+  p.tiles_n = static_cast<int>((a.N + Cfg::kBN - 1) / Cfg::kBN);
+  p.num_tiles = static_cast<int>((a.M + Cfg::kBM - 1) / Cfg::kBM) * p.tiles_n;
   p.sfa = a.a_scales;
   p.sfb = a.b_scales;
   p.gdec_a = a.a_gdec;
   p.gdec_b = a.b_gdec;
   p.bias = a.bias;
-  p.Y = a.Y;
   p.status = a.status;
-  return a.yt == AVR_BF16 ? launch_gemm_t<BN, true>(ma, mb, p, s, pdl)
-                          : launch_gemm_t<BN, false>(ma, mb, p, s, pdl);
+  auto kern = gemm_nvfp4_kernel<BN, kBf16Out>;
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
+  return launch_ex(kern, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmemBytes, s, pdl, ma, mb, msa, msb, my, p);
+}
+
+cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, bool pdl) {
+  return a.yt == AVR_BF16 ? launch_gemm_t<256, true>(a, s, pdl) : launch_gemm_t<128, false>(a, s, pdl);
 }
 
 }  // namespace avr

@@ -13,7 +13,7 @@ namespace avr {
 constexpr int kChunkRows = 256;      // rows per partial of the fixed-order mean
 constexpr int kColTile = 128;        // columns per column-reduce CTA
 constexpr int kMaxColTiles = 4096;   // K <= 524288
-constexpr int kStripCols = 256;      // columns per warp in the quantizer
+constexpr int kStripCols = 512;      // columns per warp in the quantizer (16 per lane)
 
 // Workspace layout (byte offsets, 256-aligned).  The status word and the
 // per-column-tile tickets sit at fixed offsets whatever the sizes, so a
@@ -122,6 +122,8 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, bool pdl);
 // ---------------- diagnostics ----------------
 cudaError_t launch_probe_convert(const float* in, uint8_t* e4m3, uint8_t* e2m1, int64_t n,
                                  cudaStream_t s);
+cudaError_t launch_probe_convert_sr(const float* in, const uint32_t* rbits, uint16_t* out, int64_t n,
+                                    cudaStream_t s);
 cudaError_t launch_probe_philox(uint64_t seed, uint64_t offset, uint32_t tag, int64_t n,
                                 uint32_t* out, cudaStream_t s);
 
@@ -134,6 +136,13 @@ bool make_tensor_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType 
 // cudaFuncAttributeMaxDynamicSharedMemorySize for the current device (set
 // once per device and function).
 cudaError_t set_max_dynamic_smem(const void* func, size_t bytes);
+
+// Resident CTAs per SM of `func` with this block size and dynamic shared
+// memory on the current device (cached).
+int blocks_per_sm(const void* func, int threads, size_t smem);
+
+// Streaming multiprocessors of the current device.
+int sm_count();
 
 // launch with the programmatic-stream-serialization attribute when pdl
 template <typename... KArgs, typename... Args>

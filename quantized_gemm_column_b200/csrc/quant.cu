@@ -10,11 +10,12 @@
 // packed two per byte and the scales written straight into the tcgen05
 // 128x4 scale-atom layout, so the GEMM consumes them without any reshuffle.
 //
-// Work split: a warp owns a 256-column strip and walks rows; lane i holds 8
-// consecutive columns (one 16-byte bf16 load), so a lane pair is one block
-// (amax by one shuffle), eight lanes are one 4-scale atom word, and one
-// Philox4x32-10 call gives the 8 x 16 random bits of the lane's elements.
-// Extra CTAs at the end of the grid quantize mu and form the rank-one row
+// Work split: a warp owns a 512-column strip and walks rows; lane i holds one
+// 16-element block (two 16-byte bf16 loads), so the block amax needs no
+// shuffle, four lanes make one 4-scale atom word, one Philox4x32-10 call
+// gives the block's four 32-bit random words, and stochastic rounding is the
+// hardware convert cvt.rs.satfinite.e2m1x4 (four elements per instruction).
+// Every CTA also quantizes mu and forms a share of the rank-one row
 // mu_bar W_bar that the GEMM adds as a bias.
 #include "device.cuh"
 #include "internal.h"
@@ -23,8 +24,9 @@ namespace avr {
 
 constexpr int kQuantThreads = 256;
 constexpr int kQuantWarps = kQuantThreads / 32;
-constexpr int kRowsPerCta = 32;            // rows per CTA (4 per warp)
-constexpr int kBiasRowsPerCta = 64;        // rank-one-row outputs per extra CTA
+constexpr int kRowsPerIter = 2;            // rows a warp computes per iteration (the next ones are in flight)
+constexpr int kBiasRowsPerCta = 32;       // rank-one-row outputs per CTA of the stand-alone kernel
+constexpr int kBiasMaxChunks = 4;          // 32-element chunks per lane in flight (K <= 4096 per pass)
 
 struct QuantParams {
   const void* X;
@@ -40,8 +42,7 @@ struct QuantParams {
   uint32_t tag;
   uint32_t* status;
   int n_strips;
-  int n_quant_ctas;
-  // extra CTAs
+  // mean quantization and rank-one row
   const float* slot_mu;
   uint32_t tag_mu;
   uint8_t* mu_codes;
@@ -62,92 +63,131 @@ __device__ __forceinline__ float max_of_slots(const float* slots, int n) {
   return a;
 }
 
-// Load 8 consecutive elements as fp32.
+// 16 consecutive input elements of one lane, kept as loaded (bf16: two
+// 16-byte words; fp32: four).
 template <bool kBf16>
-__device__ __forceinline__ void load8(const void* base, int64_t idx, bool active, float (&x)[8]) {
+struct Raw16 {
+  uint4 w[kBf16 ? 2 : 4];
+};
+
+template <bool kBf16>
+__device__ __forceinline__ void load16(const void* base, int64_t idx, bool active, Raw16<kBf16>& r) {
+#pragma unroll
+  for (int i = 0; i < (kBf16 ? 2 : 4); ++i) r.w[i] = make_uint4(0, 0, 0, 0);
+  if (!active) return;
+  const uint4* p = kBf16 ? reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + idx)
+                         : reinterpret_cast<const uint4*>(static_cast<const float*>(base) + idx);
+#pragma unroll
+  for (int i = 0; i < (kBf16 ? 2 : 4); ++i) r.w[i] = __ldcs(p + i);
+}
+
+template <bool kBf16>
+__device__ __forceinline__ void unpack16(const Raw16<kBf16>& r, float (&x)[16]) {
   if (kBf16) {
-    uint4 w = make_uint4(0, 0, 0, 0);
-    if (active) w = __ldcs(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + idx));
-    x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x);
-    x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
-    x[4] = bf16_lo(w.z); x[5] = bf16_hi(w.z);
-    x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
-  } else {
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-    if (active) {
-      const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx);
-      a = __ldcs(p);
-      b = __ldcs(p + 1);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint32_t u[4] = {r.w[i].x, r.w[i].y, r.w[i].z, r.w[i].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        x[8 * i + 2 * k] = bf16_lo(u[k]);
+        x[8 * i + 2 * k + 1] = bf16_hi(u[k]);
+      }
     }
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[4 * i] = __uint_as_float(r.w[i].x);
+      x[4 * i + 1] = __uint_as_float(r.w[i].y);
+      x[4 * i + 2] = __uint_as_float(r.w[i].z);
+      x[4 * i + 3] = __uint_as_float(r.w[i].w);
+    }
   }
 }
 
-// Quantize the 8 values of this lane (its lane pair forms one 16-block).
-// Returns the packed codes (8 nibbles) and the block's scale code in *S.
+// r_tab[S] = fl(g_enc / value(S)) for every E4M3 code S (0 for S = 0), one
+// IEEE division per code instead of one per block.
+__device__ __forceinline__ void fill_rscale_table(float* r_tab, float g_enc) {
+  for (int c = threadIdx.x; c < 128; c += blockDim.x)
+    r_tab[c] = (c == 0 || c == 0x7F) ? 0.0f : __fdiv_rn(g_enc, e4m3_value(static_cast<uint32_t>(c)));
+}
+
+// Quantize one 16-element block: returns the 16 packed codes (element 2k in
+// the low nibble of byte k) and the block's E4M3 scale code in *S.
+// `blk` = element index of the block's first element / 16 (its Philox counter).
 template <bool kSR>
-__device__ __forceinline__ uint32_t quant8(const float (&xr)[8], float g_enc, uint64_t seed,
-                                           uint64_t offset, uint32_t tag, uint64_t elem0,
-                                           uint32_t* S_out, float* rscale_out) {
+__device__ __forceinline__ uint2 quant16(const float (&xr)[16], float g_enc, const float* r_tab,
+                                         uint64_t seed, uint64_t offset, uint32_t tag, uint64_t blk,
+                                         uint32_t* S_out) {
   float am = 0.0f;
 #pragma unroll
-  for (int t = 0; t < 8; ++t) am = fmaxf(am, fabsf(xr[t]));
-  am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
+  for (int t = 0; t < 16; ++t) am = fmaxf(am, fabsf(xr[t]));
   const uint32_t S = e4m3_rn_satfinite(__fmul_rn(__fdiv_rn(am, 6.0f), g_enc));
-  const float r = S == 0u ? 0.0f : __fdiv_rn(g_enc, e4m3_value(S));
-  float y[8];
+  const float r = r_tab[S];
+  float y[16];
 #pragma unroll
-  for (int t = 0; t < 8; ++t) y[t] = __fmul_rn(xr[t], r);
-  uint32_t packed = 0;
+  for (int t = 0; t < 16; ++t) y[t] = __fmul_rn(xr[t], r);
+  uint2 packed;
   if (kSR) {
-    const uint4 rnd = philox_block(seed, offset, tag, elem0 >> 3);
-    const uint32_t w[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const uint32_t r16 = (w[t >> 1] >> ((t & 1) * 16)) & 0xFFFFu;
-      packed |= e2m1_sr(y[t], r16) << (4 * t);
-    }
+    const uint4 w = philox_block(seed, offset, tag, blk);
+    packed.x = e2m1x4_sr(y[0], y[1], y[2], y[3], w.x) | (e2m1x4_sr(y[4], y[5], y[6], y[7], w.y) << 16);
+    packed.y = e2m1x4_sr(y[8], y[9], y[10], y[11], w.z) | (e2m1x4_sr(y[12], y[13], y[14], y[15], w.w) << 16);
   } else {
+    uint32_t b[8];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) packed |= e2m1x2_rn(y[2 * k], y[2 * k + 1]) << (8 * k);
+    for (int k = 0; k < 8; ++k) b[k] = e2m1x2_rn(y[2 * k], y[2 * k + 1]);
+    packed.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+    packed.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
   }
   *S_out = S;
-  if (rscale_out) *rscale_out = e4m3_value(S);
   return packed;
 }
 
-// Lane 8q gathers the scale codes of lanes 8q, 8q+2, 8q+4, 8q+6 (four
-// consecutive blocks) into one little-endian word.
+// Lane 4q gathers the scale codes of lanes 4q .. 4q+3 (four consecutive
+// blocks) into one little-endian word.
 __device__ __forceinline__ uint32_t gather_scale_word(uint32_t S) {
-  const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, S, 2);
-  const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, S, 4);
-  const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, S, 6);
+  const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, S, 1);
+  const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, S, 2);
+  const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, S, 3);
   return S | (s1 << 8) | (s2 << 16) | (s3 << 24);
 }
 
-// sum_k mu_val[k] * value(w)[j, k] for the rows j of this warp; mu_val holds
-// e2m1 * e4m3 of mu (tensor scale applied by the caller).
+// bias[j] = g_dec_prod * sum_k mu_val[k] * value(w)[j, k] for the rows j of
+// this warp; mu_val holds e2m1 * e4m3 of mu.  A lane covers 32 consecutive k
+// (16 code bytes and one scale word); up to kBiasMaxChunks such loads per
+// lane are issued before any is used.
 __device__ void bias_rows(const float* s_mu, int64_t K, const uint8_t* w_codes,
                           const uint8_t* w_scales, float g_dec_prod, int64_t j_begin,
-                          int64_t j_end, float* bias) {
+                          int64_t j_end, int64_t j_step, float* bias) {
   const int lane = threadIdx.x & 31;
   const uint32_t n_kb64 = static_cast<uint32_t>(K / 64);
-  for (int64_t j = j_begin; j < j_end; ++j) {
+  for (int64_t j = j_begin; j < j_end; j += j_step) {
     float acc = 0.0f;
-    for (int64_t k0 = static_cast<int64_t>(lane) * 32; k0 < K; k0 += 32 * 32) {
-      const uint4 cw = __ldg(reinterpret_cast<const uint4*>(w_codes + j * (K / 2) + k0 / 2));
-      const uint32_t c16 = static_cast<uint32_t>(k0 / 16);
-      const float s0 = e4m3_value(__ldg(w_scales + scale_offset(j, c16, n_kb64)));
-      const float s1 = e4m3_value(__ldg(w_scales + scale_offset(j, c16 + 1, n_kb64)));
-      const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+    for (int64_t base = 0; base < K; base += 32 * 32 * kBiasMaxChunks) {
+      uint4 cw[kBiasMaxChunks];
+      uint32_t sw[kBiasMaxChunks];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float sc = q < 2 ? s0 : s1;
+      for (int u = 0; u < kBiasMaxChunks; ++u) {
+        const int64_t k0 = base + (static_cast<int64_t>(u) * 32 + lane) * 32;
+        if (k0 < K) {
+          cw[u] = __ldg(reinterpret_cast<const uint4*>(w_codes + j * (K / 2) + k0 / 2));
+          // the two scales of this chunk share one aligned 4-byte word
+          const uint64_t so = scale_offset(static_cast<uint64_t>(j), static_cast<uint32_t>(k0 / 16), n_kb64);
+          sw[u] = __ldg(reinterpret_cast<const uint32_t*>(w_scales + (so & ~uint64_t{3}))) >> (8 * (so & 3u));
+        }
+      }
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const float wv = e2m1_value((words[q] >> (4 * t)) & 0xFu) * sc;
-          acc = fmaf(wv, s_mu[k0 + q * 8 + t], acc);
+      for (int u = 0; u < kBiasMaxChunks; ++u) {
+        const int64_t k0 = base + (static_cast<int64_t>(u) * 32 + lane) * 32;
+        if (k0 < K) {
+          const float s0 = e4m3_value(sw[u] & 0xFFu), s1 = e4m3_value((sw[u] >> 8) & 0xFFu);
+          const uint32_t words[4] = {cw[u].x, cw[u].y, cw[u].z, cw[u].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float sc = q < 2 ? s0 : s1;
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+              acc = fmaf(e2m1_value((words[q] >> (4 * t)) & 0xFu) * sc, s_mu[k0 + q * 8 + t], acc);
+          }
         }
       }
     }
@@ -157,12 +197,15 @@ __device__ void bias_rows(const float* s_mu, int64_t K, const uint8_t* w_codes,
   }
 }
 
+// Q_4(mu) into shared memory (s_mu[k] = e2m1 * e4m3 of mu, the tensor scale
+// left out) by all warps of the CTA; the CTA with `writer` set also stores
+// mu_bar (codes, every scale byte of its 1 x K atom rows, g_dec).
 template <bool kSR>
-__device__ void mean_and_bias_block(const QuantParams& p, int e, float* s_mu) {
+__device__ void quantize_mean(const QuantParams& p, float* s_mu, float* r_tab, bool writer, float* g_dec_mu) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const TensorScale ts = tensor_scale(max_of_slots(p.slot_mu, p.n_tiles));
   const uint32_t n_kb64 = static_cast<uint32_t>(p.K / 64);
-  const bool writer = (e == 0) && p.mu_codes != nullptr;
+  fill_rscale_table(r_tab, ts.g_enc);
   if (writer) {
     if (threadIdx.x == 0) *p.mu_gdec = ts.g_dec;
     // zero the padding rows 1..127 of every scale atom (row 0 is written below)
@@ -171,90 +214,119 @@ __device__ void mean_and_bias_block(const QuantParams& p, int e, float* s_mu) {
     for (int64_t i = threadIdx.x; i < n_words; i += kQuantThreads)
       if ((i & 127) != 0) w[i] = 0u;
   }
+  *g_dec_mu = ts.g_dec;
+  __syncthreads();
   for (int strip = warp; strip < p.n_strips; strip += kQuantWarps) {
-    const int64_t col0 = static_cast<int64_t>(strip) * kStripCols + lane * 8;
+    const int64_t col0 = static_cast<int64_t>(strip) * kStripCols + lane * 16;
     const bool active = col0 < p.K;
-    float x[8];
+    float x[16];
 #pragma unroll
-    for (int t = 0; t < 8; ++t) x[t] = active ? __ldcg(p.mu + col0 + t) : 0.0f;
+    for (int t = 0; t < 16; ++t) x[t] = active ? __ldcg(p.mu + col0 + t) : 0.0f;
     uint32_t S;
-    float sv;
-    const uint32_t packed = quant8<kSR>(x, ts.g_enc, p.seed, p.offset, p.tag_mu,
-                                        static_cast<uint64_t>(col0), &S, &sv);
+    const uint2 packed = quant16<kSR>(x, ts.g_enc, r_tab, p.seed, p.offset, p.tag_mu,
+                                      static_cast<uint64_t>(col0 / 16), &S);
     const uint32_t sw = gather_scale_word(S);
     if (active) {
       if (writer) {
-        *reinterpret_cast<uint32_t*>(p.mu_codes + col0 / 2) = packed;
-        if ((lane & 7) == 0)
+        *reinterpret_cast<uint2*>(p.mu_codes + col0 / 2) = packed;
+        if ((lane & 3) == 0)
           *reinterpret_cast<uint32_t*>(p.mu_scales + scale_offset(0, static_cast<uint32_t>(col0 / 16), n_kb64)) = sw;
       }
+      const float sv = e4m3_value(S);
 #pragma unroll
-      for (int t = 0; t < 8; ++t) s_mu[col0 + t] = e2m1_value((packed >> (4 * t)) & 0xFu) * sv;
+      for (int t = 0; t < 8; ++t) {
+        s_mu[col0 + t] = e2m1_value((packed.x >> (4 * t)) & 0xFu) * sv;
+        s_mu[col0 + 8 + t] = e2m1_value((packed.y >> (4 * t)) & 0xFu) * sv;
+      }
     }
   }
   __syncthreads();
-  if (p.w_codes == nullptr) return;
-  const float gprod = ts.g_dec * __ldg(p.w_gdec);
-  const int64_t j0 = static_cast<int64_t>(e) * kBiasRowsPerCta;
-  const int64_t per_warp = kBiasRowsPerCta / kQuantWarps;
-  const int64_t jb = j0 + warp * per_warp;
-  const int64_t je = min64(jb + per_warp, p.n_out);
-  if (jb < je) bias_rows(s_mu, p.K, p.w_codes, p.w_scales, gprod, jb, je, p.bias);
 }
 
 template <bool kBf16, bool kSR>
 __global__ void __launch_bounds__(kQuantThreads) quant_kernel(const QuantParams p) {
-  extern __shared__ float s_mu[];   // extra CTAs only: dequantized mu (K floats)
+  extern __shared__ float s_mu[];   // dequantized mu (K floats) when the rank-one row is formed
+  __shared__ float r_tab[128];
+  __shared__ float s_genc, s_gdec, s_gdec_mu;
   pdl_wait_prior_grid();
   pdl_allow_next_grid();
-  if (static_cast<int>(blockIdx.x) >= p.n_quant_ctas) {
-    mean_and_bias_block<kSR>(p, blockIdx.x - p.n_quant_ctas, s_mu);
-    return;
-  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const TensorScale ts = tensor_scale(max_of_slots(p.slot_xr, p.n_tiles));
-  if (blockIdx.x == 0 && threadIdx.x == 0) *p.g_dec = ts.g_dec;
+  const int bid = blockIdx.x;
+  // mu_bar and the rank-one row: every CTA quantizes mu into shared memory
+  // and forms a share of the row (its warps take rows gw, gw + all warps, ...);
+  // CTA 0 also stores mu_bar.
+  const int gw = bid * kQuantWarps + warp;
+  if (p.mu != nullptr && (p.w_codes != nullptr || (p.mu_codes != nullptr && bid == 0))) {
+    quantize_mean<kSR>(p, s_mu, r_tab, bid == 0 && p.mu_codes != nullptr, &s_gdec_mu);
+    if (p.w_codes != nullptr)
+      bias_rows(s_mu, p.K, p.w_codes, p.w_scales, s_gdec_mu * __ldg(p.w_gdec), gw, p.n_out,
+                static_cast<int64_t>(gridDim.x) * kQuantWarps, p.bias);
+    __syncthreads();   // r_tab is reused below
+  }
 
-  const int strip = blockIdx.x % p.n_strips;
-  const int64_t row_base = static_cast<int64_t>(blockIdx.x / p.n_strips) * kRowsPerCta;
-  const int64_t col0 = static_cast<int64_t>(strip) * kStripCols + lane * 8;
-  const bool active = col0 < p.K;
+  // this warp's strip and first rows do not depend on the tensor scale:
+  // start their loads before it is known
+  const int warps_per_strip = (gridDim.x * kQuantWarps) / p.n_strips;
+  const bool has_work = gw < warps_per_strip * p.n_strips;
+  const int strip = gw % p.n_strips;
+  const int64_t row_step = static_cast<int64_t>(warps_per_strip) * kRowsPerIter;
+  const int64_t col0 = static_cast<int64_t>(strip) * kStripCols + lane * 16;
+  const bool active = has_work && col0 < p.K;
+  int64_t r0 = static_cast<int64_t>(gw / p.n_strips) * kRowsPerIter;
+
+  Raw16<kBf16> cur[kRowsPerIter];
+#pragma unroll
+  for (int i = 0; i < kRowsPerIter; ++i) load16<kBf16>(p.X, (r0 + i) * p.K + col0, active && r0 + i < p.rows, cur[i]);
+  float mu[16];
+#pragma unroll
+  for (int t = 0; t < 16; ++t) mu[t] = (p.mu != nullptr && active) ? __ldcg(p.mu + col0 + t) : 0.0f;
+
+  if (warp == 0) {
+    const TensorScale ts = tensor_scale(max_of_slots(p.slot_xr, p.n_tiles));
+    if (lane == 0) {
+      s_genc = ts.g_enc;
+      s_gdec = ts.g_dec;
+    }
+  }
+  __syncthreads();
+  const float g_enc = s_genc;
+  fill_rscale_table(r_tab, g_enc);
+  __syncthreads();
+  if (bid == 0 && threadIdx.x == 0) *p.g_dec = s_gdec;
+  if (!has_work) return;
   const uint32_t n_kb64 = static_cast<uint32_t>(p.K / 64);
 
-  float mu[8];
+  for (; r0 < p.rows; r0 += row_step) {
+    // the next rows of this warp are loaded while these are quantized
+    const int64_t rn = r0 + row_step;
+    Raw16<kBf16> nxt[kRowsPerIter];
 #pragma unroll
-  for (int t = 0; t < 8; ++t) mu[t] = (p.mu != nullptr && active) ? __ldcg(p.mu + col0 + t) : 0.0f;
-
-  constexpr int kRowsPerWarp = kRowsPerCta / kQuantWarps;
-  float x[kRowsPerWarp][8];
-  bool rv[kRowsPerWarp];
+    for (int i = 0; i < kRowsPerIter; ++i) load16<kBf16>(p.X, (rn + i) * p.K + col0, active && rn + i < p.rows, nxt[i]);
 #pragma unroll
-  for (int i = 0; i < kRowsPerWarp; ++i) {
-    const int64_t r = row_base + warp + i * kQuantWarps;
-    rv[i] = r < p.rows;
-    load8<kBf16>(p.X, r * p.K + col0, active && rv[i], x[i]);
-  }
+    for (int i = 0; i < kRowsPerIter; ++i) {
+      const int64_t r = r0 + i;
+      float xr[16];
+      unpack16<kBf16>(cur[i], xr);
 #pragma unroll
-  for (int i = 0; i < kRowsPerWarp; ++i) {
-    const int64_t r = row_base + warp + i * kQuantWarps;
-    float xr[8];
+      for (int t = 0; t < 16; ++t) xr[t] = __fsub_rn(xr[t], mu[t]);
+      uint32_t S;
+      const uint2 packed = quant16<kSR>(xr, g_enc, r_tab, p.seed, p.offset, p.tag,
+                                        static_cast<uint64_t>((r * p.K + col0) / 16), &S);
+      const uint32_t sw = gather_scale_word(S);
+      if (active && r < p.rows) {
+        *reinterpret_cast<uint2*>(p.codes + r * (p.K / 2) + col0 / 2) = packed;
+        if ((lane & 3) == 0)
+          *reinterpret_cast<uint32_t*>(p.scales + scale_offset(static_cast<uint64_t>(r),
+                                                               static_cast<uint32_t>(col0 / 16), n_kb64)) = sw;
+        if (p.xr_debug) {
+          float4* d = reinterpret_cast<float4*>(p.xr_debug + r * p.K + col0);
 #pragma unroll
-    for (int t = 0; t < 8; ++t) xr[t] = __fsub_rn(x[i][t], mu[t]);
-    uint32_t S;
-    const uint32_t packed = quant8<kSR>(xr, ts.g_enc, p.seed, p.offset, p.tag,
-                                        static_cast<uint64_t>(r * p.K + col0), &S, nullptr);
-    const uint32_t sw = gather_scale_word(S);
-    if (active && rv[i]) {
-      *reinterpret_cast<uint32_t*>(p.codes + r * (p.K / 2) + col0 / 2) = packed;
-      if ((lane & 7) == 0)
-        *reinterpret_cast<uint32_t*>(p.scales + scale_offset(static_cast<uint64_t>(r),
-                                                             static_cast<uint32_t>(col0 / 16), n_kb64)) = sw;
-      if (p.xr_debug) {
-        float4* d = reinterpret_cast<float4*>(p.xr_debug + r * p.K + col0);
-        d[0] = make_float4(xr[0], xr[1], xr[2], xr[3]);
-        d[1] = make_float4(xr[4], xr[5], xr[6], xr[7]);
+          for (int q = 0; q < 4; ++q) d[q] = make_float4(xr[4 * q], xr[4 * q + 1], xr[4 * q + 2], xr[4 * q + 3]);
+        }
       }
     }
+#pragma unroll
+    for (int i = 0; i < kRowsPerIter; ++i) cur[i] = nxt[i];
   }
 }
 
@@ -273,14 +345,22 @@ __global__ void zero_scale_padding(uint8_t* scales, int64_t rows, int64_t K) {
 }
 
 template <bool kBf16, bool kSR>
-static cudaError_t launch_quant_t(const QuantParams& p, int n_extra, size_t smem, cudaStream_t s,
+static cudaError_t launch_quant_t(const QuantParams& p, int64_t tasks, size_t smem, cudaStream_t s,
                                   bool pdl) {
+  const void* fn = reinterpret_cast<const void*>(quant_kernel<kBf16, kSR>);
   if (smem > 48 * 1024) {
-    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(quant_kernel<kBf16, kSR>), smem);
+    cudaError_t e = set_max_dynamic_smem(fn, smem);
     if (e != cudaSuccess) return e;
   }
-  return launch_ex(quant_kernel<kBf16, kSR>, dim3(p.n_quant_ctas + n_extra), dim3(kQuantThreads),
-                   smem, s, pdl, p);
+  // one warp per task if they all fit at once, else one full wave of
+  // resident CTAs, each warp walking rows of its strip
+  int64_t n = (tasks + kQuantWarps - 1) / kQuantWarps;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * blocks_per_sm(fn, kQuantThreads, smem);
+  if (n > cap) n = cap;
+  const int64_t min_ctas = (p.n_strips + kQuantWarps - 1) / kQuantWarps;
+  if (n < min_ctas) n = min_ctas;
+  return launch_ex(quant_kernel<kBf16, kSR>, dim3(static_cast<unsigned>(n)), dim3(kQuantThreads), smem, s,
+                   pdl, p);
 }
 
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s, bool pdl) {
@@ -300,7 +380,6 @@ cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s, bool pdl) {
   p.tag = a.tag;
   p.status = a.status;
   p.n_strips = static_cast<int>((a.K + kStripCols - 1) / kStripCols);
-  p.n_quant_ctas = static_cast<int>((a.rows + kRowsPerCta - 1) / kRowsPerCta) * p.n_strips;
   p.slot_mu = a.slot_mu;
   p.tag_mu = a.tag_mu;
   p.mu_codes = a.mu_codes;
@@ -311,13 +390,10 @@ cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s, bool pdl) {
   p.w_gdec = a.w_gdec;
   p.n_out = a.n_out;
   p.bias = a.bias;
-  int n_extra = 0;
   size_t smem = 0;
-  if (a.mu != nullptr && (a.mu_codes != nullptr || a.w_codes != nullptr)) {
-    n_extra = a.w_codes ? static_cast<int>((a.n_out + kBiasRowsPerCta - 1) / kBiasRowsPerCta) : 1;
-    if (n_extra < 1) n_extra = 1;
+  if (a.mu != nullptr && (a.mu_codes != nullptr || a.w_codes != nullptr))
     smem = static_cast<size_t>(p.n_strips) * kStripCols * sizeof(float);
-  }
+  const int64_t tasks = ((a.rows + kRowsPerIter - 1) / kRowsPerIter) * p.n_strips;
   // Padding rows of the scale atoms are written here so every output byte is
   // defined; the quantizer itself touches rows < a.rows only.
   if (a.rows % 128 != 0) {
@@ -327,10 +403,8 @@ cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s, bool pdl) {
     pdl = false;
   }
   if (a.xt == AVR_BF16)
-    return a.sr ? launch_quant_t<true, true>(p, n_extra, smem, s, pdl)
-                : launch_quant_t<true, false>(p, n_extra, smem, s, pdl);
-  return a.sr ? launch_quant_t<false, true>(p, n_extra, smem, s, pdl)
-              : launch_quant_t<false, false>(p, n_extra, smem, s, pdl);
+    return a.sr ? launch_quant_t<true, true>(p, tasks, smem, s, pdl) : launch_quant_t<true, false>(p, tasks, smem, s, pdl);
+  return a.sr ? launch_quant_t<false, true>(p, tasks, smem, s, pdl) : launch_quant_t<false, false>(p, tasks, smem, s, pdl);
 }
 
 // ---------------------------------------------------------------------------
@@ -426,11 +500,8 @@ __global__ void __launch_bounds__(kQuantThreads) bias_kernel(const BiasArgs a) {
   }
   __syncthreads();
   const float gprod = __ldg(a.mu_gdec) * __ldg(a.w_gdec);
-  const int64_t j0 = static_cast<int64_t>(blockIdx.x) * kBiasRowsPerCta;
-  const int64_t per_warp = kBiasRowsPerCta / kQuantWarps;
-  const int64_t jb = j0 + warp * per_warp;
-  const int64_t je = min64(jb + per_warp, a.n_out);
-  if (jb < je) bias_rows(s_mu, a.K, a.w_codes, a.w_scales, gprod, jb, je, a.bias);
+  bias_rows(s_mu, a.K, a.w_codes, a.w_scales, gprod, static_cast<int64_t>(blockIdx.x) * kQuantWarps + warp,
+            a.n_out, static_cast<int64_t>(gridDim.x) * kQuantWarps, a.bias);
 }
 
 cudaError_t launch_bias(const BiasArgs& a, cudaStream_t s) {
@@ -456,6 +527,14 @@ __global__ void probe_convert_kernel(const float* in, uint8_t* e4m3, uint8_t* e2
   }
 }
 
+__global__ void probe_convert_sr_kernel(const float4* in, const uint32_t* rbits, uint16_t* out, int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 v = in[i];
+    out[i] = static_cast<uint16_t>(e2m1x4_sr(v.x, v.y, v.z, v.w, rbits[i]));
+  }
+}
+
 __global__ void probe_philox_kernel(uint64_t seed, uint64_t offset, uint32_t tag, int64_t n,
                                     uint32_t* out) {
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
@@ -469,6 +548,14 @@ cudaError_t launch_probe_convert(const float* in, uint8_t* e4m3, uint8_t* e2m1, 
                                  cudaStream_t s) {
   const int64_t blocks = min64((n + 255) / 256, 148 * 16);
   probe_convert_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(in, e4m3, e2m1, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_probe_convert_sr(const float* in, const uint32_t* rbits, uint16_t* out, int64_t n,
+                                    cudaStream_t s) {
+  const int64_t blocks = min64((n + 255) / 256, 148 * 16);
+  probe_convert_sr_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(reinterpret_cast<const float4*>(in), rbits,
+                                                                         out, n);
   return cudaGetLastError();
 }
 

@@ -34,7 +34,8 @@ def _gemm(api, a_q, b_q, bias=None, out=torch.float32):
     return Y.float().cpu().numpy().astype(np.float64)
 
 
-def test_scale_layout_probe_A(api):
+@pytest.mark.parametrize("out", [torch.float32, torch.bfloat16])
+def test_scale_layout_probe_A(api, out):
     """A has every code 1.0 and random E4M3 scales; row j of B is 1.0 on the
     16-block (j mod 4) of a 64-wide K and 0 elsewhere, with scale 1.  Then
     Y[r, j] = 16 * scale_A[r, j mod 4] exactly: each output names one scale
@@ -47,12 +48,13 @@ def test_scale_layout_probe_A(api):
     for j in range(N):
         bc[j, 16 * (j % 4):16 * (j % 4) + 16] = 2
     b = F.NVFP4(F.pack_codes(bc), np.full((N, K // 16), 0x38, np.uint8), np.float32(1.0), N, K)
-    Y = _gemm(api, a, b)
+    Y = _gemm(api, a, b, out=out)
     want = 16.0 * oracle.e4m3_value(a.scales).astype(np.float64)[:, np.arange(N) % 4]
     assert np.array_equal(Y, want)
 
 
-def test_scale_layout_probe_B(api):
+@pytest.mark.parametrize("out", [torch.float32, torch.bfloat16])
+def test_scale_layout_probe_B(api, out):
     """The same with the roles swapped: Y[i, j] = 16 * scale_B[j, i mod 4]
     for N = 256 (two 128-row scale atoms of B)."""
     rng = np.random.default_rng(1)
@@ -63,12 +65,13 @@ def test_scale_layout_probe_B(api):
     a = F.NVFP4(F.pack_codes(ac), np.full((M, K // 16), 0x38, np.uint8), np.float32(1.0), M, K)
     b = F.NVFP4(F.pack_codes(np.full((N, K), 2, np.uint8)),
                 rng.integers(0x20, 0x58, (N, K // 16)).astype(np.uint8), np.float32(1.0), N, K)
-    Y = _gemm(api, a, b)
+    Y = _gemm(api, a, b, out=out)
     want = 16.0 * oracle.e4m3_value(b.scales).astype(np.float64)[:, np.arange(M) % 4].T
     assert np.array_equal(Y, want)
 
 
-def test_nibble_order_probe(api):
+@pytest.mark.parametrize("out", [torch.float32, torch.bfloat16])
+def test_nibble_order_probe(api, out):
     """Row j of B is one-hot at element j: Y[r, j] = value of A's element
     (r, j), so a swapped nibble order shows at every odd j."""
     rng = np.random.default_rng(2)
@@ -78,15 +81,16 @@ def test_nibble_order_probe(api):
     bc = np.zeros((K, K), np.uint8)
     bc[np.arange(K), np.arange(K)] = 2
     b = F.NVFP4(F.pack_codes(bc), np.full((K, K // 16), 0x38, np.uint8), np.float32(1.0), K, K)
-    Y = _gemm(api, a, b)
+    Y = _gemm(api, a, b, out=out)
     assert np.array_equal(Y, oracle.e2m1_value(ac).astype(np.float64))
 
 
-def test_k_stage_and_kblock_order(api):
-    """One-hot 64-element k-blocks across several 256-element stages: row j of
-    B selects k-block j, so Y[:, j] = 64 * scale_A[:, 4j..4j+3] mean... each
-    k-block of A holds a distinct constant, which pins the k advance inside a
-    stage and across stages (K = 640 has a partial last stage)."""
+@pytest.mark.parametrize("out", [torch.float32, torch.bfloat16])
+def test_k_stage_and_kblock_order(api, out):
+    """Each 64-element k-block of A holds one constant per row and row j of B
+    selects k-block j mod 10, so Y[:, j] = 64 * that constant: a wrong k
+    advance inside a stage or across stages (K = 640 leaves a partial last
+    stage) changes the products.  All values are exact in fp32 and bf16."""
     rng = np.random.default_rng(3)
     M, K = 128, 640
     nkb = K // 64
@@ -100,7 +104,7 @@ def test_k_stage_and_kblock_order(api):
         kb = j % nkb
         bc[j, 64 * kb:64 * kb + 64] = 2
     b = F.NVFP4(F.pack_codes(bc), np.full((N, K // 16), 0x38, np.uint8), np.float32(1.0), N, K)
-    Y = _gemm(api, a, b)
+    Y = _gemm(api, a, b, out=out)
     assert np.array_equal(Y, oracle.gemm_reference(a, b))
 
 
