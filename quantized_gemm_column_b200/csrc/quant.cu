@@ -15,8 +15,8 @@
 // shuffle, four lanes make one 4-scale atom word, one Philox4x32-10 call
 // gives the block's four 32-bit random words, and stochastic rounding is the
 // hardware convert cvt.rs.satfinite.e2m1x4 (four elements per instruction).
-// Every CTA also quantizes mu and forms a share of the rank-one row
-// mu_bar W_bar that the GEMM adds as a bias.
+// A few leading "aux" CTAs quantize mu and form the rank-one row
+// mu_bar W_bar that the GEMM adds as a bias, beside the quantizing CTAs.
 #include "device.cuh"
 #include "internal.h"
 
@@ -25,8 +25,7 @@ namespace avr {
 constexpr int kQuantThreads = 256;
 constexpr int kQuantWarps = kQuantThreads / 32;
 constexpr int kRowsPerIter = 2;            // rows a warp computes per iteration (the next ones are in flight)
-constexpr int kBiasRowsPerCta = 32;       // rank-one-row outputs per CTA of the stand-alone kernel
-constexpr int kBiasMaxChunks = 4;          // 32-element chunks per lane in flight (K <= 4096 per pass)
+constexpr int kBiasWindow = 8192;          // mu_bar values staged in shared memory at a time
 
 struct QuantParams {
   const void* X;
@@ -42,6 +41,7 @@ struct QuantParams {
   uint32_t tag;
   uint32_t* status;
   int n_strips;
+  int n_aux;              // leading CTAs that quantize mu and form the rank-one row
   // mean quantization and rank-one row
   const float* slot_mu;
   uint32_t tag_mu;
@@ -151,79 +151,145 @@ __device__ __forceinline__ uint32_t gather_scale_word(uint32_t S) {
   return S | (s1 << 8) | (s2 << 16) | (s3 << 24);
 }
 
-// bias[j] = g_dec_prod * sum_k mu_val[k] * value(w)[j, k] for the rows j of
-// this warp; mu_val holds e2m1 * e4m3 of mu.  A lane covers 32 consecutive k
-// (16 code bytes and one scale word); up to kBiasMaxChunks such loads per
-// lane are issued before any is used.
-__device__ void bias_rows(const float* s_mu, int64_t K, const uint8_t* w_codes,
-                          const uint8_t* w_scales, float g_dec_prod, int64_t j_begin,
-                          int64_t j_end, int64_t j_step, float* bias) {
-  const int lane = threadIdx.x & 31;
+// ---------------------------------------------------------------------------
+// Rank-one row mu_bar W_bar: bias[j] = g_dec(mu) g_dec(w) sum_k mu_val[k] value(w)[j, k],
+// mu_val = e2m1 * e4m3 of mu_bar.  Every mu_val is exact in f16 (an E2M1
+// magnitude has 2 significant bits and an E4M3 one 4, and the product lies
+// in [2^-10, 2688]), and so is every E2M1 value, so the per-element product
+// is taken exactly with the mixed f16 x f16 + f32 FMA and summed in fp32.
+// ---------------------------------------------------------------------------
+constexpr int kRowGroup = 32;   // output rows of one group (one per lane)
+
+// two packed E2M1 codes (one byte, element 2i in the low nibble) -> f16x2
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+  uint32_t h;
+  asm("{ .reg .b8 b; cvt.u8.u32 b, %1; cvt.rn.f16x2.e2m1x2 %0, b; }" : "=r"(h) : "r"(byte));
+  return h;
+}
+
+// c + lo(a) lo(b) + hi(a) hi(b) with f16x2 a, b and an fp32 accumulator
+__device__ __forceinline__ float fma2_f16_f32(uint32_t a, uint32_t b, float c) {
+  float d;
+  asm("{ .reg .f16 al, ah, bl, bh; .reg .f32 t;\n\t"
+      "mov.b32 {al, ah}, %1; mov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.f16 t, al, bl, %3; fma.rn.f32.f16 %0, ah, bh, t; }"
+      : "=f"(d) : "r"(a), "r"(b), "f"(c));
+  return d;
+}
+
+// Partial dot product of row j of w with the f16 values s_mu16[k - k_lo]
+// over k in [k0, k1) (multiples of 64 inside one window): one lane, 64
+// elements (two 16-byte code loads, one scale word) per step, four steps'
+// loads issued before any is used.  The E4M3 block scale is applied to each
+// 16-element partial.
+__device__ float bias_dot(const uint16_t* s_mu16, int64_t k_lo, int64_t k0, int64_t k1, int64_t j,
+                          int64_t K, const uint8_t* w_codes, const uint8_t* w_scales) {
+  constexpr int kSteps = 4;
   const uint32_t n_kb64 = static_cast<uint32_t>(K / 64);
-  for (int64_t j = j_begin; j < j_end; j += j_step) {
-    float acc = 0.0f;
-    for (int64_t base = 0; base < K; base += 32 * 32 * kBiasMaxChunks) {
-      uint4 cw[kBiasMaxChunks];
-      uint32_t sw[kBiasMaxChunks];
+  const uint8_t* row = w_codes + j * (K / 2);
+  float acc = 0.0f;
+  for (int64_t kb = k0; kb < k1; kb += 64 * kSteps) {
+    uint4 c[kSteps][2];
+    uint32_t sw[kSteps];
 #pragma unroll
-      for (int u = 0; u < kBiasMaxChunks; ++u) {
-        const int64_t k0 = base + (static_cast<int64_t>(u) * 32 + lane) * 32;
-        if (k0 < K) {
-          cw[u] = __ldg(reinterpret_cast<const uint4*>(w_codes + j * (K / 2) + k0 / 2));
-          // the two scales of this chunk share one aligned 4-byte word
-          const uint64_t so = scale_offset(static_cast<uint64_t>(j), static_cast<uint32_t>(k0 / 16), n_kb64);
-          sw[u] = __ldg(reinterpret_cast<const uint32_t*>(w_scales + (so & ~uint64_t{3}))) >> (8 * (so & 3u));
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kBiasMaxChunks; ++u) {
-        const int64_t k0 = base + (static_cast<int64_t>(u) * 32 + lane) * 32;
-        if (k0 < K) {
-          const float s0 = e4m3_value(sw[u] & 0xFFu), s1 = e4m3_value((sw[u] >> 8) & 0xFFu);
-          const uint32_t words[4] = {cw[u].x, cw[u].y, cw[u].z, cw[u].w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float sc = q < 2 ? s0 : s1;
-#pragma unroll
-            for (int t = 0; t < 8; ++t)
-              acc = fmaf(e2m1_value((words[q] >> (4 * t)) & 0xFu) * sc, s_mu[k0 + q * 8 + t], acc);
-          }
-        }
+    for (int u = 0; u < kSteps; ++u) {
+      const int64_t k = kb + 64 * u;
+      if (k < k1) {
+        const uint4* q = reinterpret_cast<const uint4*>(row + k / 2);
+        c[u][0] = __ldg(q);
+        c[u][1] = __ldg(q + 1);
+        sw[u] = __ldg(reinterpret_cast<const uint32_t*>(
+            w_scales + scale_offset(static_cast<uint64_t>(j), static_cast<uint32_t>(k / 16), n_kb64)));
       }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-    if (lane == 0) bias[j] = acc * g_dec_prod;
+    for (int u = 0; u < kSteps; ++u) {
+      const int64_t k = kb + 64 * u;
+      if (k < k1) {
+        const uint4* m = reinterpret_cast<const uint4*>(s_mu16 + (k - k_lo));   // 64 f16 = 8 x 16 B
+        const uint32_t words[8] = {c[u][0].x, c[u][0].y, c[u][0].z, c[u][0].w,
+                                   c[u][1].x, c[u][1].y, c[u][1].z, c[u][1].w};
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {           // 16-element block b: code words 2b, 2b+1
+          const uint4 m0 = m[2 * b], m1 = m[2 * b + 1];
+          const uint32_t mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+          float part = 0.0f;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t byte = (words[2 * b + q / 4] >> (8 * (q % 4))) & 0xFFu;
+            part = fma2_f16_f32(e2m1x2_to_f16x2(byte), mv[q], part);
+          }
+          acc = fmaf(part, e4m3_value((sw[u] >> (8 * b)) & 0xFFu), acc);
+        }
+      }
+    }
+  }
+  return acc;
+}
+
+// The rows of w in groups of kRowGroup, group g handled by CTA g mod
+// n_ctas: lane l takes row 32g + l and warp w the w-th of eight 64-aligned
+// segments of the window [k_lo, k_hi); warp 0 adds the eight partials in
+// warp order.  The first window stores into out[j], later windows add to it,
+// and the last one scales by g_dec_prod.  s_part: kQuantWarps * kRowGroup floats.
+__device__ void bias_window(const uint16_t* s_mu16, float* s_part, int64_t k_lo, int64_t k_hi, int64_t K,
+                            const uint8_t* w_codes, const uint8_t* w_scales, float g_dec_prod,
+                            int64_t n_out, int cta, int n_ctas, float* out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t seg = ((k_hi - k_lo + kQuantWarps * 64 - 1) / (kQuantWarps * 64)) * 64;
+  const int64_t k0 = min64(k_hi, k_lo + warp * seg), k1 = min64(k_hi, k0 + seg);
+  const int64_t n_groups = (n_out + kRowGroup - 1) / kRowGroup;
+  for (int64_t g = cta; g < n_groups; g += n_ctas) {
+    const int64_t j = g * kRowGroup + lane;
+    const float part = j < n_out ? bias_dot(s_mu16, k_lo, k0, k1, j, K, w_codes, w_scales) : 0.0f;
+    s_part[warp * kRowGroup + lane] = part;
+    __syncthreads();
+    if (warp == 0 && j < n_out) {
+      float acc = s_part[lane];
+#pragma unroll
+      for (int w = 1; w < kQuantWarps; ++w) acc += s_part[w * kRowGroup + lane];
+      if (k_lo != 0) acc += out[j];
+      out[j] = k_hi == K ? acc * g_dec_prod : acc;
+    }
+    __syncthreads();
   }
 }
 
-// Q_4(mu) into shared memory (s_mu[k] = e2m1 * e4m3 of mu, the tensor scale
-// left out) by all warps of the CTA; the CTA with `writer` set also stores
-// mu_bar (codes, every scale byte of its 1 x K atom rows, g_dec).
-template <bool kSR>
-__device__ void quantize_mean(const QuantParams& p, float* s_mu, float* r_tab, bool writer, float* g_dec_mu) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const TensorScale ts = tensor_scale(max_of_slots(p.slot_mu, p.n_tiles));
-  const uint32_t n_kb64 = static_cast<uint32_t>(p.K / 64);
-  fill_rscale_table(r_tab, ts.g_enc);
-  if (writer) {
-    if (threadIdx.x == 0) *p.mu_gdec = ts.g_dec;
-    // zero the padding rows 1..127 of every scale atom (row 0 is written below)
-    uint32_t* w = reinterpret_cast<uint32_t*>(p.mu_scales);
-    const int64_t n_words = static_cast<int64_t>(n_kb64) * 128;
-    for (int64_t i = threadIdx.x; i < n_words; i += kQuantThreads)
-      if ((i & 127) != 0) w[i] = 0u;
-  }
-  *g_dec_mu = ts.g_dec;
-  __syncthreads();
-  for (int strip = warp; strip < p.n_strips; strip += kQuantWarps) {
-    const int64_t col0 = static_cast<int64_t>(strip) * kStripCols + lane * 16;
-    const bool active = col0 < p.K;
-    float x[16];
+// 16 floats of a 64-byte aligned row (plain loads: cached in L1, so the
+// warps of an SM that read the same columns share one L2 request).
+__device__ __forceinline__ void load_f32x16(const float* p, float (&v)[16]) {
+  const float4* q = reinterpret_cast<const float4*>(p);
 #pragma unroll
-    for (int t = 0; t < 16; ++t) x[t] = active ? __ldcg(p.mu + col0 + t) : 0.0f;
+  for (int i = 0; i < 4; ++i) {
+    const float4 t = q[i];
+    v[4 * i] = t.x;
+    v[4 * i + 1] = t.y;
+    v[4 * i + 2] = t.z;
+    v[4 * i + 3] = t.w;
+  }
+}
+
+// Q_4(mu) for the window [k_lo, k_hi) by all warps of the CTA:
+// s_mu16[k - k_lo] = e2m1 * e4m3 of mu_bar in f16 (exact; the tensor scale
+// left out); with `writer` set the codes and scale words are also stored to
+// mu_bar.
+template <bool kSR>
+__device__ void quantize_mean_window(const QuantParams& p, float g_enc, const float* r_tab, int64_t k_lo,
+                                     int64_t k_hi, bool writer, uint16_t* s_mu16) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t n_kb64 = static_cast<uint32_t>(p.K / 64);
+  for (int64_t s0 = k_lo + static_cast<int64_t>(warp) * kStripCols; s0 < k_hi; s0 += kQuantWarps * kStripCols) {
+    const int64_t col0 = s0 + lane * 16;
+    const bool active = col0 < k_hi;
+    float x[16];
+    if (active) {
+      load_f32x16(p.mu + col0, x);
+    } else {
+#pragma unroll
+      for (int t = 0; t < 16; ++t) x[t] = 0.0f;
+    }
     uint32_t S;
-    const uint2 packed = quant16<kSR>(x, ts.g_enc, r_tab, p.seed, p.offset, p.tag_mu,
+    const uint2 packed = quant16<kSR>(x, g_enc, r_tab, p.seed, p.offset, p.tag_mu,
                                       static_cast<uint64_t>(col0 / 16), &S);
     const uint32_t sw = gather_scale_word(S);
     if (active) {
@@ -233,40 +299,67 @@ __device__ void quantize_mean(const QuantParams& p, float* s_mu, float* r_tab, b
           *reinterpret_cast<uint32_t*>(p.mu_scales + scale_offset(0, static_cast<uint32_t>(col0 / 16), n_kb64)) = sw;
       }
       const float sv = e4m3_value(S);
+      uint16_t* d = s_mu16 + (col0 - k_lo);
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
-        s_mu[col0 + t] = e2m1_value((packed.x >> (4 * t)) & 0xFu) * sv;
-        s_mu[col0 + 8 + t] = e2m1_value((packed.y >> (4 * t)) & 0xFu) * sv;
+        d[t] = __half_as_ushort(__float2half_rn(e2m1_value((packed.x >> (4 * t)) & 0xFu) * sv));
+        d[8 + t] = __half_as_ushort(__float2half_rn(e2m1_value((packed.y >> (4 * t)) & 0xFu) * sv));
       }
     }
   }
+}
+
+// The aux CTAs of the split quantizer: Q_4(mu) (CTA 0 stores mu_bar when
+// asked) and the rank-one row mu_bar W_bar, whose rows are shared out over
+// the warps of all aux CTAs.  They run beside the quantizing CTAs.
+template <bool kSR>
+__device__ void aux_cta(const QuantParams& p, uint16_t* s_mu16, float* s_part, float* r_tab) {
+  const TensorScale ts = tensor_scale(max_of_slots(p.slot_mu, p.n_tiles));
+  const bool writer = blockIdx.x == 0 && p.mu_codes != nullptr;
+  fill_rscale_table(r_tab, ts.g_enc);
+  if (writer) {
+    if (threadIdx.x == 0) *p.mu_gdec = ts.g_dec;
+    // zero the padding rows 1..127 of every scale atom (row 0 is written below)
+    uint32_t* w = reinterpret_cast<uint32_t*>(p.mu_scales);
+    const int64_t n_words = (p.K / 64) * 128;
+    for (int64_t i = threadIdx.x; i < n_words; i += kQuantThreads)
+      if ((i & 127) != 0) w[i] = 0u;
+  }
+  const bool bias = p.w_codes != nullptr;
+  if (!bias && !writer) return;
+  const float gprod = bias ? ts.g_dec * __ldg(p.w_gdec) : 0.0f;
   __syncthreads();
+  for (int64_t k_lo = 0; k_lo < p.K; k_lo += kBiasWindow) {
+    const int64_t k_hi = min64(p.K, k_lo + kBiasWindow);
+    quantize_mean_window<kSR>(p, ts.g_enc, r_tab, k_lo, k_hi, writer, s_mu16);
+    __syncthreads();
+    if (bias)
+      bias_window(s_mu16, s_part, k_lo, k_hi, p.K, p.w_codes, p.w_scales, gprod, p.n_out,
+                  static_cast<int>(blockIdx.x), p.n_aux, p.bias);
+    __syncthreads();
+  }
 }
 
 template <bool kBf16, bool kSR>
 __global__ void __launch_bounds__(kQuantThreads) quant_kernel(const QuantParams p) {
-  extern __shared__ float s_mu[];   // dequantized mu (K floats) when the rank-one row is formed
+  extern __shared__ uint16_t s_mu16[];   // aux CTAs: a window of mu_bar values (f16)
   __shared__ float r_tab[128];
-  __shared__ float s_genc, s_gdec, s_gdec_mu;
+  __shared__ float s_genc, s_gdec;
   pdl_wait_prior_grid();
   pdl_allow_next_grid();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bid = blockIdx.x;
-  // mu_bar and the rank-one row: every CTA quantizes mu into shared memory
-  // and forms a share of the row (its warps take rows gw, gw + all warps, ...);
-  // CTA 0 also stores mu_bar.
-  const int gw = bid * kQuantWarps + warp;
-  if (p.mu != nullptr && (p.w_codes != nullptr || (p.mu_codes != nullptr && bid == 0))) {
-    quantize_mean<kSR>(p, s_mu, r_tab, bid == 0 && p.mu_codes != nullptr, &s_gdec_mu);
-    if (p.w_codes != nullptr)
-      bias_rows(s_mu, p.K, p.w_codes, p.w_scales, s_gdec_mu * __ldg(p.w_gdec), gw, p.n_out,
-                static_cast<int64_t>(gridDim.x) * kQuantWarps, p.bias);
-    __syncthreads();   // r_tab is reused below
+  if (static_cast<int>(blockIdx.x) < p.n_aux) {
+    __shared__ float s_part[kQuantWarps * kRowGroup];
+    aux_cta<kSR>(p, s_mu16, s_part, r_tab);
+    return;
   }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bid = static_cast<int>(blockIdx.x) - p.n_aux;
+  const int n_ctas = static_cast<int>(gridDim.x) - p.n_aux;
+  const int gw = bid * kQuantWarps + warp;
 
   // this warp's strip and first rows do not depend on the tensor scale:
   // start their loads before it is known
-  const int warps_per_strip = (gridDim.x * kQuantWarps) / p.n_strips;
+  const int warps_per_strip = (n_ctas * kQuantWarps) / p.n_strips;
   const bool has_work = gw < warps_per_strip * p.n_strips;
   const int strip = gw % p.n_strips;
   const int64_t row_step = static_cast<int64_t>(warps_per_strip) * kRowsPerIter;
@@ -278,8 +371,12 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(const QuantParams 
 #pragma unroll
   for (int i = 0; i < kRowsPerIter; ++i) load16<kBf16>(p.X, (r0 + i) * p.K + col0, active && r0 + i < p.rows, cur[i]);
   float mu[16];
+  if (p.mu != nullptr && active) {
+    load_f32x16(p.mu + col0, mu);
+  } else {
 #pragma unroll
-  for (int t = 0; t < 16; ++t) mu[t] = (p.mu != nullptr && active) ? __ldcg(p.mu + col0 + t) : 0.0f;
+    for (int t = 0; t < 16; ++t) mu[t] = 0.0f;
+  }
 
   if (warp == 0) {
     const TensorScale ts = tensor_scale(max_of_slots(p.slot_xr, p.n_tiles));
@@ -353,14 +450,14 @@ static cudaError_t launch_quant_t(const QuantParams& p, int64_t tasks, size_t sm
     if (e != cudaSuccess) return e;
   }
   // one warp per task if they all fit at once, else one full wave of
-  // resident CTAs, each warp walking rows of its strip
+  // resident CTAs (less the aux CTAs), each warp walking rows of its strip
   int64_t n = (tasks + kQuantWarps - 1) / kQuantWarps;
-  const int64_t cap = static_cast<int64_t>(sm_count()) * blocks_per_sm(fn, kQuantThreads, smem);
+  int64_t cap = static_cast<int64_t>(sm_count()) * blocks_per_sm(fn, kQuantThreads, smem) - p.n_aux;
   if (n > cap) n = cap;
   const int64_t min_ctas = (p.n_strips + kQuantWarps - 1) / kQuantWarps;
   if (n < min_ctas) n = min_ctas;
-  return launch_ex(quant_kernel<kBf16, kSR>, dim3(static_cast<unsigned>(n)), dim3(kQuantThreads), smem, s,
-                   pdl, p);
+  return launch_ex(quant_kernel<kBf16, kSR>, dim3(static_cast<unsigned>(n + p.n_aux)), dim3(kQuantThreads),
+                   smem, s, pdl, p);
 }
 
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s, bool pdl) {
@@ -391,8 +488,16 @@ cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s, bool pdl) {
   p.n_out = a.n_out;
   p.bias = a.bias;
   size_t smem = 0;
-  if (a.mu != nullptr && (a.mu_codes != nullptr || a.w_codes != nullptr))
-    smem = static_cast<size_t>(p.n_strips) * kStripCols * sizeof(float);
+  if (a.mu != nullptr && (a.mu_codes != nullptr || a.w_codes != nullptr)) {
+    int64_t n_aux = 1;
+    if (a.w_codes != nullptr) {
+      n_aux = (a.n_out + kRowGroup - 1) / kRowGroup;
+      const int64_t max_aux = sm_count() / 4 > 1 ? sm_count() / 4 : 1;
+      n_aux = n_aux > max_aux ? max_aux : n_aux;
+    }
+    p.n_aux = static_cast<int>(n_aux);
+    smem = static_cast<size_t>(min64(a.K, kBiasWindow)) * sizeof(uint16_t);
+  }
   const int64_t tasks = ((a.rows + kRowsPerIter - 1) / kRowsPerIter) * p.n_strips;
   // Padding rows of the scale atoms are written here so every output byte is
   // defined; the quantizer itself touches rows < a.rows only.
@@ -490,27 +595,28 @@ cudaError_t launch_quant_transposed(const QuantTransposedArgs& a, cudaStream_t s
 // rank-one row alone, from an already quantized mu
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kQuantThreads) bias_kernel(const BiasArgs a) {
-  extern __shared__ float s_mu[];
-  const int warp = threadIdx.x >> 5;
+  extern __shared__ uint16_t s_mu16[];
+  __shared__ float s_part[kQuantWarps * kRowGroup];
   const uint32_t n_kb64 = static_cast<uint32_t>(a.K / 64);
-  for (int64_t k = threadIdx.x; k < a.K; k += kQuantThreads) {
-    const uint32_t byte = a.mu_codes[k / 2];
-    const uint32_t code = (k & 1) ? (byte >> 4) : (byte & 0xFu);
-    s_mu[k] = e2m1_value(code) * e4m3_value(a.mu_scales[scale_offset(0, static_cast<uint32_t>(k / 16), n_kb64)]);
-  }
-  __syncthreads();
   const float gprod = __ldg(a.mu_gdec) * __ldg(a.w_gdec);
-  bias_rows(s_mu, a.K, a.w_codes, a.w_scales, gprod, static_cast<int64_t>(blockIdx.x) * kQuantWarps + warp,
-            a.n_out, static_cast<int64_t>(gridDim.x) * kQuantWarps, a.bias);
+  for (int64_t k_lo = 0; k_lo < a.K; k_lo += kBiasWindow) {
+    const int64_t k_hi = min64(a.K, k_lo + kBiasWindow);
+    for (int64_t k = k_lo + threadIdx.x; k < k_hi; k += kQuantThreads) {
+      const uint32_t byte = a.mu_codes[k / 2];
+      const uint32_t code = (k & 1) ? (byte >> 4) : (byte & 0xFu);
+      const float v = e2m1_value(code) * e4m3_value(a.mu_scales[scale_offset(0, static_cast<uint32_t>(k / 16), n_kb64)]);
+      s_mu16[k - k_lo] = __half_as_ushort(__float2half_rn(v));
+    }
+    __syncthreads();
+    bias_window(s_mu16, s_part, k_lo, k_hi, a.K, a.w_codes, a.w_scales, gprod, a.n_out,
+                static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x), a.bias);
+    __syncthreads();
+  }
 }
 
 cudaError_t launch_bias(const BiasArgs& a, cudaStream_t s) {
-  const size_t smem = static_cast<size_t>(a.K) * sizeof(float);
-  if (smem > 48 * 1024) {
-    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(bias_kernel), smem);
-    if (e != cudaSuccess) return e;
-  }
-  const unsigned grid = static_cast<unsigned>((a.n_out + kBiasRowsPerCta - 1) / kBiasRowsPerCta);
+  const size_t smem = static_cast<size_t>(min64(a.K, kBiasWindow)) * sizeof(uint16_t);
+  const unsigned grid = static_cast<unsigned>((a.n_out + kRowGroup - 1) / kRowGroup);
   bias_kernel<<<grid, kQuantThreads, smem, s>>>(a);
   return cudaGetLastError();
 }

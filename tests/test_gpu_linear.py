@@ -48,7 +48,8 @@ def test_tiny_forward_fp32(api, rm):
     assert np.linalg.norm(Yg - Yref) / np.linalg.norm(Yref) <= 1e-5
 
 
-@pytest.mark.parametrize("l,m,n", [(300, 192, 320), (1024, 512, 768)])
+@pytest.mark.parametrize("l,m,n", [(300, 192, 320), (1024, 512, 768),
+                                   (256, 8320, 192)])   # forward K above the mean window
 def test_forward_and_dgrad_bf16(api, l, m, n):
     rng = inputs.rng_for(60, l)
     X = inputs.to_bf16(inputs.spiked_activations(rng, l, m, 2, (8.0, 4.0), n_hot=3))
@@ -90,16 +91,17 @@ def test_vanilla_forward_and_dgrad(api):
         assert np.linalg.norm(g - r) / np.linalg.norm(r) <= 1e-5
 
 
-def test_bias_row_entry_point(api):
+@pytest.mark.parametrize("K", [512, 8384])   # one and two windows of K
+def test_bias_row_entry_point(api, K):
     rng = np.random.default_rng(5)
-    mu_q = oracle.nvfp4_quantize(rng.standard_normal((1, 512)).astype(np.float32), "rne")
-    w_q = oracle.nvfp4_quantize(rng.standard_normal((320, 512)).astype(np.float32), "rne")
+    mu_q = oracle.nvfp4_quantize(rng.standard_normal((1, K)).astype(np.float32), "rne")
+    w_q = oracle.nvfp4_quantize(rng.standard_normal((320, K)).astype(np.float32), "rne")
     bias = torch.empty(320, dtype=torch.float32, device="cuda")
-    ws = api.workspace(0, 512)
+    ws = api.workspace(0, K)
     api.averis_bias_row(from_oracle(mu_q, api), from_oracle(w_q, api), bias, ws)
     ref = oracle.bias_row(mu_q, w_q)
-    tol = 512 * 2.0 ** -24 * (np.abs(oracle.nvfp4_dequantize(mu_q)) @
-                              np.abs(oracle.nvfp4_dequantize(w_q)).T)[0] + 1e-30
+    tol = K * 2.0 ** -24 * (np.abs(oracle.nvfp4_dequantize(mu_q)) @
+                            np.abs(oracle.nvfp4_dequantize(w_q)).T)[0] + 1e-30
     assert np.all(np.abs(bias.cpu().numpy() - ref) <= tol)
 
 

@@ -43,7 +43,8 @@ def _split(api, Xd, rm, seed=7, offset=0, grad=False):
 
 
 SHAPES = [(256, 128, "f32"), (300, 192, "bf16"), (1024, 1024, "bf16"), (4133, 640, "bf16"),
-          (512, 6144, "bf16"), (64, 64, "f32"), (1, 256, "bf16")]
+          (512, 6144, "bf16"), (64, 64, "f32"), (1, 256, "bf16"),
+          (40, 8256, "bf16")]     # K above the 8192-column window of the mean quantizer
 
 
 @pytest.mark.parametrize("l,K,dt", SHAPES)
