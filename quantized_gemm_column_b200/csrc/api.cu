@@ -69,14 +69,19 @@ bool make_tensor_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType 
 
 cudaError_t set_max_dynamic_smem(const void* func, size_t bytes) {
   static std::mutex mu;
-  static std::set<std::pair<int, const void*>> done;
+  static std::map<std::pair<int, const void*>, size_t> done;   // largest size set so far
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> g(mu);
-  if (done.count({dev, func})) return cudaSuccess;
+  auto it = done.find({dev, func});
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
-  if (e == cudaSuccess) done.insert({dev, func});
+  if (e != cudaSuccess) return e;
+  // every kernel of the library asks for the largest shared-memory carveout,
+  // so that back-to-back launches never wait for the SM to re-split L1
+  e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess) done[{dev, func}] = bytes;
   return e;
 }
 

@@ -104,6 +104,28 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// L2 eviction-priority policies for the cache-hinted loads below.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int32_t x, int32_t y, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+        "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
@@ -246,11 +268,13 @@ constexpr uint32_t kLayoutSwizzle64B = 4;
 __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
-    const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
-    const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
-    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
-    k0 += 0x9E3779B9u;
-    k1 += 0xBB67AE85u;
+    // one 32 x 32 -> 64-bit multiply gives both halves of each product
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c.x;
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c.z;
+    const uint32_t lo0 = static_cast<uint32_t>(p0), hi0 = static_cast<uint32_t>(p0 >> 32);
+    const uint32_t lo1 = static_cast<uint32_t>(p1), hi1 = static_cast<uint32_t>(p1 >> 32);
+    c = make_uint4(hi1 ^ c.y ^ (k0 + static_cast<uint32_t>(r) * 0x9E3779B9u), lo1,
+                   hi0 ^ c.w ^ (k1 + static_cast<uint32_t>(r) * 0xBB67AE85u), lo0);
   }
   return c;
 }
@@ -338,6 +362,34 @@ __device__ __forceinline__ float e2m1_value(uint32_t c) {
 // tcgen05 128x4 atom layout (512-byte atoms, row-group major).
 __device__ __forceinline__ uint64_t scale_offset(uint64_t r, uint32_t c, uint32_t n_kb64) {
   return ((r >> 7) * n_kb64 + (c >> 2)) * 512ull + (r & 31u) * 16u + ((r >> 5) & 3u) * 4u + (c & 3u);
+}
+
+// fl(a - c) for the two bf16 halves of w (element 2i in the low half) and
+// fp32 c: the mixed-precision subtract widens the bf16 exactly, then rounds
+// once, i.e. the same bits as __fsub_rn(float(a), c).
+__device__ __forceinline__ void sub_bf16x2_f32(uint32_t w, float c_lo, float c_hi, float& d_lo, float& d_hi) {
+  asm("{\n\t.reg .b16 l, h;\n\t"
+      "mov.b32 {l, h}, %2;\n\t"
+      "sub.rn.f32.bf16 %0, l, %3;\n\t"
+      "sub.rn.f32.bf16 %1, h, %4;\n\t}"
+      : "=f"(d_lo), "=f"(d_hi) : "r"(w), "f"(c_lo), "f"(c_hi));
+}
+
+// max(a, b, c) in one three-input instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// (a0 * b, a1 * b) rounded to nearest, as one packed f32x2 multiply
+__device__ __forceinline__ void fmul2(float a0, float a1, float b, float& d0, float& d1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "mov.b64 b, {%4, %4};\n\t"
+      "mul.rn.f32x2 d, a, b;\n\t"
+      "mov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b));
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

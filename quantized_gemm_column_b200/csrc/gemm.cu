@@ -175,46 +175,65 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
   } else if (warp == 0) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      int it = 0, tcount = 0;
+      // The issuing thread is on the critical path: every tcgen05 instruction
+      // it is late with idles the tensor pipe, so the loop keeps its
+      // bookkeeping to increments (stage, phase and scale-buffer counters)
+      // and issues a full stage's copies and MMAs unrolled, with descriptors
+      // advanced by constants.
+      uint32_t st = 0, ph = 0, sf_buf = 0;
+      const int n_full = static_cast<int>(p.K / Cfg::kStageK);               // stages of kKbPerStage k-blocks
+      const int tail_kb = static_cast<int>((p.K % Cfg::kStageK) / 64);       // k-blocks of a last, partial stage
+      int tcount = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tcount) {
         const int ab = tcount % Cfg::kAccBufs;
         const int use = tcount / Cfg::kAccBufs;
-        if (use >= 1 && !mbar_wait(&acc_empty[ab], static_cast<uint32_t>(use - 1) & 1u, p.status)) {
-          ok = false;
-          break;
-        }
+        if (use >= 1 && !mbar_wait(&acc_empty[ab], static_cast<uint32_t>(use - 1) & 1u, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(ab * Cfg::kAccCols);
-        for (int ks = 0; ks < n_kst; ++ks, ++it) {
-          const int st = it % Cfg::kStages;
-          if (!mbar_wait(&full[st], static_cast<uint32_t>(it / Cfg::kStages) & 1u, p.status)) {
+        for (int ks = 0; ks < n_kst; ++ks) {
+          if (!mbar_wait(&full[st], ph, p.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const int nkb = static_cast<int>(min64(Cfg::kKbPerStage, (p.K - static_cast<int64_t>(ks) * Cfg::kStageK) / 64));
-          const uint32_t buf = static_cast<uint32_t>(it & 1);
-          const uint32_t sfa_t = tmem + Cfg::kSfCol + buf * (Cfg::kSfaCols + Cfg::kSfbCols);
+          const uint32_t sfa_t = tmem + Cfg::kSfCol + sf_buf * (Cfg::kSfaCols + Cfg::kSfbCols);
           const uint32_t sfb_t = sfa_t + Cfg::kSfaCols;
-          for (int kb = 0; kb < nkb; ++kb) {
-            tc_cp_32x128b_warpx4(sfa_t + 4 * kb,
-                                 smem_desc(smem_u32(sSfa + st * Cfg::kSfaBytes + kb * 512), 0, 128, kLayoutSwizzleNone));
+          // 16-byte-unit descriptor fields: +32 per 512-byte scale atom, +2 per 32-byte k-block step
+          const uint64_t sfa_d = smem_desc(smem_u32(sSfa + st * Cfg::kSfaBytes), 0, 128, kLayoutSwizzleNone);
+          const uint64_t sfb_d = smem_desc(smem_u32(sSfb + st * Cfg::kSfbBytes), 0, 128, kLayoutSwizzleNone);
+          const uint64_t a0 = smem_desc(smem_u32(sA + st * Cfg::kABytes), 16, Cfg::kSbo, Cfg::kSwizzle);
+          const uint64_t b0 = smem_desc(smem_u32(sB + st * Cfg::kBBytes), 16, Cfg::kSbo, Cfg::kSwizzle);
+          if (ks < n_full) {
 #pragma unroll
-            for (int g = 0; g < Cfg::kBN / 128; ++g)
-              tc_cp_32x128b_warpx4(sfb_t + (Cfg::kBN / 32) * kb + 4 * g,
-                                   smem_desc(smem_u32(sSfb + st * Cfg::kSfbBytes + g * Cfg::kKbPerStage * 512 + kb * 512),
-                                             0, 128, kLayoutSwizzleNone));
-          }
-          const uint32_t a_base = smem_u32(sA + st * Cfg::kABytes);
-          const uint32_t b_base = smem_u32(sB + st * Cfg::kBBytes);
-          for (int kb = 0; kb < nkb; ++kb) {
-            const uint64_t adesc = smem_desc(a_base + kb * 32, 16, Cfg::kSbo, Cfg::kSwizzle);
-            const uint64_t bdesc = smem_desc(b_base + kb * 32, 16, Cfg::kSbo, Cfg::kSwizzle);
-            mma_nvf4(d_tmem, adesc, bdesc, Cfg::kIdesc, sfa_t + 4 * kb, sfb_t + (Cfg::kBN / 32) * kb,
-                     (ks > 0 || kb > 0) ? 1u : 0u);
+            for (int kb = 0; kb < Cfg::kKbPerStage; ++kb) {
+              tc_cp_32x128b_warpx4(sfa_t + 4 * kb, sfa_d + static_cast<uint64_t>(32 * kb));
+#pragma unroll
+              for (int g = 0; g < Cfg::kBN / 128; ++g)
+                tc_cp_32x128b_warpx4(sfb_t + (Cfg::kBN / 32) * kb + 4 * g,
+                                     sfb_d + static_cast<uint64_t>(32 * (g * Cfg::kKbPerStage + kb)));
+            }
+#pragma unroll
+            for (int kb = 0; kb < Cfg::kKbPerStage; ++kb)
+              mma_nvf4(d_tmem, a0 + static_cast<uint64_t>(2 * kb), b0 + static_cast<uint64_t>(2 * kb), Cfg::kIdesc,
+                       sfa_t + 4 * kb, sfb_t + (Cfg::kBN / 32) * kb, (ks > 0 || kb > 0) ? 1u : 0u);
+          } else {
+            for (int kb = 0; kb < tail_kb; ++kb) {
+              tc_cp_32x128b_warpx4(sfa_t + 4 * kb, sfa_d + static_cast<uint64_t>(32 * kb));
+              for (int g = 0; g < Cfg::kBN / 128; ++g)
+                tc_cp_32x128b_warpx4(sfb_t + (Cfg::kBN / 32) * kb + 4 * g,
+                                     sfb_d + static_cast<uint64_t>(32 * (g * Cfg::kKbPerStage + kb)));
+            }
+            for (int kb = 0; kb < tail_kb; ++kb)
+              mma_nvf4(d_tmem, a0 + static_cast<uint64_t>(2 * kb), b0 + static_cast<uint64_t>(2 * kb), Cfg::kIdesc,
+                       sfa_t + 4 * kb, sfb_t + (Cfg::kBN / 32) * kb, (ks > 0 || kb > 0) ? 1u : 0u);
           }
           tc_commit(&empty[st]);
+          sf_buf ^= 1u;
+          if (++st == Cfg::kStages) {
+            st = 0;
+            ph ^= 1u;
+          }
         }
         tc_commit(&acc_full[ab]);
       }
@@ -232,6 +251,14 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
       const int ab = tcount % Cfg::kAccBufs;
       const int64_t m0 = static_cast<int64_t>(tile / p.tiles_n) * Cfg::kBM;
       const int64_t n0 = static_cast<int64_t>(tile % p.tiles_n) * Cfg::kBN;
+      // lane l holds the bias of column 32 cc + l of each of its chunks, fetched
+      // before the accumulator is ready so the load hides behind the mainloop
+      float bias_l[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int64_t col = n0 + 32 * (4 * h + c) + lane;
+        bias_l[c] = (p.bias != nullptr && col < p.N) ? __ldg(p.bias + col) : 0.0f;
+      }
       const bool ok = mbar_wait(&acc_full[ab], static_cast<uint32_t>(tcount / Cfg::kAccBufs) & 1u, p.status);
       // all epilogue threads agree, so the .sync.aligned loads below run in
       // every lane of every warp or in none
@@ -240,7 +267,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
       // the previous tile's store must have read the staging tile
       if (leader) bulk_wait_group_read<0>();
       named_barrier(1, kEpiThreads);
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int cc = 4 * h + c;              // 32-column chunk of the tile
         uint32_t v[32];
@@ -248,18 +275,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
                                static_cast<uint32_t>(ab * Cfg::kAccCols + 32 * cc), v);
         tmem_ld_wait();
         float b[32];
-        const int64_t col = n0 + 32 * cc;
-        if (p.bias != nullptr && col < p.N) {
-          const float4* bp = reinterpret_cast<const float4*>(p.bias + col);
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const float4 t = __ldg(bp + u);
-            b[4 * u] = t.x; b[4 * u + 1] = t.y; b[4 * u + 2] = t.z; b[4 * u + 3] = t.w;
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) b[j] = 0.0f;
-        }
+        for (int j = 0; j < 32; ++j) b[j] = __shfl_sync(0xFFFFFFFFu, bias_l[c], j);
         if (kBf16Out) {
           // 32 bf16 = 64 bytes = four 16-byte pieces of row r in box cc/2
           uint8_t* box = sOut + (cc >> 1) * (Cfg::kBM * 128);

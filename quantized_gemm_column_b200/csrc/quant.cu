@@ -81,25 +81,24 @@ __device__ __forceinline__ void load16(const void* base, int64_t idx, bool activ
   for (int i = 0; i < (kBf16 ? 2 : 4); ++i) r.w[i] = __ldcs(p + i);
 }
 
+// xr = fl(x - mu) for the 16 loaded elements of a lane
 template <bool kBf16>
-__device__ __forceinline__ void unpack16(const Raw16<kBf16>& r, float (&x)[16]) {
+__device__ __forceinline__ void sub_mu16(const Raw16<kBf16>& r, const float (&mu)[16], float (&xr)[16]) {
   if (kBf16) {
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const uint32_t u[4] = {r.w[i].x, r.w[i].y, r.w[i].z, r.w[i].w};
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        x[8 * i + 2 * k] = bf16_lo(u[k]);
-        x[8 * i + 2 * k + 1] = bf16_hi(u[k]);
-      }
+      for (int k = 0; k < 4; ++k)
+        sub_bf16x2_f32(u[k], mu[8 * i + 2 * k], mu[8 * i + 2 * k + 1], xr[8 * i + 2 * k], xr[8 * i + 2 * k + 1]);
     }
   } else {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      x[4 * i] = __uint_as_float(r.w[i].x);
-      x[4 * i + 1] = __uint_as_float(r.w[i].y);
-      x[4 * i + 2] = __uint_as_float(r.w[i].z);
-      x[4 * i + 3] = __uint_as_float(r.w[i].w);
+      xr[4 * i] = __fsub_rn(__uint_as_float(r.w[i].x), mu[4 * i]);
+      xr[4 * i + 1] = __fsub_rn(__uint_as_float(r.w[i].y), mu[4 * i + 1]);
+      xr[4 * i + 2] = __fsub_rn(__uint_as_float(r.w[i].z), mu[4 * i + 2]);
+      xr[4 * i + 3] = __fsub_rn(__uint_as_float(r.w[i].w), mu[4 * i + 3]);
     }
   }
 }
@@ -118,14 +117,15 @@ template <bool kSR>
 __device__ __forceinline__ uint2 quant16(const float (&xr)[16], float g_enc, const float* r_tab,
                                          uint64_t seed, uint64_t offset, uint32_t tag, uint64_t blk,
                                          uint32_t* S_out) {
-  float am = 0.0f;
+  float am = fmax3(fabsf(xr[0]), fabsf(xr[1]), fabsf(xr[2]));
 #pragma unroll
-  for (int t = 0; t < 16; ++t) am = fmaxf(am, fabsf(xr[t]));
+  for (int t = 3; t < 15; t += 2) am = fmax3(am, fabsf(xr[t]), fabsf(xr[t + 1]));
+  am = fmaxf(am, fabsf(xr[15]));
   const uint32_t S = e4m3_rn_satfinite(__fmul_rn(__fdiv_rn(am, 6.0f), g_enc));
   const float r = r_tab[S];
   float y[16];
 #pragma unroll
-  for (int t = 0; t < 16; ++t) y[t] = __fmul_rn(xr[t], r);
+  for (int t = 0; t < 16; t += 2) fmul2(xr[t], xr[t + 1], r, y[t], y[t + 1]);
   uint2 packed;
   if (kSR) {
     const uint4 w = philox_block(seed, offset, tag, blk);
@@ -403,9 +403,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(const QuantParams 
     for (int i = 0; i < kRowsPerIter; ++i) {
       const int64_t r = r0 + i;
       float xr[16];
-      unpack16<kBf16>(cur[i], xr);
-#pragma unroll
-      for (int t = 0; t < 16; ++t) xr[t] = __fsub_rn(xr[t], mu[t]);
+      sub_mu16<kBf16>(cur[i], mu, xr);
       uint32_t S;
       const uint2 packed = quant16<kSR>(xr, g_enc, r_tab, p.seed, p.offset, p.tag,
                                         static_cast<uint64_t>((r * p.K + col0) / 16), &S);
@@ -445,10 +443,8 @@ template <bool kBf16, bool kSR>
 static cudaError_t launch_quant_t(const QuantParams& p, int64_t tasks, size_t smem, cudaStream_t s,
                                   bool pdl) {
   const void* fn = reinterpret_cast<const void*>(quant_kernel<kBf16, kSR>);
-  if (smem > 48 * 1024) {
-    cudaError_t e = set_max_dynamic_smem(fn, smem);
-    if (e != cudaSuccess) return e;
-  }
+  cudaError_t e = set_max_dynamic_smem(fn, smem);
+  if (e != cudaSuccess) return e;
   // one warp per task if they all fit at once, else one full wave of
   // resident CTAs (less the aux CTAs), each warp walking rows of its strip
   int64_t n = (tasks + kQuantWarps - 1) / kQuantWarps;
