@@ -96,14 +96,16 @@ __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_consta
     p.part[2 * plane + o] = mn;
   }
 
-  // Last CTA of this column tile finalizes it.
-  __threadfence();
+  // Last CTA of this column tile finalizes it.  The CTA barrier orders every
+  // thread's partial stores before thread 0's ticket, an acquire-release
+  // increment at GPU scope: it publishes them (release, cumulative over the
+  // barrier) and, for the last CTA, makes every other CTA's partials visible
+  // to the fold below (acquire, passed on by the second barrier).
   __syncthreads();
-  if (tid == 0) s_last = (atomicInc(&p.tickets[t], static_cast<uint32_t>(p.C - 1)) ==
-                          static_cast<uint32_t>(p.C - 1));
+  if (tid == 0) s_last = ticket_inc_acq_rel(&p.tickets[t], static_cast<uint32_t>(p.C - 1)) ==
+                         static_cast<uint32_t>(p.C - 1);
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
 
   // Each thread folds its column's chunk partials in chunk order; the loads
   // of a batch of kBatch chunks (three planes) are all issued before the

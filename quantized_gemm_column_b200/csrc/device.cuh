@@ -27,6 +27,14 @@ __device__ __forceinline__ void raise_status(uint32_t* status, uint32_t code) {
   if (status) atomicCAS(status, 0u, code);
 }
 
+// atomicInc (wrapping to 0 after `limit`) with acquire-release semantics at GPU
+// scope; returns the old value.
+__device__ __forceinline__ uint32_t ticket_inc_acq_rel(uint32_t* addr, uint32_t limit) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.inc.u32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(limit) : "memory");
+  return old;
+}
+
 // Wall-clock bound for every spin-wait: after this many nanoseconds of
 // waiting the kernel records AVR_ERR_DEVICE_TIMEOUT and gives up.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
