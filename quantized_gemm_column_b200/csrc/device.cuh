@@ -98,6 +98,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   return true;
 }
 
+// Like mbar_wait, but polling with test_wait, which never suspends the
+// thread: for hand-offs on the critical path, where waking from a suspended
+// try_wait costs a few hundred nanoseconds.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_poll(uint64_t* bar, uint32_t parity, uint32_t* status) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t spins = 0;
+  while (!mbar_test(bar, parity)) {
+    if (((++spins) & 1023u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+      raise_status(status, AVR_ERR_DEVICE_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------------------
 // TMA (tensor) loads and bulk copies, global -> shared, completing on an
 // mbarrier.  No cluster multicast anywhere in this library.

@@ -183,13 +183,19 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
       uint32_t st = 0, ph = 0, sf_buf = 0;
       const int n_full = static_cast<int>(p.K / Cfg::kStageK);               // stages of kKbPerStage k-blocks
       const int tail_kb = static_cast<int>((p.K % Cfg::kStageK) / 64);       // k-blocks of a last, partial stage
+      // a tile's first scale copies go out before the wait for its accumulator
+      // (they write the scale area, not the accumulator), so they overlap the
+      // previous tile's epilogue
+      auto wait_acc_empty = [&](int ab, int use) {
+        if (!mbar_wait_poll(&acc_empty[ab], static_cast<uint32_t>(use - 1) & 1u, p.status)) return false;
+        tc_fence_after();
+        return true;
+      };
       int tcount = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tcount) {
         const int ab = tcount % Cfg::kAccBufs;
         const int use = tcount / Cfg::kAccBufs;
-        if (use >= 1 && !mbar_wait(&acc_empty[ab], static_cast<uint32_t>(use - 1) & 1u, p.status)) break;
-        tc_fence_after();
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(ab * Cfg::kAccCols);
         for (int ks = 0; ks < n_kst; ++ks) {
           if (!mbar_wait(&full[st], ph, p.status)) {
@@ -213,6 +219,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
                 tc_cp_32x128b_warpx4(sfb_t + (Cfg::kBN / 32) * kb + 4 * g,
                                      sfb_d + static_cast<uint64_t>(32 * (g * Cfg::kKbPerStage + kb)));
             }
+            if (ks == 0 && use >= 1 && !wait_acc_empty(ab, use)) {
+              ok = false;
+              break;
+            }
 #pragma unroll
             for (int kb = 0; kb < Cfg::kKbPerStage; ++kb)
               mma_nvf4(d_tmem, a0 + static_cast<uint64_t>(2 * kb), b0 + static_cast<uint64_t>(2 * kb), Cfg::kIdesc,
@@ -223,6 +233,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
               for (int g = 0; g < Cfg::kBN / 128; ++g)
                 tc_cp_32x128b_warpx4(sfb_t + (Cfg::kBN / 32) * kb + 4 * g,
                                      sfb_d + static_cast<uint64_t>(32 * (g * Cfg::kKbPerStage + kb)));
+            }
+            if (ks == 0 && use >= 1 && !wait_acc_empty(ab, use)) {
+              ok = false;
+              break;
             }
             for (int kb = 0; kb < tail_kb; ++kb)
               mma_nvf4(d_tmem, a0 + static_cast<uint64_t>(2 * kb), b0 + static_cast<uint64_t>(2 * kb), Cfg::kIdesc,
@@ -259,7 +273,9 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
         const int64_t col = n0 + 32 * (4 * h + c) + lane;
         bias_l[c] = (p.bias != nullptr && col < p.N) ? __ldg(p.bias + col) : 0.0f;
       }
-      const bool ok = mbar_wait(&acc_full[ab], static_cast<uint32_t>(tcount / Cfg::kAccBufs) & 1u, p.status);
+      uint32_t okw = 0;
+      if (lane == 0) okw = mbar_wait_poll(&acc_full[ab], static_cast<uint32_t>(tcount / Cfg::kAccBufs) & 1u, p.status) ? 1u : 0u;
+      const bool ok = __shfl_sync(0xFFFFFFFFu, okw, 0) != 0;
       // all epilogue threads agree, so the .sync.aligned loads below run in
       // every lane of every warp or in none
       if (named_barrier_or(1, kEpiThreads, !ok)) break;
@@ -267,16 +283,9 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
       // the previous tile's store must have read the staging tile
       if (leader) bulk_wait_group_read<0>();
       named_barrier(1, kEpiThreads);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      // one 32-column chunk: alpha * acc + bias, converted, into the staging tile
+      auto emit = [&](int c, const uint32_t (&v)[32]) {
         const int cc = 4 * h + c;              // 32-column chunk of the tile
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) +
-                               static_cast<uint32_t>(ab * Cfg::kAccCols + 32 * cc), v);
-        tmem_ld_wait();
-        float b[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) b[j] = __shfl_sync(0xFFFFFFFFu, bias_l[c], j);
         if (kBf16Out) {
           // 32 bf16 = 64 bytes = four 16-byte pieces of row r in box cc/2
           uint8_t* box = sOut + (cc >> 1) * (Cfg::kBM * 128);
@@ -286,8 +295,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const int j = 8 * u + 2 * k;
-              const __nv_bfloat162 pr = __floats2bfloat162_rn(fmaf(alpha, __uint_as_float(v[j]), b[j]),
-                                                              fmaf(alpha, __uint_as_float(v[j + 1]), b[j + 1]));
+              const float b0 = __shfl_sync(0xFFFFFFFFu, bias_l[c], j);
+              const float b1 = __shfl_sync(0xFFFFFFFFu, bias_l[c], j + 1);
+              const __nv_bfloat162 pr = __floats2bfloat162_rn(fmaf(alpha, __uint_as_float(v[j]), b0),
+                                                              fmaf(alpha, __uint_as_float(v[j + 1]), b1));
               w[k] = *reinterpret_cast<const uint32_t*>(&pr);
             }
             const int piece = ((cc & 1) * 4 + u) ^ (r & 7);
@@ -298,19 +309,31 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
           uint8_t* box = sOut + cc * (Cfg::kBM * 128);
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
-            const int j = 4 * u;
-            const float4 f = make_float4(fmaf(alpha, __uint_as_float(v[j]), b[j]),
-                                         fmaf(alpha, __uint_as_float(v[j + 1]), b[j + 1]),
-                                         fmaf(alpha, __uint_as_float(v[j + 2]), b[j + 2]),
-                                         fmaf(alpha, __uint_as_float(v[j + 3]), b[j + 3]));
-            *reinterpret_cast<float4*>(box + r * 128 + ((u ^ (r & 7)) * 16)) = f;
+            float f[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              f[k] = fmaf(alpha, __uint_as_float(v[4 * u + k]), __shfl_sync(0xFFFFFFFFu, bias_l[c], 4 * u + k));
+            *reinterpret_cast<float4*>(box + r * 128 + ((u ^ (r & 7)) * 16)) = make_float4(f[0], f[1], f[2], f[3]);
           }
         }
+      };
+      // two chunks per tensor-memory round trip; the accumulator goes back to
+      // the MMA warp as soon as the last two are in registers
+      const uint32_t t_row = tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(ab * Cfg::kAccCols);
+#pragma unroll
+      for (int c2 = 0; c2 < 4; c2 += 2) {
+        uint32_t v0[32], v1[32];
+        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(32 * (4 * h + c2)), v0);
+        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(32 * (4 * h + c2 + 1)), v1);
+        tmem_ld_wait();
+        if (c2 == 2) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[ab]);
+        }
+        emit(c2, v0);
+        emit(c2 + 1, v1);
       }
-      // accumulator drained: hand it back to the MMA warp
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[ab]);
       // staging tile complete and visible to the TMA engine: store it
       fence_proxy_async_smem();
       named_barrier(1, kEpiThreads);
