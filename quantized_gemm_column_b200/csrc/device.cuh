@@ -312,6 +312,33 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
   return c;
 }
 
+// Philox4x32-10 with its round keys computed once: a thread that draws many
+// blocks under one (seed, tag) keeps k0 + r W0 and k1 + r W1 in registers.
+struct PhiloxKeys {
+  uint32_t k0[10], k1[10];
+};
+__device__ __forceinline__ PhiloxKeys philox_keys(uint64_t seed) {
+  PhiloxKeys k;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    k.k0[r] = static_cast<uint32_t>(seed) + static_cast<uint32_t>(r) * 0x9E3779B9u;
+    k.k1[r] = static_cast<uint32_t>(seed >> 32) + static_cast<uint32_t>(r) * 0xBB67AE85u;
+  }
+  return k;
+}
+// counter (lo32 g, hi32 g, tag, 0)
+__device__ __forceinline__ uint4 philox_keyed(uint64_t g, uint32_t tag, const PhiloxKeys& k) {
+  uint4 c = make_uint4(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), tag, 0u);
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c.x;
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c.z;
+    c = make_uint4(static_cast<uint32_t>(p1 >> 32) ^ c.y ^ k.k0[r], static_cast<uint32_t>(p1),
+                   static_cast<uint32_t>(p0 >> 32) ^ c.w ^ k.k1[r], static_cast<uint32_t>(p0));
+  }
+  return c;
+}
+
 // The 128 random bits of the 16 elements e with floor(e/16) = blk (word k
 // for elements 16 blk + 4k .. 16 blk + 4k + 3): counter (lo32(offset+blk),
 // hi32(offset+blk), tag, 0), key (lo32(seed), hi32(seed)).

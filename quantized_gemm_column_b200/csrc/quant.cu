@@ -71,6 +71,16 @@ struct Raw16 {
 };
 
 template <bool kBf16>
+__device__ __forceinline__ void load16_ptr(const uint8_t* ptr, bool active, Raw16<kBf16>& r) {
+#pragma unroll
+  for (int i = 0; i < (kBf16 ? 2 : 4); ++i) r.w[i] = make_uint4(0, 0, 0, 0);
+  if (!active) return;
+  const uint4* q = reinterpret_cast<const uint4*>(ptr);
+#pragma unroll
+  for (int i = 0; i < (kBf16 ? 2 : 4); ++i) r.w[i] = __ldcs(q + i);
+}
+
+template <bool kBf16>
 __device__ __forceinline__ void load16(const void* base, int64_t idx, bool active, Raw16<kBf16>& r) {
 #pragma unroll
   for (int i = 0; i < (kBf16 ? 2 : 4); ++i) r.w[i] = make_uint4(0, 0, 0, 0);
@@ -113,9 +123,9 @@ __device__ __forceinline__ void fill_rscale_table(float* r_tab, float g_enc) {
 // Quantize one 16-element block: returns the 16 packed codes (element 2k in
 // the low nibble of byte k) and the block's E4M3 scale code in *S.
 // `blk` = element index of the block's first element / 16 (its Philox counter).
+// `rw` holds the block's four random words (stochastic rounding only).
 template <bool kSR>
-__device__ __forceinline__ uint2 quant16(const float (&xr)[16], float g_enc, const float* r_tab,
-                                         uint64_t seed, uint64_t offset, uint32_t tag, uint64_t blk,
+__device__ __forceinline__ uint2 quant16(const float (&xr)[16], float g_enc, const float* r_tab, uint4 rw,
                                          uint32_t* S_out) {
   float am = fmax3(fabsf(xr[0]), fabsf(xr[1]), fabsf(xr[2]));
 #pragma unroll
@@ -128,7 +138,7 @@ __device__ __forceinline__ uint2 quant16(const float (&xr)[16], float g_enc, con
   for (int t = 0; t < 16; t += 2) fmul2(xr[t], xr[t + 1], r, y[t], y[t + 1]);
   uint2 packed;
   if (kSR) {
-    const uint4 w = philox_block(seed, offset, tag, blk);
+    const uint4 w = rw;
     packed.x = e2m1x4_sr(y[0], y[1], y[2], y[3], w.x) | (e2m1x4_sr(y[4], y[5], y[6], y[7], w.y) << 16);
     packed.y = e2m1x4_sr(y[8], y[9], y[10], y[11], w.z) | (e2m1x4_sr(y[12], y[13], y[14], y[15], w.w) << 16);
   } else {
@@ -289,8 +299,9 @@ __device__ void quantize_mean_window(const QuantParams& p, float g_enc, const fl
       for (int t = 0; t < 16; ++t) x[t] = 0.0f;
     }
     uint32_t S;
-    const uint2 packed = quant16<kSR>(x, g_enc, r_tab, p.seed, p.offset, p.tag_mu,
-                                      static_cast<uint64_t>(col0 / 16), &S);
+    const uint4 rw = kSR ? philox_block(p.seed, p.offset, p.tag_mu, static_cast<uint64_t>(col0 / 16))
+                         : make_uint4(0u, 0u, 0u, 0u);
+    const uint2 packed = quant16<kSR>(x, g_enc, r_tab, rw, &S);
     const uint32_t sw = gather_scale_word(S);
     if (active) {
       if (writer) {
@@ -393,26 +404,35 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(const QuantParams 
   if (!has_work) return;
   const uint32_t n_kb64 = static_cast<uint32_t>(p.K / 64);
 
-  for (; r0 < p.rows; r0 += row_step) {
-    // the next rows of this warp are loaded while these are quantized
-    const int64_t rn = r0 + row_step;
-    Raw16<kBf16> nxt[kRowsPerIter];
-#pragma unroll
-    for (int i = 0; i < kRowsPerIter; ++i) load16<kBf16>(p.X, (rn + i) * p.K + col0, active && rn + i < p.rows, nxt[i]);
+  // Rows r0 and r0 + 1 of each iteration; the next iteration's rows are loaded
+  // into the other buffer while these are quantized (two buffers, unrolled
+  // by two, so no register copies).  Pointers and the Philox counter advance
+  // by constant strides.
+  const int elem = kBf16 ? 2 : 4;
+  const uint8_t* xp = static_cast<const uint8_t*>(p.X) + (r0 * p.K + col0) * elem;
+  const int64_t x_row = p.K * elem, x_step = row_step * p.K * elem;
+  uint8_t* cp = p.codes + r0 * (p.K / 2) + col0 / 2;
+  const int64_t c_row = p.K / 2, c_step = row_step * (p.K / 2);
+  uint64_t g = p.offset + static_cast<uint64_t>((r0 * p.K + col0) / 16);
+  const uint64_t g_row = static_cast<uint64_t>(p.K / 16), g_step = static_cast<uint64_t>(row_step * (p.K / 16));
+  const uint32_t c16 = static_cast<uint32_t>(col0 / 16);
+  PhiloxKeys keys;
+  if (kSR) keys = philox_keys(p.seed);
+
+  auto do_rows = [&](const Raw16<kBf16> (&buf)[kRowsPerIter]) {
 #pragma unroll
     for (int i = 0; i < kRowsPerIter; ++i) {
       const int64_t r = r0 + i;
       float xr[16];
-      sub_mu16<kBf16>(cur[i], mu, xr);
+      sub_mu16<kBf16>(buf[i], mu, xr);
+      const uint4 rw = kSR ? philox_keyed(g + i * g_row, p.tag, keys) : make_uint4(0u, 0u, 0u, 0u);
       uint32_t S;
-      const uint2 packed = quant16<kSR>(xr, g_enc, r_tab, p.seed, p.offset, p.tag,
-                                        static_cast<uint64_t>((r * p.K + col0) / 16), &S);
+      const uint2 packed = quant16<kSR>(xr, g_enc, r_tab, rw, &S);
       const uint32_t sw = gather_scale_word(S);
       if (active && r < p.rows) {
-        *reinterpret_cast<uint2*>(p.codes + r * (p.K / 2) + col0 / 2) = packed;
+        *reinterpret_cast<uint2*>(cp + i * c_row) = packed;
         if ((lane & 3) == 0)
-          *reinterpret_cast<uint32_t*>(p.scales + scale_offset(static_cast<uint64_t>(r),
-                                                               static_cast<uint32_t>(col0 / 16), n_kb64)) = sw;
+          *reinterpret_cast<uint32_t*>(p.scales + scale_offset(static_cast<uint64_t>(r), c16, n_kb64)) = sw;
         if (p.xr_debug) {
           float4* d = reinterpret_cast<float4*>(p.xr_debug + r * p.K + col0);
 #pragma unroll
@@ -420,8 +440,23 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(const QuantParams 
         }
       }
     }
+    r0 += row_step;
+    xp += x_step;
+    cp += c_step;
+    g += g_step;
+  };
+  auto load_rows = [&](Raw16<kBf16> (&buf)[kRowsPerIter]) {   // the rows after the current ones
 #pragma unroll
-    for (int i = 0; i < kRowsPerIter; ++i) cur[i] = nxt[i];
+    for (int i = 0; i < kRowsPerIter; ++i)
+      load16_ptr<kBf16>(xp + x_step + i * x_row, active && r0 + row_step + i < p.rows, buf[i]);
+  };
+  Raw16<kBf16> nxt[kRowsPerIter];
+  while (r0 < p.rows) {
+    load_rows(nxt);
+    do_rows(cur);
+    if (r0 >= p.rows) break;
+    load_rows(cur);
+    do_rows(nxt);
   }
 }
 
