@@ -8,8 +8,10 @@
 // added to every output row:
 //   Y[i, j] = g_dec(A) g_dec(B) * acc[i, j] + bias[j].
 //
-// Persistent kernel, one CTA per SM, output tiles handed out round-robin;
-// K staged 256 elements (128 bytes per row, 128-byte swizzle) at a time.
+// Persistent kernel, one CTA per SM; each CTA takes a contiguous run of
+// output tiles, M fastest, so consecutive tiles share their B (weight)
+// columns.  K is staged 256 elements (128 bytes per row, 128-byte swizzle) at
+// a time.
 //   warp 0     : allocates tensor memory; one thread copies the scale atoms
 //                shared -> tensor memory (tcgen05.cp 32x128b, replicated into
 //                the four lane quarters) and issues
@@ -18,10 +20,18 @@
 //                tile, the B code tile, and A's and B's 512-byte scale atoms
 //                (2-D copies over the atom array, out-of-range atoms read as
 //                zero).  A thread issues one bulk copy at a time, so the
-//                four copies of a stage go out from four warps;
-//   warps 5..  : epilogue -- tcgen05.ld of the accumulator (each warp one
-//                32-lane quarter and a run of columns), alpha * acc + bias,
-//                convert, write a 128-byte-swizzled staging tile, TMA-store it.
+//                copies of a stage go out from separate warps;
+//   warps 5..  : epilogue -- the tile's bias row is fetched into registers
+//                while the mainloop runs; tcgen05.ld of the accumulator (each
+//                warp one 32-lane quarter and a run of columns), alpha * acc +
+//                bias, convert, a 128-byte-swizzled staging tile, TMA store.
+//
+// Resident weight scales (bf16 output, K <= 1792): the scale copies cost as
+// much tensor-pipe time as the MMAs they feed, and B's scales repeat for
+// every tile of a column block.  So when all of K's B scales fit in tensor
+// memory beside the accumulator, warp 4 loads them once per column block into
+// a shared buffer, the MMA thread copies them into tensor memory once, and a
+// stage then needs only A's four scale copies.
 #include "device.cuh"
 #include "internal.h"
 
@@ -29,11 +39,11 @@ namespace avr {
 
 // Two tile shapes:
 //  BN = 256 (bf16 output): MMAs of M 128 x N 256, the shape that reaches the
-//    tensor cores' rate; 3 stages; one accumulator of 256 columns (the scale
-//    buffers take the rest of tensor memory), drained by 8 epilogue warps into
-//    a 64 KB staging tile.
+//    tensor cores' rate; 3 stages; one accumulator of 256 columns, released to
+//    the MMA thread as soon as its last tcgen05.ld lands; the 64 KB output
+//    tile leaves through a 32 KB staging buffer in two rounds.
 //  BN = 128 (fp32 output): 4 stages; two accumulators, so the epilogue
-//    overlaps the next tile's mainloop.
+//    overlaps the next tile's mainloop; a 64 KB staging tile.
 template <int BN, bool kBf16Out>
 struct GemmCfg {
   static constexpr int kBM = 128, kBN = BN;
@@ -54,18 +64,25 @@ struct GemmCfg {
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
   static constexpr int kOutElem = kBf16Out ? 2 : 4;
   static constexpr int kBoxCols = 128 / kOutElem;          // columns per 128-byte swizzled store box
-  static constexpr int kBoxes = kBN / kBoxCols;
-  static constexpr int kStageOutBytes = kBM * kBN * kOutElem;
-  static constexpr int kOutOffset = kStages * kStageBytes;
-  static constexpr int kBarOffset = kOutOffset + kStageOutBytes;
-  // dynamic shared memory starts 1024-aligned when a kernel has no static
-  // shared memory; the kernel checks it and refuses to run otherwise
-  static constexpr int kSmemBytes = kBarOffset + 128;
+  static constexpr int kOutRounds = kBf16Out ? 2 : 1;      // staging rounds per tile
+  static constexpr int kStageOutBytes = kBM * kBN * kOutElem / kOutRounds;
+  static constexpr int kBoxesPerRound = kBN / kBoxCols / kOutRounds;
+  // resident B scales (bf16 output only): up to kResMaxKb k-blocks
   static constexpr int kAccCols = kBN;
   static constexpr int kSfaCols = kKbPerStage * 4;
   static constexpr int kSfbCols = kKbPerStage * (kBN / 32);
-  static constexpr int kSfCol = kAccBufs * kAccCols;         // 2 scale buffers after the accumulators
+  static constexpr int kSfCol = kAccBufs * kAccCols;       // scale buffers after the accumulators
   static constexpr int kTmemCols = 512;
+  static constexpr int kResSfbCol = kSfCol + 2 * kSfaCols;  // resident mode: SFA x2, then all of SFB
+  static constexpr int kResMaxKb = kBf16Out ? (kTmemCols - kResSfbCol) / (kBN / 32) : 0;
+  static constexpr int kResMaxStages = kResMaxKb / kKbPerStage;
+  static constexpr int kResBytes = kResMaxStages * kSfbBytes;
+  static constexpr int kOutOffset = kStages * kStageBytes;
+  static constexpr int kResOffset = kOutOffset + kStageOutBytes;
+  static constexpr int kBarOffset = kResOffset + kResBytes;
+  // dynamic shared memory starts 1024-aligned when a kernel has no static
+  // shared memory; the kernel checks it and refuses to run otherwise
+  static constexpr int kSmemBytes = kBarOffset + 128;
   static_assert(kSfCol + 2 * (kSfaCols + kSfbCols) <= kTmemCols, "tensor memory budget");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   // instruction descriptor: E2M1 A and B (format 1), UE4M3 scales, K-major
@@ -76,13 +93,24 @@ struct GemmCfg {
 
 struct GemmParams {
   int64_t M, N, K;
-  int tiles_n, num_tiles;
-  const uint8_t* sfa;
-  const uint8_t* sfb;
+  int tiles_m, num_tiles;
+  int sfb_resident;       // 1: B's scales for all of K live in tensor memory
   const float* gdec_a;
   const float* gdec_b;
   const float* bias;
   uint32_t* status;
+};
+
+// The contiguous run of tiles [first, first + count) of this CTA; tile t is
+// (m block t mod tiles_m, n block t / tiles_m).
+struct TileRun {
+  int first, count;
+  __device__ __forceinline__ TileRun(int num_tiles) {
+    const int q = num_tiles / static_cast<int>(gridDim.x), r = num_tiles % static_cast<int>(gridDim.x);
+    const int b = static_cast<int>(blockIdx.x);
+    first = b * q + (b < r ? b : r);
+    count = q + (b < r ? 1 : 0);
+  }
 };
 
 template <int BN, bool kBf16Out>
@@ -103,14 +131,19 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
   uint8_t* sSfa = sB + Cfg::kStages * Cfg::kBBytes;
   uint8_t* sSfb = sSfa + Cfg::kStages * Cfg::kSfaBytes;
   uint8_t* sOut = smem + Cfg::kOutOffset;
+  uint8_t* sRes = smem + Cfg::kResOffset;      // resident B scales, one kSfbBytes slab per stage of K
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOffset);
   uint64_t* empty = full + Cfg::kStages;
   uint64_t* acc_full = empty + Cfg::kStages;   // [kAccBufs]
   uint64_t* acc_empty = acc_full + 2;          // [kAccBufs]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* res_full = acc_empty + 2;          // resident B scales loaded
+  uint64_t* res_empty = res_full + 1;          // resident B scales copied to tensor memory
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(res_empty + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_kst = static_cast<int>((p.K + Cfg::kStageK - 1) / Cfg::kStageK);
+  const bool res = p.sfb_resident != 0;
+  const TileRun run(p.num_tiles);
 
   if (threadIdx.x == 0) {
     prefetch_tensormap(&map_a);
@@ -119,13 +152,15 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
     prefetch_tensormap(&map_sfb);
     prefetch_tensormap(&map_y);
     for (int s = 0; s < Cfg::kStages; ++s) {
-      mbar_init(&full[s], 4);                  // one arrival per producer warp
+      mbar_init(&full[s], res ? 3 : 4);        // one arrival per per-stage producer warp
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < Cfg::kAccBufs; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], Cfg::kEpiWarps);   // one arrival per epilogue warp
     }
+    mbar_init(res_full, 1);
+    mbar_init(res_empty, 1);
     fence_mbarrier_init();
   }
   if (warp == 0) {
@@ -143,31 +178,50 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
     if (lane == 0) {
       // ---------------- producers: warp 1 A, 2 B, 3 A's scales, 4 B's scales ----------------
       const int role = warp - 1;
-      int it = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-        const int32_t m0 = (tile / p.tiles_n) * Cfg::kBM;
-        const int32_t n0 = (tile % p.tiles_n) * Cfg::kBN;
-        for (int ks = 0; ks < n_kst; ++ks, ++it) {
-          const int st = it % Cfg::kStages;
-          if (it >= Cfg::kStages &&
-              !mbar_wait(&empty[st], static_cast<uint32_t>((it / Cfg::kStages) - 1) & 1u, p.status)) {
-            ok = false;
-            break;
-          }
-          if (role == 0) {
-            mbar_arrive_expect_tx(&full[st], Cfg::kABytes);
-            tma_load_2d(sA + st * Cfg::kABytes, &map_a, &full[st], ks * Cfg::kRowBytes, m0);
-          } else if (role == 1) {
-            mbar_arrive_expect_tx(&full[st], Cfg::kBBytes);
-            tma_load_2d(sB + st * Cfg::kBBytes, &map_b, &full[st], ks * Cfg::kRowBytes, n0);
-          } else if (role == 2) {
-            // 4 atoms (2 KB) of the tile's 128-row group, as 256 eight-byte elements
-            mbar_arrive_expect_tx(&full[st], Cfg::kSfaBytes);
-            tma_load_2d(sSfa + st * Cfg::kSfaBytes, &map_sfa, &full[st], ks * 256, m0 / 128);
-          } else {
-            mbar_arrive_expect_tx(&full[st], Cfg::kSfbBytes);
-            tma_load_2d(sSfb + st * Cfg::kSfbBytes, &map_sfb, &full[st], ks * 256, n0 / 128);
+      if (role == 3 && res) {
+        // B's scales for all of K, once per column block
+        int n_prev = -1, uses = 0;
+        for (int i = 0; i < run.count; ++i) {
+          const int n_blk = (run.first + i) / p.tiles_m;
+          if (n_blk == n_prev) continue;
+          n_prev = n_blk;
+          if (uses >= 1 && !mbar_wait(res_empty, static_cast<uint32_t>(uses - 1) & 1u, p.status)) break;
+          ++uses;
+          mbar_arrive_expect_tx(res_full, static_cast<uint32_t>(n_kst * Cfg::kSfbBytes));
+          for (int ks = 0; ks < n_kst; ++ks)
+            tma_load_2d(sRes + ks * Cfg::kSfbBytes, &map_sfb, res_full, ks * 256, n_blk * (Cfg::kBN / 128));
+        }
+      } else {
+        uint32_t st = 0, ph = 0;
+        int it = 0;
+        bool ok = true;
+        for (int i = 0; i < run.count && ok; ++i) {
+          const int tile = run.first + i;
+          const int32_t m0 = (tile % p.tiles_m) * Cfg::kBM;
+          const int32_t n0 = (tile / p.tiles_m) * Cfg::kBN;
+          for (int ks = 0; ks < n_kst; ++ks, ++it) {
+            if (it >= Cfg::kStages && !mbar_wait(&empty[st], ph ^ 1u, p.status)) {
+              ok = false;
+              break;
+            }
+            if (role == 0) {
+              mbar_arrive_expect_tx(&full[st], Cfg::kABytes);
+              tma_load_2d(sA + st * Cfg::kABytes, &map_a, &full[st], ks * Cfg::kRowBytes, m0);
+            } else if (role == 1) {
+              mbar_arrive_expect_tx(&full[st], Cfg::kBBytes);
+              tma_load_2d(sB + st * Cfg::kBBytes, &map_b, &full[st], ks * Cfg::kRowBytes, n0);
+            } else if (role == 2) {
+              // 4 atoms (2 KB) of the tile's 128-row group, as 256 eight-byte elements
+              mbar_arrive_expect_tx(&full[st], Cfg::kSfaBytes);
+              tma_load_2d(sSfa + st * Cfg::kSfaBytes, &map_sfa, &full[st], ks * 256, m0 / 128);
+            } else {
+              mbar_arrive_expect_tx(&full[st], Cfg::kSfbBytes);
+              tma_load_2d(sSfb + st * Cfg::kSfbBytes, &map_sfb, &full[st], ks * 256, n0 / 128);
+            }
+            if (++st == Cfg::kStages) {
+              st = 0;
+              ph ^= 1u;
+            }
           }
         }
       }
@@ -179,33 +233,51 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
       // it is late with idles the tensor pipe, so the loop keeps its
       // bookkeeping to increments (stage, phase and scale-buffer counters)
       // and issues a full stage's copies and MMAs unrolled, with descriptors
-      // advanced by constants.
+      // advanced by constants (16-byte units: +32 per 512-byte scale atom, +2
+      // per 32-byte k-block step).  A tile's first copies go out before the
+      // wait for its accumulator: they write the scale area, not the
+      // accumulator, and so overlap the previous tile's epilogue.
       uint32_t st = 0, ph = 0, sf_buf = 0;
       const int n_full = static_cast<int>(p.K / Cfg::kStageK);               // stages of kKbPerStage k-blocks
       const int tail_kb = static_cast<int>((p.K % Cfg::kStageK) / 64);       // k-blocks of a last, partial stage
-      // a tile's first scale copies go out before the wait for its accumulator
-      // (they write the scale area, not the accumulator), so they overlap the
-      // previous tile's epilogue
+      const uint32_t sfa_stride = res ? Cfg::kSfaCols : Cfg::kSfaCols + Cfg::kSfbCols;
       auto wait_acc_empty = [&](int ab, int use) {
         if (!mbar_wait_poll(&acc_empty[ab], static_cast<uint32_t>(use - 1) & 1u, p.status)) return false;
         tc_fence_after();
         return true;
       };
-      int tcount = 0;
+      int n_prev = -1, res_uses = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tcount) {
-        const int ab = tcount % Cfg::kAccBufs;
-        const int use = tcount / Cfg::kAccBufs;
+      for (int i = 0; i < run.count && ok; ++i) {
+        const int tile = run.first + i;
+        const int ab = i % Cfg::kAccBufs;
+        const int use = i / Cfg::kAccBufs;
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(ab * Cfg::kAccCols);
+        if (res && tile / p.tiles_m != n_prev) {
+          // a new column block: its B scales, all of K, into tensor memory
+          n_prev = tile / p.tiles_m;
+          if (!mbar_wait(res_full, static_cast<uint32_t>(res_uses) & 1u, p.status)) break;
+          tc_fence_after();
+          const uint64_t r_d = smem_desc(smem_u32(sRes), 0, 128, kLayoutSwizzleNone);
+          for (int ks = 0; ks < n_kst; ++ks)
+#pragma unroll
+            for (int kb = 0; kb < Cfg::kKbPerStage; ++kb)
+#pragma unroll
+              for (int g = 0; g < Cfg::kBN / 128; ++g)
+                tc_cp_32x128b_warpx4(tmem + Cfg::kResSfbCol + (Cfg::kBN / 32) * (ks * Cfg::kKbPerStage + kb) + 4 * g,
+                                     r_d + static_cast<uint64_t>(32 * ((ks * (Cfg::kBN / 128) + g) * Cfg::kKbPerStage + kb)));
+          tc_commit(res_empty);
+          ++res_uses;
+        }
         for (int ks = 0; ks < n_kst; ++ks) {
           if (!mbar_wait(&full[st], ph, p.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sfa_t = tmem + Cfg::kSfCol + sf_buf * (Cfg::kSfaCols + Cfg::kSfbCols);
-          const uint32_t sfb_t = sfa_t + Cfg::kSfaCols;
-          // 16-byte-unit descriptor fields: +32 per 512-byte scale atom, +2 per 32-byte k-block step
+          const uint32_t sfa_t = tmem + Cfg::kSfCol + sf_buf * sfa_stride;
+          const uint32_t sfb_t = res ? tmem + Cfg::kResSfbCol + (Cfg::kBN / 32) * (ks * Cfg::kKbPerStage)
+                                     : sfa_t + Cfg::kSfaCols;
           const uint64_t sfa_d = smem_desc(smem_u32(sSfa + st * Cfg::kSfaBytes), 0, 128, kLayoutSwizzleNone);
           const uint64_t sfb_d = smem_desc(smem_u32(sSfb + st * Cfg::kSfbBytes), 0, 128, kLayoutSwizzleNone);
           const uint64_t a0 = smem_desc(smem_u32(sA + st * Cfg::kABytes), 16, Cfg::kSbo, Cfg::kSwizzle);
@@ -214,10 +286,12 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
 #pragma unroll
             for (int kb = 0; kb < Cfg::kKbPerStage; ++kb) {
               tc_cp_32x128b_warpx4(sfa_t + 4 * kb, sfa_d + static_cast<uint64_t>(32 * kb));
+              if (!res) {
 #pragma unroll
-              for (int g = 0; g < Cfg::kBN / 128; ++g)
-                tc_cp_32x128b_warpx4(sfb_t + (Cfg::kBN / 32) * kb + 4 * g,
-                                     sfb_d + static_cast<uint64_t>(32 * (g * Cfg::kKbPerStage + kb)));
+                for (int g = 0; g < Cfg::kBN / 128; ++g)
+                  tc_cp_32x128b_warpx4(sfb_t + (Cfg::kBN / 32) * kb + 4 * g,
+                                       sfb_d + static_cast<uint64_t>(32 * (g * Cfg::kKbPerStage + kb)));
+              }
             }
             if (ks == 0 && use >= 1 && !wait_acc_empty(ab, use)) {
               ok = false;
@@ -230,9 +304,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
           } else {
             for (int kb = 0; kb < tail_kb; ++kb) {
               tc_cp_32x128b_warpx4(sfa_t + 4 * kb, sfa_d + static_cast<uint64_t>(32 * kb));
-              for (int g = 0; g < Cfg::kBN / 128; ++g)
-                tc_cp_32x128b_warpx4(sfb_t + (Cfg::kBN / 32) * kb + 4 * g,
-                                     sfb_d + static_cast<uint64_t>(32 * (g * Cfg::kKbPerStage + kb)));
+              if (!res)
+                for (int g = 0; g < Cfg::kBN / 128; ++g)
+                  tc_cp_32x128b_warpx4(sfb_t + (Cfg::kBN / 32) * kb + 4 * g,
+                                       sfb_d + static_cast<uint64_t>(32 * (g * Cfg::kKbPerStage + kb)));
             }
             if (ks == 0 && use >= 1 && !wait_acc_empty(ab, use)) {
               ok = false;
@@ -260,11 +335,11 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
     const int r = 32 * q + lane;               // row of the tile
     const bool leader = (ew == 0 && lane == 0);
     const float alpha = __ldg(p.gdec_a) * __ldg(p.gdec_b);
-    int tcount = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
-      const int ab = tcount % Cfg::kAccBufs;
-      const int64_t m0 = static_cast<int64_t>(tile / p.tiles_n) * Cfg::kBM;
-      const int64_t n0 = static_cast<int64_t>(tile % p.tiles_n) * Cfg::kBN;
+    for (int i = 0; i < run.count; ++i) {
+      const int tile = run.first + i;
+      const int ab = i % Cfg::kAccBufs;
+      const int64_t m0 = static_cast<int64_t>(tile % p.tiles_m) * Cfg::kBM;
+      const int64_t n0 = static_cast<int64_t>(tile / p.tiles_m) * Cfg::kBN;
       // lane l holds the bias of column 32 cc + l of each of its chunks, fetched
       // before the accumulator is ready so the load hides behind the mainloop
       float bias_l[4];
@@ -274,21 +349,19 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
         bias_l[c] = (p.bias != nullptr && col < p.N) ? __ldg(p.bias + col) : 0.0f;
       }
       uint32_t okw = 0;
-      if (lane == 0) okw = mbar_wait_poll(&acc_full[ab], static_cast<uint32_t>(tcount / Cfg::kAccBufs) & 1u, p.status) ? 1u : 0u;
+      if (lane == 0) okw = mbar_wait_poll(&acc_full[ab], static_cast<uint32_t>(i / Cfg::kAccBufs) & 1u, p.status) ? 1u : 0u;
       const bool ok = __shfl_sync(0xFFFFFFFFu, okw, 0) != 0;
       // all epilogue threads agree, so the .sync.aligned loads below run in
       // every lane of every warp or in none
       if (named_barrier_or(1, kEpiThreads, !ok)) break;
       tc_fence_after();
-      // the previous tile's store must have read the staging tile
-      if (leader) bulk_wait_group_read<0>();
-      named_barrier(1, kEpiThreads);
-      // one 32-column chunk: alpha * acc + bias, converted, into the staging tile
+      const uint32_t t_row = tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(ab * Cfg::kAccCols);
+      // chunk c (of this warp's four) = alpha * acc + bias, converted, into the staging buffer
       auto emit = [&](int c, const uint32_t (&v)[32]) {
         const int cc = 4 * h + c;              // 32-column chunk of the tile
         if (kBf16Out) {
-          // 32 bf16 = 64 bytes = four 16-byte pieces of row r in box cc/2
-          uint8_t* box = sOut + (cc >> 1) * (Cfg::kBM * 128);
+          // 32 bf16 = 64 bytes = four 16-byte pieces of row r in box h of this round
+          uint8_t* box = sOut + h * (Cfg::kBM * 128);
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             uint32_t w[4];
@@ -317,9 +390,26 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
           }
         }
       };
+      // the staging buffer is free once the previous store has read it
+      auto staging_free = [&]() {
+        if (leader) bulk_wait_group_read<0>();
+        named_barrier(1, kEpiThreads);
+      };
+      auto store_round = [&](int first_box_col) {   // make the round visible to the TMA engine, store it
+        fence_proxy_async_smem();
+        named_barrier(1, kEpiThreads);
+        if (leader) {
+#pragma unroll
+          for (int bx = 0; bx < Cfg::kBoxesPerRound; ++bx) {
+            const int64_t col = n0 + first_box_col + bx * (kBf16Out ? 128 : Cfg::kBoxCols);
+            if (col < p.N)
+              tma_store_2d(&map_y, sOut + bx * (Cfg::kBM * 128), static_cast<int32_t>(col), static_cast<int32_t>(m0));
+          }
+          bulk_commit_group();
+        }
+      };
       // two chunks per tensor-memory round trip; the accumulator goes back to
-      // the MMA warp as soon as the last two are in registers
-      const uint32_t t_row = tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(ab * Cfg::kAccCols);
+      // the MMA thread as soon as the last two are in registers
 #pragma unroll
       for (int c2 = 0; c2 < 4; c2 += 2) {
         uint32_t v0[32], v1[32];
@@ -331,20 +421,13 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[ab]);
         }
+        if (kBf16Out || c2 == 0) staging_free();
         emit(c2, v0);
         emit(c2 + 1, v1);
+        // bf16: one round per chunk pair (box h holds columns 128 h + 64 (c2/2) .. +63)
+        if (kBf16Out) store_round(64 * (c2 / 2));
       }
-      // staging tile complete and visible to the TMA engine: store it
-      fence_proxy_async_smem();
-      named_barrier(1, kEpiThreads);
-      if (leader) {
-#pragma unroll
-        for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-          if (n0 + bx * Cfg::kBoxCols < p.N)
-            tma_store_2d(&map_y, sOut + bx * (Cfg::kBM * 128), static_cast<int32_t>(n0 + bx * Cfg::kBoxCols),
-                         static_cast<int32_t>(m0));
-        bulk_commit_group();
-      }
+      if (!kBf16Out) store_round(0);
     }
     if (leader) bulk_wait_group_all();
   }
@@ -384,10 +467,10 @@ static cudaError_t launch_gemm_t(const GemmArgs& a, cudaStream_t s, bool pdl) {
   p.M = a.M;
   p.N = a.N;
   p.K = a.K;
-  p.tiles_n = static_cast<int>((a.N + Cfg::kBN - 1) / Cfg::kBN);
-  p.num_tiles = static_cast<int>((a.M + Cfg::kBM - 1) / Cfg::kBM) * p.tiles_n;
-  p.sfa = a.a_scales;
-  p.sfb = a.b_scales;
+  p.tiles_m = static_cast<int>((a.M + Cfg::kBM - 1) / Cfg::kBM);
+  p.num_tiles = p.tiles_m * static_cast<int>((a.N + Cfg::kBN - 1) / Cfg::kBN);
+  const int64_t n_kst = (a.K + Cfg::kStageK - 1) / Cfg::kStageK;
+  p.sfb_resident = (Cfg::kResMaxStages > 0 && n_kst <= Cfg::kResMaxStages) ? 1 : 0;
   p.gdec_a = a.a_gdec;
   p.gdec_b = a.b_gdec;
   p.bias = a.bias;
