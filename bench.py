@@ -177,6 +177,26 @@ def run_reference(args, rank, world):
 
 
 # ---------------------------------------------------------------------------
+# multi-rank plumbing (replicas; the only collective is this timing reduction)
+# ---------------------------------------------------------------------------
+def max_over_ranks(values, device):
+    """Element-wise maximum of `values` over all ranks (identity on one rank).
+    Every rank must call it at the same point; it runs outside the timed region."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def job_value(flops_per_step, world, step_ms):
+    """Whole-job throughput (TFLOP/s): every rank runs its own step of
+    flops_per_step; the slowest rank's step time counts."""
+    return flops_per_step * world / (step_ms * 1e-3) / 1e12
+
+
+# ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
 def run_gpu(args, rank, world, local_rank):
@@ -279,12 +299,9 @@ def run_gpu(args, rank, world, local_rank):
     if st:
         raise RuntimeError(f"device status {st} in the timed region")
 
-    ms_t = torch.tensor([ms, ms_van], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms, ms_van = float(ms_t[0]), float(ms_t[1])
+    ms, ms_van = max_over_ranks([ms, ms_van], dev)
     step_ms = ms / args.steps
-    value = FLOPS_PER_STEP * world / (step_ms * 1e-3) / 1e12
+    value = job_value(FLOPS_PER_STEP, world, step_ms)
 
     # per-kernel-group timing (same stream, events around n launches each)
     xr = api.NVFP4Tensor(L, M, dev)
@@ -365,10 +382,8 @@ def run_gpu(args, rank, world, local_rank):
             e2e_step(i)
         b.record(stream)
         torch.cuda.synchronize(dev)
-    e2e_ms = torch.tensor([a.elapsed_time(b) / e2e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_val = FLOPS_PER_STEP * world / (float(e2e_ms) * 1e-3) / 1e12
+    e2e_ms = max_over_ranks([a.elapsed_time(b) / e2e_steps], dev)[0]
+    e2e_val = job_value(FLOPS_PER_STEP, world, e2e_ms)
     h2d = (X0.numel() + D0.numel()) * 2
     d2h = (Y.numel() + dX.numel()) * 2
 
