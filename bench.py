@@ -177,6 +177,39 @@ def run_reference(args, rank, world):
 
 
 # ---------------------------------------------------------------------------
+# measured DRAM traffic (ncu), valid only for the kernel sources it was taken on
+# ---------------------------------------------------------------------------
+KERNEL_SOURCES = ["colreduce.cu", "quant.cu", "gemm.cu", "device.cuh", "internal.h"]
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "traffic_qkv_step.md")
+
+
+def kernel_digest():
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "quantized_gemm_column_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(key):
+    """DRAM bytes per step of a kernel group from the committed ncu summary,
+    or None if the summary is missing or was taken on other kernel sources."""
+    try:
+        fields = {}
+        for line in open(TRAFFIC_PROFILE):
+            line = line.strip()
+            if line.startswith("traffic-") and ":" in line:
+                k, v = line.split(":", 1)
+                fields[k.strip()] = v.strip()
+        if fields.get("traffic-digest") != kernel_digest():
+            return None
+        return int(fields[f"traffic-{key}-bytes-per-step"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------------
 # multi-rank plumbing (replicas; the only collective is this timing reduction)
 # ---------------------------------------------------------------------------
 def max_over_ranks(values, device):
@@ -349,12 +382,16 @@ def run_gpu(args, rank, world, local_rank):
     if gemm_share >= 0.5:
         roof = {"bound": "tensor", "kernel": "gemm_nvfp4_kernel (fwd + dgrad)",
                 "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
-                "frac": gemm_tflops / fp4_peak, "traffic": None,
+                "frac": gemm_tflops / fp4_peak, "traffic": measured_traffic("gemm"),
+                "traffic_unit": "DRAM bytes per step (fwd + dgrad launches)",
                 "peak_source": f"{peak_src} bf16 x 4 (nominal FP4:BF16 ratio)"}
     else:
         roof = {"bound": "hbm", "kernel": "colreduce_kernel + quant_kernel (split-quant, X and dY)",
                 "achieved": sq_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": sq_gbs / hbm_peak,
-                "traffic": None, "peak_source": f"{peak_src} HBM copy"}
+                "traffic": measured_traffic("split-quant"),
+                "traffic_unit": "DRAM bytes per step (4 launches: reduce and quantize, X and dY)",
+                "algorithmic_bytes_per_step": sq_bytes(L, M) + sq_bytes(L, N),
+                "peak_source": f"{peak_src} HBM copy"}
 
     # end to end through the public API with host buffers
     Xh = X0.pin_memory()

@@ -83,3 +83,17 @@ def test_reference_arm_under_torchrun(tmp_path):
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_measured_traffic_follows_kernel_sources(tmp_path, monkeypatch):
+    """The roofline's DRAM traffic comes from the committed ncu summary only
+    while the kernel sources hash to the digest it records."""
+    import bench
+    prof = tmp_path / "traffic.md"
+    prof.write_text(f"    traffic-digest: {bench.kernel_digest()}\n"
+                    "    traffic-split-quant-bytes-per-step: 123\n")
+    monkeypatch.setattr(bench, "TRAFFIC_PROFILE", str(prof))
+    assert bench.measured_traffic("split-quant") == 123
+    assert bench.measured_traffic("gemm") is None
+    prof.write_text("    traffic-digest: 0000000000000000\n    traffic-split-quant-bytes-per-step: 123\n")
+    assert bench.measured_traffic("split-quant") is None
