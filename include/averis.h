@@ -19,6 +19,9 @@
  *   [GS2]   gist.science technical summary, section 2 "Il Metodo Proposto:
  *           Averis": X_R = X - 1 mu_X^T, mean and residual quantized
  *           separately, forward and backward recombined.
+ *   [R7.2]  Lighthouse review page, section 七 "对我们的启示", under "实践建议",
+ *           item 2: monitor the mean-energy ratio
+ *           R = ||mu||_2 / sqrt(E||x||^2 / N) as a training-stability signal.
  *
  * Readings where the pages are silent (the same readings the CPU oracle
  * follows): 16-element blocks along the contraction axis with unsigned E4M3
@@ -124,11 +127,28 @@ const char* averis_status_string(avr_status status);
  *   grad = 0 for activations X (random-stream tags 1 and 2), 1 for output
  *   gradients D (tags 3 and 4).  rm selects RNE or Philox SR; the stream of
  *   element e (row-major index) is keyed by `seed` and counted from
- *   `offset` + e/8.  Launches 2 kernels (column reduce, split-quantize). */
+ *   `offset` + e/16.  Launches 2 kernels (column reduce, split-quantize). */
 avr_status averis_split_quant(const void* X, avr_dtype xt, int64_t l, int64_t K, avr_round rm,
                               uint64_t seed, uint64_t offset, int grad, float* mu,
                               const avr_nvfp4* mu_q, const avr_nvfp4* xr_q, float* xr_debug,
                               void* ws, size_t ws_bytes, avr_stream stream);
+
+/* Mean-energy ratio monitor [R7.2]:
+ *   R = ||mu_X||_2 / sqrt(E_i ||x_i||^2 / m),
+ * mu_X the column mean of X [l, K] (m = K features, l >= 1 tokens), E_i the
+ * average over the l rows.  The pages leave N in the formula undefined; it
+ * is read as the feature count m, so that R = sqrt(m) when every row equals
+ * the mean and R = 0 when the columns average to zero.
+ *   mu [K] fp32 out : the column mean in the fixed order of averis_split_quant
+ *                     (nullable; the workspace holds it otherwise).
+ *   R  fp32 device scalar out.
+ * mu in fp32 as the split computes it; column sums of squares in fp32 (fma,
+ * rows of a 256-row chunk in order, chunk partials in chunk order); the two
+ * norms in fp64.  Non-finite X latches AVR_ERR_NONFINITE.  l == 0 is
+ * rejected with AVR_ERR_UNSUPPORTED_SHAPE (R is 0/0).  Launches 2 kernels
+ * (column reduce with sums of squares, one-CTA ratio). */
+avr_status averis_mean_energy_ratio(const void* X, avr_dtype xt, int64_t l, int64_t K, float* mu,
+                                    float* R, void* ws, size_t ws_bytes, avr_stream stream);
 
 /* averis_split_quant for callers that cannot allocate.  The paper has no
  * counterpart to this entry point; it exists for the library's users.

@@ -59,6 +59,8 @@ _SIGS = {
     "averis_split_quant": (_c_int, [_c_ptr, _c_int, _c_i64, _c_i64, _c_int, _c_u64, _c_u64, _c_int,
                                     _c_ptr, ctypes.POINTER(avr_nvfp4), ctypes.POINTER(avr_nvfp4),
                                     _c_ptr, _c_ptr, _c_size, _c_ptr]),
+    "averis_mean_energy_ratio": (_c_int, [_c_ptr, _c_int, _c_i64, _c_i64, _c_ptr, _c_ptr, _c_ptr,
+                                          _c_size, _c_ptr]),
     "nvfp4_quant": (_c_int, [_c_ptr, _c_int, _c_i64, _c_i64, _c_int, _c_u64, _c_u64, _c_int,
                              ctypes.POINTER(avr_nvfp4), _c_ptr, _c_size, _c_ptr]),
     "averis_quant_weight": (_c_int, [_c_ptr, _c_int, _c_i64, _c_i64, ctypes.POINTER(avr_nvfp4),
@@ -191,6 +193,13 @@ def averis_split_quant(X, rm, seed, offset, grad, mu, mu_q, xr_q, xr_debug, ws, 
     _check(load().averis_split_quant(_ptr(X), _dtype(X), l, K, _round(rm), seed, offset, int(grad),
                                      _ptr(mu), _s(mu_q), _s(xr_q), _ptr(xr_debug), _ptr(ws),
                                      ws.numel(), _stream(stream)), "averis_split_quant")
+
+
+def averis_mean_energy_ratio(X, mu, R, ws, stream=None):
+    """R = ||mu_X|| / sqrt(E||x||^2 / m) into the 1-element fp32 device tensor R."""
+    l, K = X.shape
+    _check(load().averis_mean_energy_ratio(_ptr(X), _dtype(X), l, K, _ptr(mu), _ptr(R), _ptr(ws),
+                                           ws.numel(), _stream(stream)), "averis_mean_energy_ratio")
 
 
 def nvfp4_quant(X, rm, seed, offset, grad, out, ws, stream=None):

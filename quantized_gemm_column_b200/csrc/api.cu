@@ -32,6 +32,8 @@ WsLayout ws_layout(int64_t l, int64_t K, int64_t N) {
   w.bias = off;      off = round_up(off + static_cast<size_t>(N) * sizeof(float), 256);
   w.xr_codes = off;  off = round_up(off + static_cast<size_t>(l) * static_cast<size_t>(K) / 2, 256);
   w.xr_scales = off; off = round_up(off + scales_bytes(l, K), 256);
+  w.energy_partials = off; off = round_up(off + C * static_cast<size_t>(K) * sizeof(float), 256);
+  w.energy = off;    off = round_up(off + static_cast<size_t>(K) * sizeof(float), 256);
   w.total = off;
   return w;
 }
@@ -175,6 +177,7 @@ static avr_status split_chain(const void* X, avr_dtype xt, int64_t l, int64_t K,
   ca.K = K;
   ca.split = split;
   ca.mu_out = mu_buf;
+  ca.energy = 0;
   ca.ws = ws.base;
   ca.lay = &ws.lay;
   AVR_TRY(cuda_status(launch_colreduce(ca, s, true)));
@@ -293,6 +296,30 @@ avr_status averis_split_quant(const void* X, avr_dtype xt, int64_t l, int64_t K,
   float* mu_buf = mu ? mu : w.at<float>(w.lay.mu);
   return split_chain(X, xt, l, K, 1, rm, seed, offset, grad ? 3u : 1u, grad ? 4u : 2u, mu_buf, mu_q,
                      xr_q, xr_debug, nullptr, nullptr, w, stream);
+}
+
+avr_status averis_mean_energy_ratio(const void* X, avr_dtype xt, int64_t l, int64_t K, float* mu,
+                                    float* R, void* ws, size_t ws_bytes, avr_stream stream) {
+  if (!dtype_ok(xt)) return AVR_ERR_INVALID_ARG;
+  if (!k_ok(K) || !l_ok(l) || l == 0) return AVR_ERR_UNSUPPORTED_SHAPE;
+  if (!X || !R) return AVR_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(mu)) return AVR_ERR_MISALIGNED;
+  Ws w;
+  AVR_TRY(make_ws(ws, ws_bytes, l, K, 0, &w));
+  AVR_TRY(device_ok());
+  float* mu_buf = mu ? mu : w.at<float>(w.lay.mu);
+  ColReduceArgs ca;
+  ca.X = X;
+  ca.xt = xt;
+  ca.l = l;
+  ca.K = K;
+  ca.split = 1;
+  ca.mu_out = mu_buf;
+  ca.energy = 1;
+  ca.ws = w.base;
+  ca.lay = &w.lay;
+  AVR_TRY(cuda_status(launch_colreduce(ca, stream, true)));
+  return cuda_status(launch_energy_ratio(mu_buf, w.at<float>(w.lay.energy), K, l, R, w.status(), stream, true));
 }
 
 avr_status nvfp4_quant(const void* X, avr_dtype xt, int64_t rows, int64_t K, avr_round rm,

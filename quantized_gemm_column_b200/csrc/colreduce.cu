@@ -30,10 +30,12 @@ struct ColReduceParams {
   float* slot_xr;         // [T] max |X_R| (split) or max |X| (vanilla)
   float* slot_mu;         // [T] max |mu|
   float* mu_out;          // [K]
+  float* part_e;          // [C][K]: sum of squares (energy pass only)
+  float* energy;          // [K] column sums of squares, chunks in order (energy pass only)
   uint32_t* status;
 };
 
-template <bool kBf16>
+template <bool kBf16, bool kEnergy>
 __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_constant__ CUtensorMap map,
                                                              const ColReduceParams p) {
   extern __shared__ __align__(1024) uint8_t tile[];
@@ -69,7 +71,7 @@ __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_consta
 
   // Sequential fp32 sum of this column over the chunk, plus max and min.
   if (col < p.K) {
-    float s = 0.0f, mx = -INFINITY, mn = INFINITY;
+    float s = 0.0f, mx = -INFINITY, mn = INFINITY, e = 0.0f;
     if (kBf16) {
       const uint16_t* v = reinterpret_cast<const uint16_t*>(tile) + tid;
 #pragma unroll 8
@@ -78,6 +80,7 @@ __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_consta
         s = __fadd_rn(s, x);
         mx = fmaxf(mx, x);
         mn = fminf(mn, x);
+        if (kEnergy) e = __fmaf_rn(x, x, e);
       }
     } else {
       const float* v = reinterpret_cast<const float*>(tile) + tid;
@@ -87,8 +90,10 @@ __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_consta
         s = __fadd_rn(s, x);
         mx = fmaxf(mx, x);
         mn = fminf(mn, x);
+        if (kEnergy) e = __fmaf_rn(x, x, e);
       }
     }
+    if (kEnergy) p.part_e[static_cast<int64_t>(c) * p.K + col] = e;
     const int64_t o = static_cast<int64_t>(c) * p.K + col;
     const int64_t plane = static_cast<int64_t>(p.C) * p.K;
     p.part[o] = s;
@@ -135,6 +140,20 @@ __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_consta
         }
       }
     }
+    if (kEnergy) {
+      // the column's sum of squares, chunks in order
+      float E = 0.0f;
+      for (int c0 = 0; c0 < p.C; c0 += kBatch) {
+        float pe[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u)
+          if (c0 + u < p.C) pe[u] = __ldcg(&p.part_e[static_cast<int64_t>(c0 + u) * p.K + col]);
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u)
+          if (c0 + u < p.C) E = __fadd_rn(E, pe[u]);
+      }
+      p.energy[col] = E;
+    }
   }
   if (col < p.K) {
     if (!isfinite(S)) raise_status(p.status, AVR_ERR_NONFINITE);
@@ -170,6 +189,15 @@ __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_consta
   }
 }
 
+template <bool kBf16, bool kEnergy>
+static cudaError_t launch_colreduce_t(const CUtensorMap& map, const ColReduceParams& p, dim3 grid, size_t smem,
+                                      cudaStream_t s, bool pdl) {
+  const void* fn = reinterpret_cast<const void*>(colreduce_kernel<kBf16, kEnergy>);
+  cudaError_t e = set_max_dynamic_smem(fn, smem);
+  if (e != cudaSuccess) return e;
+  return launch_ex(colreduce_kernel<kBf16, kEnergy>, grid, dim3(kColTile), smem, s, pdl, map, p);
+}
+
 cudaError_t launch_colreduce(const ColReduceArgs& a, cudaStream_t s, bool pdl) {
   const bool bf16 = a.xt == AVR_BF16;
   const int elem = bf16 ? 2 : 4;
@@ -188,18 +216,60 @@ cudaError_t launch_colreduce(const ColReduceArgs& a, cudaStream_t s, bool pdl) {
   p.slot_xr = reinterpret_cast<float*>(a.ws + a.lay->slots);
   p.slot_mu = p.slot_xr + kMaxColTiles;
   p.mu_out = a.mu_out;
+  p.part_e = reinterpret_cast<float*>(a.ws + a.lay->energy_partials);
+  p.energy = reinterpret_cast<float*>(a.ws + a.lay->energy);
   p.status = reinterpret_cast<uint32_t*>(a.ws + a.lay->status);
   const int T = static_cast<int>((a.K + kColTile - 1) / kColTile);
   const size_t smem = static_cast<size_t>(kChunkRows) * kColTile * elem;
-  dim3 grid(T, p.C);
-  if (bf16) {
-    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(colreduce_kernel<true>), smem);
-    if (e != cudaSuccess) return e;
-    return launch_ex(colreduce_kernel<true>, grid, dim3(kColTile), smem, s, pdl, map, p);
+  const dim3 grid(T, p.C);
+  if (a.energy) {
+    return bf16 ? launch_colreduce_t<true, true>(map, p, grid, smem, s, pdl)
+                : launch_colreduce_t<false, true>(map, p, grid, smem, s, pdl);
   }
-  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(colreduce_kernel<false>), smem);
-  if (e != cudaSuccess) return e;
-  return launch_ex(colreduce_kernel<false>, grid, dim3(kColTile), smem, s, pdl, map, p);
+  return bf16 ? launch_colreduce_t<true, false>(map, p, grid, smem, s, pdl)
+              : launch_colreduce_t<false, false>(map, p, grid, smem, s, pdl);
+}
+
+// ---------------------------------------------------------------------------
+// Mean-energy ratio R = ||mu||_2 / sqrt(E||x||^2 / m) (Lighthouse review,
+// 实践建议 item 2, with N read as the feature count m), from the reduce's mu
+// and column sums of squares: E||x||^2 = (1/l) sum_j energy_j.  One CTA; the
+// two sums run in fp64 in a fixed order (thread t over columns t, t + 256,
+// ..., then a fixed tree).
+// ---------------------------------------------------------------------------
+constexpr int kRatioThreads = 256;
+
+__global__ void __launch_bounds__(kRatioThreads) energy_ratio_kernel(const float* mu, const float* energy, int64_t K,
+                                                                     int64_t l, float* R, uint32_t* status) {
+  __shared__ double s_m[kRatioThreads], s_e[kRatioThreads];
+  pdl_wait_prior_grid();
+  double sm = 0.0, se = 0.0;
+  for (int64_t j = threadIdx.x; j < K; j += kRatioThreads) {
+    const double u = static_cast<double>(__ldcg(mu + j));
+    sm = fma(u, u, sm);
+    se += static_cast<double>(__ldcg(energy + j));
+  }
+  s_m[threadIdx.x] = sm;
+  s_e[threadIdx.x] = se;
+  __syncthreads();
+  for (int w = kRatioThreads / 2; w > 0; w >>= 1) {
+    if (static_cast<int>(threadIdx.x) < w) {
+      s_m[threadIdx.x] += s_m[threadIdx.x + w];
+      s_e[threadIdx.x] += s_e[threadIdx.x + w];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const double mean_sq = s_e[0] / static_cast<double>(l) / static_cast<double>(K);   // E||x||^2 / m
+    const double r = mean_sq > 0.0 ? sqrt(s_m[0]) / sqrt(mean_sq) : 0.0;
+    if (!isfinite(r)) raise_status(status, AVR_ERR_NONFINITE);
+    *R = static_cast<float>(r);
+  }
+}
+
+cudaError_t launch_energy_ratio(const float* mu, const float* energy, int64_t K, int64_t l, float* R,
+                                uint32_t* status, cudaStream_t s, bool pdl) {
+  return launch_ex(energy_ratio_kernel, dim3(1), dim3(kRatioThreads), 0, s, pdl, mu, energy, K, l, R, status);
 }
 
 }  // namespace avr

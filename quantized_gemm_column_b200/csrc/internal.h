@@ -29,6 +29,7 @@ struct WsLayout {
   size_t xr_gdec = 0;
   size_t bias = 0;                                  // float[N]
   size_t xr_codes = 0, xr_scales = 0;               // Q_4(X_R), l x K
+  size_t energy_partials = 0, energy = 0;           // float[C][K], float[K]: the R monitor's sums of squares
   size_t total = 0;
 };
 WsLayout ws_layout(int64_t l, int64_t K, int64_t N);
@@ -42,10 +43,15 @@ struct ColReduceArgs {
   int64_t l, K;
   int split;              // 1: mean + residual amax; 0: amax of X only (vanilla)
   float* mu_out;          // [K], written when split (nullable otherwise)
+  int energy;             // 1: also the column sums of squares (the R monitor)
   char* ws;               // workspace base
   const WsLayout* lay;
 };
 cudaError_t launch_colreduce(const ColReduceArgs& a, cudaStream_t s, bool pdl);
+
+// R = ||mu|| / sqrt(E||x||^2 / m) from mu [K] and the column sums of squares [K]
+cudaError_t launch_energy_ratio(const float* mu, const float* energy, int64_t K, int64_t l, float* R,
+                                uint32_t* status, cudaStream_t s, bool pdl);
 
 // ---------------- K2: split quantizer (+ mean quantizer, rank-one row) ----------------
 struct QuantArgs {

@@ -94,6 +94,7 @@ extern "C" avr_status averis_split_quant_noalloc(const void* X, avr_dtype xt, in
   ca.K = K;
   ca.split = 1;
   ca.mu_out = mu_buf;
+  ca.energy = 0;
   ca.ws = base;
   ca.lay = &lay;
   if (launch_colreduce(ca, s, false) != cudaSuccess) return AVR_ERR_CUDA;

@@ -85,3 +85,18 @@ def test_validation_rejects_before_any_launch(lib):
     b = api.avr_nvfp4(16, 16, 16, 100, 128)
     assert lib.nvfp4_gemm(ctypes.byref(a), ctypes.byref(b), None, ctypes.c_void_p(16), 1, ws, 1 << 30,
                           None) == api.AVR_ERR_UNSUPPORTED_SHAPE
+
+
+def test_mean_energy_ratio_validation(lib):
+    """The R monitor rejects bad arguments, and l = 0 (R is 0/0), before any launch."""
+    from quantized_gemm_column_b200 import api
+    ws = ctypes.c_void_p(256)
+    R = ctypes.c_void_p(16)
+    f = lib.averis_mean_energy_ratio
+    assert f(None, 1, 256, 128, None, R, ws, 1 << 30, None) == api.AVR_ERR_INVALID_ARG
+    assert f(ctypes.c_void_p(16), 1, 256, 128, None, None, ws, 1 << 30, None) == api.AVR_ERR_INVALID_ARG
+    assert f(ctypes.c_void_p(16), 1, 0, 128, None, R, ws, 1 << 30, None) == api.AVR_ERR_UNSUPPORTED_SHAPE
+    assert f(ctypes.c_void_p(16), 1, 256, 96, None, R, ws, 1 << 30, None) == api.AVR_ERR_UNSUPPORTED_SHAPE
+    assert f(ctypes.c_void_p(24), 1, 256, 128, None, R, ws, 1 << 30, None) == api.AVR_ERR_MISALIGNED
+    assert f(ctypes.c_void_p(16), 1, 256, 128, None, R, ws, 64, None) == api.AVR_ERR_WORKSPACE_TOO_SMALL
+    assert f(ctypes.c_void_p(16), 9, 256, 128, None, R, ws, 1 << 30, None) == api.AVR_ERR_INVALID_ARG

@@ -65,3 +65,19 @@ def test_mean_energy_ratio_grows_with_mean_scale():
     r = [stats.mean_energy_ratio(inputs.bf16_as_f32(inputs.workload3(c, l=1024, m=256)[0]))
          for c in (0.0, 2.0, 8.0)]
     assert r[0] < r[1] < r[2]
+
+
+def test_mean_energy_ratio_closed_forms():
+    """Constant rows x_i = c give mu = c and ||x_i||^2 = ||c||^2, so R = sqrt(m)
+    exactly; rows in +/- pairs give mu = 0, so R = 0."""
+    rng = np.random.default_rng(3)
+    m = 96
+    c = rng.standard_normal(m)
+    X = np.tile(c, (40, 1))
+    assert stats.mean_energy_ratio(X) == pytest.approx(math.sqrt(m), rel=1e-12)
+    Y = rng.standard_normal((20, m))
+    pairs = np.stack([Y, -Y], axis=1).reshape(40, m)     # y1, -y1, y2, -y2, ...
+    assert stats.mean_energy_ratio(pairs) < 1e-12
+    # scaling X leaves R unchanged
+    Z = rng.standard_normal((64, m)) + 0.5
+    assert stats.mean_energy_ratio(3.0 * Z) == pytest.approx(stats.mean_energy_ratio(Z), rel=1e-12)
