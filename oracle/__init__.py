@@ -61,6 +61,13 @@ from .averis import (
     gemm_reference,
     averis_linear_reference,
     vanilla_linear_reference,
+    padded_tokens,
+    transpose_padded,
+    averis_split_quant_t,
+    vanilla_quant_t,
+    wgrad_reference,
+    averis_wgrad_reference,
+    vanilla_wgrad_reference,
 )
 from . import stats
 

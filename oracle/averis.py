@@ -26,6 +26,13 @@ Readings where the pages are silent:
     for dgrad (stored [m, n/2]); weights are always rounded to nearest even;
   * stochastic rounding (when selected) applies to the split operands X_R,
     mu_X, D_R, mu_D and to the vanilla operands, each with its own stream tag.
+  * weight gradient (the pages name W4A4G4 but give no Averis equation for
+    it): dW = X^T D = X_R^T D_R + l mu_X^T mu_D, since 1^T X_R = 0 removes both
+    cross terms.  The two residuals are quantized along the tokens (the
+    contraction axis), as [m, L] and [n, L] tensors with L = l rounded up to
+    a multiple of 64 and zero padding; their tensor scales are those of the
+    row-wise residuals (same amax); the rank-one term uses the same
+    quantized means mu_bar_X, mu_bar_D as the forward and dgrad.
 """
 
 import numpy as np
@@ -38,7 +45,10 @@ CHUNK = 256
 TAGS = {
     "x_r": 1, "mu_x": 2, "d_r": 3, "mu_d": 4,
     "w_fwd": 5, "w_dgrad": 6, "vanilla_x": 7, "vanilla_d": 8,
+    "x_r_t": 9, "d_r_t": 10, "vanilla_x_t": 11, "vanilla_d_t": 12,
 }
+
+TOKEN_ALIGN = 64     # the token axis of the weight-gradient operands is padded to this
 
 
 def _as_f32(X):
@@ -142,3 +152,67 @@ def averis_linear_reference(X, w_q: NVFP4, rounding="sr", seed=0, offset=0, grad
 def vanilla_linear_reference(X, w_q: NVFP4, rounding="sr", seed=0, offset=0, grad=False):
     x_q = vanilla_quant(X, rounding, seed, offset, grad)
     return gemm_reference(x_q, w_q), dict(x_q=x_q)
+
+
+# ---------------------------------------------------------------------------
+# weight gradient: operands quantized along the tokens
+# ---------------------------------------------------------------------------
+
+def padded_tokens(l):
+    """L = l rounded up to a multiple of 64 (the contraction length of dW)."""
+    return (int(l) + TOKEN_ALIGN - 1) // TOKEN_ALIGN * TOKEN_ALIGN
+
+
+def transpose_padded(T):
+    """[l, K] -> [K, L]: T^T with zero columns l .. L-1."""
+    T = np.asarray(T, dtype=np.float32)
+    l, K = T.shape
+    out = np.zeros((K, padded_tokens(l)), dtype=np.float32)
+    out[:, :l] = T.T
+    return out
+
+
+def averis_split_quant_t(X, rounding="sr", seed=0, offset=0, grad=False):
+    """(mu, mu_bar, X_bar_R^T): the split of X (grad=False) or D (grad=True)
+    with the residual quantized along the tokens, [K, L].  mu_bar is the same
+    tensor averis_split_quant gives (same stream tag)."""
+    X = _as_f32(X)
+    _check_finite(X)
+    mu, XR, A = column_mean_and_residual_amax(X)
+    _check_finite(mu)
+    t_rt, t_mu = (TAGS["d_r_t"], TAGS["mu_d"]) if grad else (TAGS["x_r_t"], TAGS["mu_x"])
+    xrt_q = nvfp4_quantize(transpose_padded(XR), rounding, seed, offset, t_rt, amax=A)
+    mu_q = nvfp4_quantize(mu[None, :], rounding, seed, offset, t_mu)
+    return mu, mu_q, xrt_q
+
+
+def vanilla_quant_t(X, rounding="sr", seed=0, offset=0, grad=False):
+    """Q_4(X^T) along the tokens with no split, [K, L]."""
+    X = _as_f32(X)
+    _check_finite(X)
+    tag = TAGS["vanilla_d_t"] if grad else TAGS["vanilla_x_t"]
+    return nvfp4_quantize(transpose_padded(X), rounding, seed, offset, tag)
+
+
+def wgrad_reference(xt_q: NVFP4, dt_q: NVFP4, mu_x_q=None, mu_d_q=None, l=0):
+    """fp64 dW = deq(A^T) deq(B^T)^T (+ l deq(mu_bar_X)^T deq(mu_bar_D)), [m, n]."""
+    dW = nvfp4_dequantize(xt_q) @ nvfp4_dequantize(dt_q).T
+    if mu_x_q is not None:
+        dW = dW + float(l) * np.outer(nvfp4_dequantize(mu_x_q)[0], nvfp4_dequantize(mu_d_q)[0])
+    return dW
+
+
+def averis_wgrad_reference(X, D, rounding="sr", seed=0, offset=0):
+    """Weight gradient of the Averis linear from X [l, m] and D [l, n]: fp64 dW
+    [m, n] plus the operands."""
+    l = np.asarray(X).shape[0]
+    mu_x, mu_x_q, xrt_q = averis_split_quant_t(X, rounding, seed, offset, grad=False)
+    mu_d, mu_d_q, drt_q = averis_split_quant_t(D, rounding, seed, offset, grad=True)
+    dW = wgrad_reference(xrt_q, drt_q, mu_x_q, mu_d_q, l)
+    return dW, dict(mu_x=mu_x, mu_d=mu_d, mu_x_q=mu_x_q, mu_d_q=mu_d_q, xrt_q=xrt_q, drt_q=drt_q)
+
+
+def vanilla_wgrad_reference(X, D, rounding="sr", seed=0, offset=0):
+    xt_q = vanilla_quant_t(X, rounding, seed, offset, grad=False)
+    dt_q = vanilla_quant_t(D, rounding, seed, offset, grad=True)
+    return wgrad_reference(xt_q, dt_q), dict(xt_q=xt_q, dt_q=dt_q)
