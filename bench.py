@@ -42,7 +42,7 @@ FLOPS_PER_STEP = 2 * (2 * L * M * N)
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=1000)
+    p.add_argument("--steps", type=int, default=4000)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="averis", choices=["averis", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -62,7 +62,8 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.lines = []
+        self.lines = []          # (monotonic time, csv line)
+        self.window = None
 
     def __enter__(self):
         try:
@@ -72,13 +73,25 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            # the timed region starts only once nvidia-smi is sampling
+            t_end = time.monotonic() + 5.0
+            while not self.lines and time.monotonic() < t_end and self.proc.poll() is None:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def region(self, t0, t1):
+        """The timed region, in time.monotonic() seconds."""
+        self.window = (t0, t1)
+        # a region shorter than the sampling period still gets the next sample
+        t_end = time.monotonic() + 1.0
+        while self.proc is not None and time.monotonic() < t_end and not any(t > t1 for t, _ in self.lines):
+            time.sleep(0.01)
 
     def __exit__(self, *exc):
         if self.proc:
@@ -90,9 +103,20 @@ class ClockSampler:
             self.t.join(timeout=2)
 
     def summary(self):
+        """Median SM clock and active reasons over the samples taken inside the
+        timed region; if the region was shorter than the sampling period, the
+        first sample after it (labelled with samples_in_region = 0)."""
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        lines = self.lines
+        inside = lines
+        if self.window is not None:
+            t0, t1 = self.window
+            inside = [(t, ln) for t, ln in lines if t0 <= t <= t1]
+            if not inside:
+                inside = [(t, ln) for t, ln in lines if t > t1][:1]
+        n_inside = sum(1 for t, _ in inside if self.window is None or t <= self.window[1])
+        for _, ln in inside:
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) != 6:
                 continue
@@ -105,9 +129,9 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(nm)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples_in_region": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples_in_region": n_inside}
 
 
 # ---------------------------------------------------------------------------
@@ -325,8 +349,10 @@ def run_gpu(args, rank, world, local_rank):
         torch.cuda.synchronize(dev)
 
     with ClockSampler(local_rank) as clk:
+        t0 = time.monotonic()
         ms = timed(args.steps)
         ms_van = timed(args.steps, vanilla=True)
+        clk.region(t0, time.monotonic())
     clocks = clk.summary()
     st = api.averis_check_status(ws, stream)
     if st:
@@ -448,7 +474,7 @@ def run_gpu(args, rank, world, local_rank):
         "weight_quant_us": wq_us,
         "roofline": roof,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
-                   "reasons": clocks["reasons"]},
+                   "reasons": clocks["reasons"], "samples_in_region": clocks["samples_in_region"]},
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 6 * args.steps,
         "cpu_baseline": cpu,

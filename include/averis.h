@@ -238,6 +238,63 @@ avr_status nvfp4_linear_dgrad(const void* D, avr_dtype dt, int64_t l, int64_t m,
                               avr_stream stream);
 
 /* -------------------------------------------------------------------------
+ * Weight gradient [R3.1], [RAv]
+ *
+ * The pages train W4A4G4 (all three GEMMs of a linear in FP4) but write the
+ * Averis split only for the forward and dgrad.  For dW = X^T D (X [l, m],
+ * D [l, n], Y = X W) the same split gives
+ *     X^T D = X_R^T D_R + l mu_X^T mu_D
+ * (both cross terms vanish because 1^T X_R = 0), so the residual product
+ * runs on the tensor cores and the mean part is a rank-one fp32 term.
+ * Readings: the residuals are quantized along the tokens (the contraction
+ * axis) as [m, L] and [n, L] tensors, L = l rounded up to a multiple of 64,
+ * tokens l..L-1 exact zeros; their tensor scales are the row-wise
+ * residuals' (same amax); the rank-one term uses the quantized means
+ * mu_bar_X, mu_bar_D (the bits averis_split_quant gives for the same seed and
+ * offset).  Random-stream tags: 9 (X_R^T), 10 (D_R^T), 11/12 (vanilla X^T,
+ * D^T); element (j, i) of the [K, L] tensor counts from offset + (j L + i)/16.
+ * ------------------------------------------------------------------------- */
+
+/* Split of X [l, K] (grad = 0) or D (grad = 1) with the residual quantized
+ * along the tokens.
+ *   mu     [K] fp32 out (nullable), mu_q 1 x K out (nullable): as averis_split_quant.
+ *   xrt_q  out: Q_4((X - 1 mu)^T), rows = K, K-field = L.
+ * Workspace: averis_workspace_size(l, K, 0).  Launches 2 kernels. */
+avr_status averis_split_quant_t(const void* X, avr_dtype xt, int64_t l, int64_t K, avr_round rm,
+                                uint64_t seed, uint64_t offset, int grad, float* mu,
+                                const avr_nvfp4* mu_q, const avr_nvfp4* xrt_q, void* ws,
+                                size_t ws_bytes, avr_stream stream);
+
+/* Q_4(X^T) along the tokens with no split (the vanilla comparison). */
+avr_status nvfp4_quant_t(const void* X, avr_dtype xt, int64_t l, int64_t K, avr_round rm,
+                         uint64_t seed, uint64_t offset, int grad, const avr_nvfp4* out, void* ws,
+                         size_t ws_bytes, avr_stream stream);
+
+/* Workspace bytes of averis_wgrad_gemm and the two *_linear_wgrad calls. */
+size_t averis_wgrad_workspace_size(int64_t l, int64_t m, int64_t n);
+
+/* dW [m, n] = g(A) g(B) deq(A) deq(B)^T + l deq(mu_bar_X)^T deq(mu_bar_D)
+ * from xrt_q [m, L] and drt_q [n, L] (L = l rounded up to 64); mu_x_q 1 x m
+ * and mu_d_q 1 x n are both given (Averis) or both NULL (plain product).
+ * wt: fp32 or bf16 output.  Needs m % 64 == 0, n % 64 == 0, l >= 1.
+ * Launches 2 kernels (rank-one factors, GEMM) or 1. */
+avr_status averis_wgrad_gemm(const avr_nvfp4* xrt_q, const avr_nvfp4* drt_q, const avr_nvfp4* mu_x_q,
+                             const avr_nvfp4* mu_d_q, int64_t l, void* dW, avr_dtype wt, void* ws,
+                             size_t ws_bytes, avr_stream stream);
+
+/* The whole Averis weight gradient from X [l, m] and D [l, n]: the two
+ * token-axis splits into workspace scratch, then averis_wgrad_gemm.
+ * l == 0 writes dW = 0.  Launches 6 kernels. */
+avr_status averis_linear_wgrad(const void* X, avr_dtype xt, const void* D, avr_dtype dt, int64_t l,
+                               int64_t m, int64_t n, avr_round rm, uint64_t seed, uint64_t offset,
+                               void* dW, avr_dtype wt, void* ws, size_t ws_bytes, avr_stream stream);
+
+/* Vanilla NVFP4 weight gradient Q_4(X^T) Q_4(D^T)^T.  Launches 5 kernels. */
+avr_status nvfp4_linear_wgrad(const void* X, avr_dtype xt, const void* D, avr_dtype dt, int64_t l,
+                              int64_t m, int64_t n, avr_round rm, uint64_t seed, uint64_t offset,
+                              void* dW, avr_dtype wt, void* ws, size_t ws_bytes, avr_stream stream);
+
+/* -------------------------------------------------------------------------
  * Diagnostics (used by the tests to pin the number formats on the device)
  * ------------------------------------------------------------------------- */
 

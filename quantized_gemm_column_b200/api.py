@@ -59,6 +59,19 @@ _SIGS = {
     "averis_split_quant": (_c_int, [_c_ptr, _c_int, _c_i64, _c_i64, _c_int, _c_u64, _c_u64, _c_int,
                                     _c_ptr, ctypes.POINTER(avr_nvfp4), ctypes.POINTER(avr_nvfp4),
                                     _c_ptr, _c_ptr, _c_size, _c_ptr]),
+    "averis_split_quant_t": (_c_int, [_c_ptr, _c_int, _c_i64, _c_i64, _c_int, _c_u64, _c_u64, _c_int,
+                                      _c_ptr, ctypes.POINTER(avr_nvfp4), ctypes.POINTER(avr_nvfp4),
+                                      _c_ptr, _c_size, _c_ptr]),
+    "nvfp4_quant_t": (_c_int, [_c_ptr, _c_int, _c_i64, _c_i64, _c_int, _c_u64, _c_u64, _c_int,
+                               ctypes.POINTER(avr_nvfp4), _c_ptr, _c_size, _c_ptr]),
+    "averis_wgrad_workspace_size": (_c_size, [_c_i64, _c_i64, _c_i64]),
+    "averis_wgrad_gemm": (_c_int, [ctypes.POINTER(avr_nvfp4), ctypes.POINTER(avr_nvfp4),
+                                   ctypes.POINTER(avr_nvfp4), ctypes.POINTER(avr_nvfp4), _c_i64,
+                                   _c_ptr, _c_int, _c_ptr, _c_size, _c_ptr]),
+    "averis_linear_wgrad": (_c_int, [_c_ptr, _c_int, _c_ptr, _c_int, _c_i64, _c_i64, _c_i64, _c_int,
+                                     _c_u64, _c_u64, _c_ptr, _c_int, _c_ptr, _c_size, _c_ptr]),
+    "nvfp4_linear_wgrad": (_c_int, [_c_ptr, _c_int, _c_ptr, _c_int, _c_i64, _c_i64, _c_i64, _c_int,
+                                    _c_u64, _c_u64, _c_ptr, _c_int, _c_ptr, _c_size, _c_ptr]),
     "averis_mean_energy_ratio": (_c_int, [_c_ptr, _c_int, _c_i64, _c_i64, _c_ptr, _c_ptr, _c_ptr,
                                           _c_size, _c_ptr]),
     "nvfp4_quant": (_c_int, [_c_ptr, _c_int, _c_i64, _c_i64, _c_int, _c_u64, _c_u64, _c_int,
@@ -193,6 +206,55 @@ def averis_split_quant(X, rm, seed, offset, grad, mu, mu_q, xr_q, xr_debug, ws, 
     _check(load().averis_split_quant(_ptr(X), _dtype(X), l, K, _round(rm), seed, offset, int(grad),
                                      _ptr(mu), _s(mu_q), _s(xr_q), _ptr(xr_debug), _ptr(ws),
                                      ws.numel(), _stream(stream)), "averis_split_quant")
+
+
+def padded_tokens(l):
+    """The token axis of the weight-gradient operands: l rounded up to 64."""
+    return (int(l) + 63) // 64 * 64
+
+
+def averis_wgrad_workspace_size(l, m, n):
+    return int(load().averis_wgrad_workspace_size(l, m, n))
+
+
+def wgrad_workspace(l, m, n, device="cuda"):
+    """A zero-initialised workspace for the weight-gradient calls."""
+    return torch.zeros(averis_wgrad_workspace_size(l, m, n), dtype=torch.uint8, device=device)
+
+
+def averis_split_quant_t(X, rm, seed, offset, grad, mu, mu_q, xrt_q, ws, stream=None):
+    l, K = X.shape
+    _check(load().averis_split_quant_t(_ptr(X), _dtype(X), l, K, _round(rm), seed, offset, int(grad),
+                                       _ptr(mu), _s(mu_q), _s(xrt_q), _ptr(ws), ws.numel(),
+                                       _stream(stream)), "averis_split_quant_t")
+
+
+def nvfp4_quant_t(X, rm, seed, offset, grad, out, ws, stream=None):
+    l, K = X.shape
+    _check(load().nvfp4_quant_t(_ptr(X), _dtype(X), l, K, _round(rm), seed, offset, int(grad),
+                                _s(out), _ptr(ws), ws.numel(), _stream(stream)), "nvfp4_quant_t")
+
+
+def averis_wgrad_gemm(xrt_q, drt_q, mu_x_q, mu_d_q, l, dW, ws, stream=None):
+    _check(load().averis_wgrad_gemm(_s(xrt_q), _s(drt_q), _s(mu_x_q), _s(mu_d_q), l, _ptr(dW),
+                                    _dtype(dW), _ptr(ws), ws.numel(), _stream(stream)),
+           "averis_wgrad_gemm")
+
+
+def averis_linear_wgrad(X, D, rm, seed, offset, dW, ws, stream=None):
+    l, m = X.shape
+    n = D.shape[1]
+    _check(load().averis_linear_wgrad(_ptr(X), _dtype(X), _ptr(D), _dtype(D), l, m, n, _round(rm),
+                                      seed, offset, _ptr(dW), _dtype(dW), _ptr(ws), ws.numel(),
+                                      _stream(stream)), "averis_linear_wgrad")
+
+
+def nvfp4_linear_wgrad(X, D, rm, seed, offset, dW, ws, stream=None):
+    l, m = X.shape
+    n = D.shape[1]
+    _check(load().nvfp4_linear_wgrad(_ptr(X), _dtype(X), _ptr(D), _dtype(D), l, m, n, _round(rm),
+                                     seed, offset, _ptr(dW), _dtype(dW), _ptr(ws), ws.numel(),
+                                     _stream(stream)), "nvfp4_linear_wgrad")
 
 
 def averis_mean_energy_ratio(X, mu, R, ws, stream=None):

@@ -38,6 +38,29 @@ WsLayout ws_layout(int64_t l, int64_t K, int64_t N) {
   return w;
 }
 
+int64_t padded_tokens(int64_t l) { return (l + 63) / 64 * 64; }
+
+WgLayout wgrad_layout(int64_t l, int64_t m, int64_t n) {
+  WgLayout w;
+  w.base = ws_layout(l, m > n ? m : n, 0);
+  const size_t L = static_cast<size_t>(padded_tokens(l));
+  const size_t M = static_cast<size_t>(m), N = static_cast<size_t>(n);
+  size_t off = w.base.total;
+  w.xt_codes = off;   off = round_up(off + M * L / 2, 256);
+  w.xt_scales = off;  off = round_up(off + scales_bytes(m, static_cast<int64_t>(L)), 256);
+  w.dt_codes = off;   off = round_up(off + N * L / 2, 256);
+  w.dt_scales = off;  off = round_up(off + scales_bytes(n, static_cast<int64_t>(L)), 256);
+  w.mux_codes = off;  off = round_up(off + M / 2, 256);
+  w.mux_scales = off; off = round_up(off + scales_bytes(1, m), 256);
+  w.mud_codes = off;  off = round_up(off + N / 2, 256);
+  w.mud_scales = off; off = round_up(off + scales_bytes(1, n), 256);
+  w.gdec = off;       off += 256;
+  w.u = off;          off = round_up(off + M * sizeof(float), 256);
+  w.v = off;          off = round_up(off + N * sizeof(float), 256);
+  w.total = off;
+  return w;
+}
+
 // ---------------------------------------------------------------------------
 // driver entry point for tensor maps (no link-time dependency on libcuda)
 // ---------------------------------------------------------------------------
@@ -215,8 +238,51 @@ static avr_status split_chain(const void* X, avr_dtype xt, int64_t l, int64_t K,
   return cuda_status(launch_quant(qa, s, true));
 }
 
+// K1 + K2 along the tokens (+ mean quantizer when mu_q is given), for the
+// weight gradient
+static avr_status split_chain_tokens(const void* X, avr_dtype xt, int64_t l, int64_t K, int split,
+                                     avr_round rm, uint64_t seed, uint64_t offset, uint32_t tag,
+                                     uint32_t tag_mu, float* mu_buf, const avr_nvfp4* mu_q,
+                                     const avr_nvfp4* xt_q, const Ws& ws, cudaStream_t s) {
+  ColReduceArgs ca;
+  ca.X = X;
+  ca.xt = xt;
+  ca.l = l;
+  ca.K = K;
+  ca.split = split;
+  ca.mu_out = mu_buf;
+  ca.energy = 0;
+  ca.ws = ws.base;
+  ca.lay = &ws.lay;
+  AVR_TRY(cuda_status(launch_colreduce(ca, s, true)));
+  QuantArgs qa = {};
+  qa.X = X;
+  qa.xt = xt;
+  qa.rows = l;
+  qa.K = K;
+  qa.mu = split ? mu_buf : nullptr;
+  qa.n_tiles = n_tiles(K);
+  qa.slot_xr = ws.slot_xr();
+  qa.codes = xt_q->codes;
+  qa.scales = xt_q->scales;
+  qa.g_dec = xt_q->g_dec;
+  qa.seed = seed;
+  qa.offset = offset;
+  qa.tag = tag;
+  qa.sr = rm == AVR_SR;
+  qa.status = ws.status();
+  qa.slot_mu = ws.slot_mu();
+  qa.tag_mu = tag_mu;
+  if (mu_q) {
+    qa.mu_codes = mu_q->codes;
+    qa.mu_scales = mu_q->scales;
+    qa.mu_gdec = mu_q->g_dec;
+  }
+  return cuda_status(launch_quant_tokens(qa, s, true));
+}
+
 static avr_status gemm(const avr_nvfp4* a, const avr_nvfp4* b, const float* bias, void* Y,
-                       avr_dtype yt, uint32_t* status, cudaStream_t s) {
+                       avr_dtype yt, uint32_t* status, cudaStream_t s, const float* row_scale = nullptr) {
   GemmArgs g;
   g.a_codes = a->codes;
   g.a_scales = a->scales;
@@ -228,6 +294,7 @@ static avr_status gemm(const avr_nvfp4* a, const avr_nvfp4* b, const float* bias
   g.N = b->rows;
   g.K = a->K;
   g.bias = bias;
+  g.row_scale = row_scale;
   g.Y = Y;
   g.yt = yt;
   g.status = status;
@@ -461,6 +528,136 @@ avr_status nvfp4_linear_dgrad(const void* D, avr_dtype dt, int64_t l, int64_t m,
                               avr_stream stream) {
   return linear(D, dt, l, n, m, w_dgrad, 0, rm, seed, offset, 8u, 0u, dX, xt, nullptr, nullptr, ws,
                 ws_bytes, stream);
+}
+
+// ---------------------------------------------------------------------------
+// weight gradient
+// ---------------------------------------------------------------------------
+static avr_status quant_tokens_entry(const void* X, avr_dtype xt, int64_t l, int64_t K, avr_round rm,
+                                     uint64_t seed, uint64_t offset, int split, uint32_t tag,
+                                     uint32_t tag_mu, float* mu, const avr_nvfp4* mu_q,
+                                     const avr_nvfp4* xt_q, void* ws, size_t ws_bytes, avr_stream stream) {
+  if (!dtype_ok(xt) || !round_ok(rm)) return AVR_ERR_INVALID_ARG;
+  if (!k_ok(K) || !l_ok(l)) return AVR_ERR_UNSUPPORTED_SHAPE;
+  if (l == 0) return AVR_OK;   // no tokens: nothing is read or written
+  if (!X) return AVR_ERR_INVALID_ARG;
+  AVR_TRY(check_nvfp4(xt_q, K, padded_tokens(l)));
+  if (mu_q) AVR_TRY(check_nvfp4(mu_q, 1, K));
+  if (!aligned16(X) || !aligned16(mu)) return AVR_ERR_MISALIGNED;
+  Ws w;
+  AVR_TRY(make_ws(ws, ws_bytes, l, K, 0, &w));
+  AVR_TRY(device_ok());
+  float* mu_buf = mu ? mu : w.at<float>(w.lay.mu);
+  return split_chain_tokens(X, xt, l, K, split, rm, seed, offset, tag, tag_mu, mu_buf, mu_q, xt_q, w, stream);
+}
+
+avr_status averis_split_quant_t(const void* X, avr_dtype xt, int64_t l, int64_t K, avr_round rm,
+                                uint64_t seed, uint64_t offset, int grad, float* mu,
+                                const avr_nvfp4* mu_q, const avr_nvfp4* xrt_q, void* ws,
+                                size_t ws_bytes, avr_stream stream) {
+  return quant_tokens_entry(X, xt, l, K, rm, seed, offset, 1, grad ? 10u : 9u, grad ? 4u : 2u, mu, mu_q,
+                            xrt_q, ws, ws_bytes, stream);
+}
+
+avr_status nvfp4_quant_t(const void* X, avr_dtype xt, int64_t l, int64_t K, avr_round rm,
+                         uint64_t seed, uint64_t offset, int grad, const avr_nvfp4* out, void* ws,
+                         size_t ws_bytes, avr_stream stream) {
+  return quant_tokens_entry(X, xt, l, K, rm, seed, offset, 0, grad ? 12u : 11u, 0u, nullptr, nullptr, out,
+                            ws, ws_bytes, stream);
+}
+
+size_t averis_wgrad_workspace_size(int64_t l, int64_t m, int64_t n) {
+  if (l < 0 || m <= 0 || n <= 0) return 0;
+  return wgrad_layout(l, m, n).total;
+}
+
+static avr_status make_wg(void* ws, size_t ws_bytes, int64_t l, int64_t m, int64_t n, WgLayout* lay, Ws* w) {
+  if (!ws) return AVR_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return AVR_ERR_MISALIGNED;
+  *lay = wgrad_layout(l, m, n);
+  if (ws_bytes < lay->total) return AVR_ERR_WORKSPACE_TOO_SMALL;
+  w->base = static_cast<char*>(ws);
+  w->lay = lay->base;
+  return AVR_OK;
+}
+
+// dW = alpha acc (+ u v^T) once the four operands are in place
+static avr_status wgrad_product(const avr_nvfp4* xt_q, const avr_nvfp4* dt_q, const avr_nvfp4* mu_x_q,
+                                const avr_nvfp4* mu_d_q, int64_t l, void* dW, avr_dtype wt, const Ws& w,
+                                const WgLayout& lay, cudaStream_t s) {
+  if (!mu_x_q) return gemm(xt_q, dt_q, nullptr, dW, wt, w.status(), s);
+  float* u = w.at<float>(lay.u);
+  float* v = w.at<float>(lay.v);
+  AVR_TRY(cuda_status(launch_mean_dequant(mu_x_q->codes, mu_x_q->scales, mu_x_q->g_dec, xt_q->rows, mu_d_q->codes,
+                                          mu_d_q->scales, mu_d_q->g_dec, dt_q->rows, l, u, v, s, true)));
+  return gemm(xt_q, dt_q, v, dW, wt, w.status(), s, u);
+}
+
+avr_status averis_wgrad_gemm(const avr_nvfp4* xrt_q, const avr_nvfp4* drt_q, const avr_nvfp4* mu_x_q,
+                             const avr_nvfp4* mu_d_q, int64_t l, void* dW, avr_dtype wt, void* ws,
+                             size_t ws_bytes, avr_stream stream) {
+  if (!xrt_q || !drt_q || !dtype_ok(wt)) return AVR_ERR_INVALID_ARG;
+  if ((mu_x_q == nullptr) != (mu_d_q == nullptr)) return AVR_ERR_INVALID_ARG;
+  const int64_t m = xrt_q->rows, n = drt_q->rows, L = xrt_q->K;
+  if (!k_ok(m) || !n_ok(n) || !k_ok(L) || l < 1 || padded_tokens(l) != L) return AVR_ERR_UNSUPPORTED_SHAPE;
+  if (!dW) return AVR_ERR_INVALID_ARG;
+  AVR_TRY(check_nvfp4(xrt_q, m, L));
+  AVR_TRY(check_nvfp4(drt_q, n, L));
+  if (mu_x_q) {
+    AVR_TRY(check_nvfp4(mu_x_q, 1, m));
+    AVR_TRY(check_nvfp4(mu_d_q, 1, n));
+  }
+  if (!aligned16(dW)) return AVR_ERR_MISALIGNED;
+  WgLayout lay;
+  Ws w;
+  AVR_TRY(make_wg(ws, ws_bytes, l, m, n, &lay, &w));
+  AVR_TRY(device_ok());
+  return wgrad_product(xrt_q, drt_q, mu_x_q, mu_d_q, l, dW, wt, w, lay, stream);
+}
+
+static avr_status linear_wgrad(const void* X, avr_dtype xt, const void* D, avr_dtype dt, int64_t l,
+                               int64_t m, int64_t n, int split, avr_round rm, uint64_t seed,
+                               uint64_t offset, void* dW, avr_dtype wt, void* ws, size_t ws_bytes,
+                               avr_stream stream) {
+  if (!dtype_ok(xt) || !dtype_ok(dt) || !dtype_ok(wt) || !round_ok(rm)) return AVR_ERR_INVALID_ARG;
+  if (!k_ok(m) || !n_ok(n) || !l_ok(l)) return AVR_ERR_UNSUPPORTED_SHAPE;
+  if (!dW) return AVR_ERR_INVALID_ARG;
+  if (!aligned16(dW)) return AVR_ERR_MISALIGNED;
+  if (l == 0) {   // an empty sum over tokens
+    AVR_TRY(device_ok());
+    const size_t bytes = static_cast<size_t>(m) * static_cast<size_t>(n) * (wt == AVR_BF16 ? 2 : 4);
+    return cuda_status(cudaMemsetAsync(dW, 0, bytes, stream));
+  }
+  if (!X || !D) return AVR_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(D)) return AVR_ERR_MISALIGNED;
+  WgLayout lay;
+  Ws w;
+  AVR_TRY(make_wg(ws, ws_bytes, l, m, n, &lay, &w));
+  AVR_TRY(device_ok());
+  const int64_t L = padded_tokens(l);
+  float* g = w.at<float>(lay.gdec);
+  avr_nvfp4 xq = {w.at<uint8_t>(lay.xt_codes), w.at<uint8_t>(lay.xt_scales), g, m, L};
+  avr_nvfp4 dq = {w.at<uint8_t>(lay.dt_codes), w.at<uint8_t>(lay.dt_scales), g + 1, n, L};
+  avr_nvfp4 mxq = {w.at<uint8_t>(lay.mux_codes), w.at<uint8_t>(lay.mux_scales), g + 2, 1, m};
+  avr_nvfp4 mdq = {w.at<uint8_t>(lay.mud_codes), w.at<uint8_t>(lay.mud_scales), g + 3, 1, n};
+  float* mu_buf = w.at<float>(w.lay.mu);
+  AVR_TRY(split_chain_tokens(X, xt, l, m, split, rm, seed, offset, split ? 9u : 11u, 2u, mu_buf,
+                             split ? &mxq : nullptr, &xq, w, stream));
+  AVR_TRY(split_chain_tokens(D, dt, l, n, split, rm, seed, offset, split ? 10u : 12u, 4u, mu_buf,
+                             split ? &mdq : nullptr, &dq, w, stream));
+  return wgrad_product(&xq, &dq, split ? &mxq : nullptr, split ? &mdq : nullptr, l, dW, wt, w, lay, stream);
+}
+
+avr_status averis_linear_wgrad(const void* X, avr_dtype xt, const void* D, avr_dtype dt, int64_t l,
+                               int64_t m, int64_t n, avr_round rm, uint64_t seed, uint64_t offset,
+                               void* dW, avr_dtype wt, void* ws, size_t ws_bytes, avr_stream stream) {
+  return linear_wgrad(X, xt, D, dt, l, m, n, 1, rm, seed, offset, dW, wt, ws, ws_bytes, stream);
+}
+
+avr_status nvfp4_linear_wgrad(const void* X, avr_dtype xt, const void* D, avr_dtype dt, int64_t l,
+                              int64_t m, int64_t n, avr_round rm, uint64_t seed, uint64_t offset,
+                              void* dW, avr_dtype wt, void* ws, size_t ws_bytes, avr_stream stream) {
+  return linear_wgrad(X, xt, D, dt, l, m, n, 0, rm, seed, offset, dW, wt, ws, ws_bytes, stream);
 }
 
 avr_status averis_probe_convert(const float* in, uint8_t* e4m3, uint8_t* e2m1, int64_t n,

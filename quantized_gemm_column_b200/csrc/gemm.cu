@@ -7,6 +7,8 @@
 // per-16 scales, and the row mu_bar W_bar (one value per output column) is
 // added to every output row:
 //   Y[i, j] = g_dec(A) g_dec(B) * acc[i, j] + bias[j].
+// The weight gradient's rank-one term l mu_bar_X^T mu_bar_D uses the same
+// epilogue with a row factor: Y[i, j] = alpha acc[i, j] + u[i] v[j].
 //
 // Persistent kernel, one CTA per SM; each CTA takes a contiguous run of
 // output tiles, M fastest, so consecutive tiles share their B (weight)
@@ -98,6 +100,7 @@ struct GemmParams {
   const float* gdec_a;
   const float* gdec_b;
   const float* bias;
+  const float* row_scale;   // rank-one epilogue only: Y = alpha acc + row_scale[i] bias[j]
   uint32_t* status;
 };
 
@@ -113,7 +116,7 @@ struct TileRun {
   }
 };
 
-template <int BN, bool kBf16Out>
+template <int BN, bool kBf16Out, bool kRank1>
 __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                       const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
@@ -348,6 +351,9 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
         const int64_t col = n0 + 32 * (4 * h + c) + lane;
         bias_l[c] = (p.bias != nullptr && col < p.N) ? __ldg(p.bias + col) : 0.0f;
       }
+      // rank-one epilogue: this thread's row factor (the bias row becomes the column factor)
+      float u_r = 1.0f;
+      if (kRank1) u_r = (m0 + r < p.M) ? __ldg(p.row_scale + m0 + r) : 0.0f;
       uint32_t okw = 0;
       if (lane == 0) okw = mbar_wait_poll(&acc_full[ab], static_cast<uint32_t>(i / Cfg::kAccBufs) & 1u, p.status) ? 1u : 0u;
       const bool ok = __shfl_sync(0xFFFFFFFFu, okw, 0) != 0;
@@ -368,8 +374,12 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const int j = 8 * u + 2 * k;
-              const float b0 = __shfl_sync(0xFFFFFFFFu, bias_l[c], j);
-              const float b1 = __shfl_sync(0xFFFFFFFFu, bias_l[c], j + 1);
+              float b0 = __shfl_sync(0xFFFFFFFFu, bias_l[c], j);
+              float b1 = __shfl_sync(0xFFFFFFFFu, bias_l[c], j + 1);
+              if (kRank1) {
+                b0 = __fmul_rn(u_r, b0);
+                b1 = __fmul_rn(u_r, b1);
+              }
               const __nv_bfloat162 pr = __floats2bfloat162_rn(fmaf(alpha, __uint_as_float(v[j]), b0),
                                                               fmaf(alpha, __uint_as_float(v[j + 1]), b1));
               w[k] = *reinterpret_cast<const uint32_t*>(&pr);
@@ -384,8 +394,11 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
           for (int u = 0; u < 8; ++u) {
             float f[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              f[k] = fmaf(alpha, __uint_as_float(v[4 * u + k]), __shfl_sync(0xFFFFFFFFu, bias_l[c], 4 * u + k));
+            for (int k = 0; k < 4; ++k) {
+              float b = __shfl_sync(0xFFFFFFFFu, bias_l[c], 4 * u + k);
+              if (kRank1) b = __fmul_rn(u_r, b);
+              f[k] = fmaf(alpha, __uint_as_float(v[4 * u + k]), b);
+            }
             *reinterpret_cast<float4*>(box + r * 128 + ((u ^ (r & 7)) * 16)) = make_float4(f[0], f[1], f[2], f[3]);
           }
         }
@@ -439,7 +452,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
   }
 }
 
-template <int BN, bool kBf16Out>
+template <int BN, bool kBf16Out, bool kRank1>
 static cudaError_t launch_gemm_t(const GemmArgs& a, cudaStream_t s, bool pdl) {
   using Cfg = GemmCfg<BN, kBf16Out>;
   constexpr CUtensorMapSwizzle kOpSwizzle = CU_TENSOR_MAP_SWIZZLE_128B;
@@ -474,8 +487,9 @@ static cudaError_t launch_gemm_t(const GemmArgs& a, cudaStream_t s, bool pdl) {
   p.gdec_a = a.a_gdec;
   p.gdec_b = a.b_gdec;
   p.bias = a.bias;
+  p.row_scale = a.row_scale;
   p.status = a.status;
-  auto kern = gemm_nvfp4_kernel<BN, kBf16Out>;
+  auto kern = gemm_nvfp4_kernel<BN, kBf16Out, kRank1>;
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
@@ -483,7 +497,11 @@ static cudaError_t launch_gemm_t(const GemmArgs& a, cudaStream_t s, bool pdl) {
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, bool pdl) {
-  return a.yt == AVR_BF16 ? launch_gemm_t<256, true>(a, s, pdl) : launch_gemm_t<128, false>(a, s, pdl);
+  if (a.row_scale != nullptr) {
+    if (a.bias == nullptr) return cudaErrorInvalidValue;
+    return a.yt == AVR_BF16 ? launch_gemm_t<256, true, true>(a, s, pdl) : launch_gemm_t<128, false, true>(a, s, pdl);
+  }
+  return a.yt == AVR_BF16 ? launch_gemm_t<256, true, false>(a, s, pdl) : launch_gemm_t<128, false, false>(a, s, pdl);
 }
 
 }  // namespace avr

@@ -34,6 +34,20 @@ struct WsLayout {
 };
 WsLayout ws_layout(int64_t l, int64_t K, int64_t N);
 
+// Weight-gradient workspace: the split's regions for K = max(m, n), then the
+// four token-axis operands (L = l rounded up to 64), their decode scales and
+// the rank-one factors u [m], v [n].
+int64_t padded_tokens(int64_t l);
+struct WgLayout {
+  WsLayout base;
+  size_t xt_codes = 0, xt_scales = 0, dt_codes = 0, dt_scales = 0;
+  size_t mux_codes = 0, mux_scales = 0, mud_codes = 0, mud_scales = 0;
+  size_t gdec = 0;        // float[4]: X_R^T, D_R^T, mu_bar_X, mu_bar_D
+  size_t u = 0, v = 0;
+  size_t total = 0;
+};
+WgLayout wgrad_layout(int64_t l, int64_t m, int64_t n);
+
 size_t scales_bytes(int64_t rows, int64_t K);
 
 // ---------------- K1: fixed-order column reduce ----------------
@@ -83,6 +97,16 @@ struct QuantArgs {
 };
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s, bool pdl);
 
+// The same split quantized along the tokens (a.rows = l tokens, a.K
+// features): codes [K][L/2] and scales of a K x L tensor, L = l rounded up to
+// 64, zero padding.  xr_debug and the rank-one row (w_*) are not used.
+cudaError_t launch_quant_tokens(const QuantArgs& a, cudaStream_t s, bool pdl);
+
+// u = l * deq(mu_bar_X) [m], v = deq(mu_bar_D) [n]
+cudaError_t launch_mean_dequant(const uint8_t* codes_x, const uint8_t* scales_x, const float* gdec_x, int64_t m,
+                                const uint8_t* codes_d, const uint8_t* scales_d, const float* gdec_d, int64_t n,
+                                int64_t l, float* u, float* v, cudaStream_t s, bool pdl);
+
 // Q_4 of T = W^T for W [m, n] (T [n, m], blocks along m), round to nearest even.
 struct QuantTransposedArgs {
   const void* W;
@@ -119,6 +143,7 @@ struct GemmArgs {
   const float* b_gdec;
   int64_t M, N, K;
   const float* bias;   // nullable
+  const float* row_scale = nullptr;   // nullable: Y = alpha acc + row_scale[i] * bias[j] (rank-one term)
   void* Y;
   avr_dtype yt;
   uint32_t* status;

@@ -53,6 +53,7 @@ struct QuantParams {
   const float* w_gdec;
   int64_t n_out;
   float* bias;
+  int64_t lp;             // token-axis quantizer: tokens rounded up to a multiple of 64
 };
 
 __device__ __forceinline__ float max_of_slots(const float* slots, int n) {
@@ -541,6 +542,204 @@ cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s, bool pdl) {
   if (a.xt == AVR_BF16)
     return a.sr ? launch_quant_t<true, true>(p, tasks, smem, s, pdl) : launch_quant_t<true, false>(p, tasks, smem, s, pdl);
   return a.sr ? launch_quant_t<false, true>(p, tasks, smem, s, pdl) : launch_quant_t<false, false>(p, tasks, smem, s, pdl);
+}
+
+// ---------------------------------------------------------------------------
+// The split quantized along the tokens, for the weight gradient:
+// T = (X - 1 mu)^T [K, L] with L = l rounded up to 64 and T[j][i] = 0 for
+// i >= l, quantized along its rows (16-token blocks), so that dW = X^T D
+// splits into X_bar_R^T D_bar_R on the tensor cores plus a rank-one term.
+// The tensor scale is the row-wise residual's (same amax, from the column
+// reduce); the random stream of element (j, i) of T counts from
+// offset + (j L + i) / 16.
+//
+// A CTA takes 128 tokens x 128 features: one TMA box into shared memory
+// (tokens beyond l read as zero and are replaced by exact zeros), then
+// thread t owns feature 128 c0 + t % 128 and 64 consecutive tokens: four
+// blocks, 32 bytes of codes (one full sector) and one 4-scale atom word.
+// With mean quantization asked for, CTA 0 is an aux CTA that quantizes mu
+// exactly as the row-wise quantizer does (same function, same tag).
+// ---------------------------------------------------------------------------
+constexpr int kTokTile = 128;     // tokens per CTA
+constexpr int kFeatTile = 128;    // features per CTA
+
+template <bool kBf16, bool kSR>
+__global__ void __launch_bounds__(kQuantThreads) quant_tokens_kernel(const __grid_constant__ CUtensorMap map,
+                                                                     const QuantParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_tile[];   // the X tile, or (aux CTA) mu_bar in f16
+  __shared__ float r_tab[128];
+  __shared__ uint64_t bar;
+  __shared__ float s_genc, s_gdec;
+  __shared__ uint32_t s_ok;
+  constexpr uint32_t kElem = kBf16 ? 2u : 4u;
+  constexpr uint32_t kTileBytes = kTokTile * kFeatTile * kElem;
+  if (static_cast<int>(blockIdx.x) < p.n_aux) {
+    __shared__ float s_part[kQuantWarps * kRowGroup];
+    pdl_wait_prior_grid();
+    pdl_allow_next_grid();
+    aux_cta<kSR>(p, reinterpret_cast<uint16_t*>(smem_tile), s_part, r_tab);
+    return;
+  }
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bid = static_cast<int>(blockIdx.x) - p.n_aux;
+  const int tiles_k = static_cast<int>((p.K + kFeatTile - 1) / kFeatTile);
+  const int64_t f0 = static_cast<int64_t>(bid % tiles_k) * kFeatTile;   // first feature
+  const int64_t t0 = static_cast<int64_t>(bid / tiles_k) * kTokTile;    // first token
+  if (tid == 0) {
+    prefetch_tensormap(&map);
+    mbar_init(&bar, 1);
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  pdl_wait_prior_grid();
+  pdl_allow_next_grid();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bar, kTileBytes);
+    tma_load_2d(smem_tile, &map, &bar, static_cast<int32_t>(f0), static_cast<int32_t>(t0));
+  }
+  const int c = tid % kFeatTile, grp = tid / kFeatTile;
+  const int64_t j = f0 + c;                                  // feature = row of T
+  const int64_t i0 = t0 + 64 * grp;                          // first token of this thread
+  const float mu = (p.mu != nullptr && j < p.K) ? __ldg(p.mu + j) : 0.0f;
+  if (warp == 0) {
+    const TensorScale ts = tensor_scale(max_of_slots(p.slot_xr, p.n_tiles));
+    if (lane == 0) {
+      s_genc = ts.g_enc;
+      s_gdec = ts.g_dec;
+    }
+  }
+  __syncthreads();
+  fill_rscale_table(r_tab, s_genc);
+  if (tid == 0) {
+    s_ok = mbar_wait(&bar, 0, p.status) ? 1u : 0u;
+    if (!s_ok) mbar_wait(&bar, 0, nullptr);   // a second bounded wait for the copy in flight
+  }
+  __syncthreads();
+  if (bid == 0 && tid == 0) *p.g_dec = s_gdec;
+  if (!s_ok || j >= p.K || i0 >= p.lp) return;
+
+  const float g_enc = s_genc;
+  PhiloxKeys keys;
+  if (kSR) keys = philox_keys(p.seed);
+  const uint64_t g = p.offset + static_cast<uint64_t>((j * p.lp + i0) / 16);
+  uint32_t packed[8], sw = 0;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    float xr[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      const int rr = 64 * grp + 16 * b + t;                 // token within the tile
+      const uint32_t idx = static_cast<uint32_t>(rr * kFeatTile + c);
+      const float x = kBf16 ? __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(smem_tile)[idx]) << 16)
+                            : reinterpret_cast<const float*>(smem_tile)[idx];
+      xr[t] = (t0 + rr < p.rows) ? __fsub_rn(x, mu) : 0.0f;
+    }
+    const uint4 rw = kSR ? philox_keyed(g + b, p.tag, keys) : make_uint4(0u, 0u, 0u, 0u);
+    uint32_t S;
+    const uint2 pk = quant16<kSR>(xr, g_enc, r_tab, rw, &S);
+    packed[2 * b] = pk.x;
+    packed[2 * b + 1] = pk.y;
+    sw |= S << (8 * b);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(p.codes + j * (p.lp / 2) + i0 / 2);
+  dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+  *reinterpret_cast<uint32_t*>(p.scales + scale_offset(static_cast<uint64_t>(j), static_cast<uint32_t>(i0 / 16),
+                                                       static_cast<uint32_t>(p.lp / 64))) = sw;
+}
+
+template <bool kBf16, bool kSR>
+static cudaError_t launch_quant_tokens_t(const CUtensorMap& map, const QuantParams& p, int64_t ctas, size_t smem,
+                                         cudaStream_t s, bool pdl) {
+  const void* fn = reinterpret_cast<const void*>(quant_tokens_kernel<kBf16, kSR>);
+  cudaError_t e = set_max_dynamic_smem(fn, smem);
+  if (e != cudaSuccess) return e;
+  return launch_ex(quant_tokens_kernel<kBf16, kSR>, dim3(static_cast<unsigned>(ctas)), dim3(kQuantThreads), smem, s,
+                   pdl, map, p);
+}
+
+cudaError_t launch_quant_tokens(const QuantArgs& a, cudaStream_t s, bool pdl) {
+  const bool bf16 = a.xt == AVR_BF16;
+  const int elem = bf16 ? 2 : 4;
+  CUtensorMap map;
+  if (!make_tensor_map_2d(&map, a.X, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                          elem, static_cast<uint64_t>(a.rows), static_cast<uint64_t>(a.K), kTokTile, kFeatTile,
+                          CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  QuantParams p = {};
+  p.rows = a.rows;
+  p.K = a.K;
+  p.lp = (a.rows + 63) / 64 * 64;
+  p.mu = a.mu;
+  p.n_tiles = a.n_tiles;
+  p.slot_xr = a.slot_xr;
+  p.codes = a.codes;
+  p.scales = a.scales;
+  p.g_dec = a.g_dec;
+  p.seed = a.seed;
+  p.offset = a.offset;
+  p.tag = a.tag;
+  p.status = a.status;
+  p.slot_mu = a.slot_mu;
+  p.tag_mu = a.tag_mu;
+  p.mu_codes = a.mu_codes;
+  p.mu_scales = a.mu_scales;
+  p.mu_gdec = a.mu_gdec;
+  size_t smem = static_cast<size_t>(kTokTile) * kFeatTile * elem;
+  if (a.mu != nullptr && a.mu_codes != nullptr) {
+    p.n_aux = 1;
+    const size_t aux = static_cast<size_t>(min64(a.K, kBiasWindow)) * sizeof(uint16_t);
+    if (aux > smem) smem = aux;
+  }
+  // scale rows K .. next multiple of 128 (features past K) are zero
+  if (a.K % 128 != 0) {
+    zero_scale_padding<<<32, 256, 0, s>>>(a.scales, a.K, p.lp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    pdl = false;
+  }
+  const int64_t ctas = p.n_aux + ((a.K + kFeatTile - 1) / kFeatTile) * ((p.lp + kTokTile - 1) / kTokTile);
+  if (bf16)
+    return a.sr ? launch_quant_tokens_t<true, true>(map, p, ctas, smem, s, pdl)
+                : launch_quant_tokens_t<true, false>(map, p, ctas, smem, s, pdl);
+  return a.sr ? launch_quant_tokens_t<false, true>(map, p, ctas, smem, s, pdl)
+              : launch_quant_tokens_t<false, false>(map, p, ctas, smem, s, pdl);
+}
+
+// ---------------------------------------------------------------------------
+// dequantized means for the weight gradient's rank-one term:
+// u[i] = l * deq(mu_bar_X)[i], v[j] = deq(mu_bar_D)[j], deq = e2m1 * e4m3 * g_dec
+// ---------------------------------------------------------------------------
+__global__ void mean_dequant_kernel(const uint8_t* codes_x, const uint8_t* scales_x, const float* gdec_x, int64_t m,
+                                    const uint8_t* codes_d, const uint8_t* scales_d, const float* gdec_d, int64_t n,
+                                    float l, float* u, float* v) {
+  pdl_wait_prior_grid();
+  pdl_allow_next_grid();
+  const float gx = __ldg(gdec_x), gd = __ldg(gdec_d);
+  for (int64_t k = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; k < m + n;
+       k += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const bool is_x = k < m;
+    const int64_t e = is_x ? k : k - m;
+    const int64_t K = is_x ? m : n;
+    const uint8_t* codes = is_x ? codes_x : codes_d;
+    const uint8_t* scales = is_x ? scales_x : scales_d;
+    const uint32_t byte = codes[e / 2];
+    const uint32_t code = (e & 1) ? (byte >> 4) : (byte & 0xFu);
+    const float sv = e4m3_value(scales[scale_offset(0, static_cast<uint32_t>(e / 16), static_cast<uint32_t>(K / 64))]);
+    const float val = __fmul_rn(__fmul_rn(e2m1_value(code), sv), is_x ? gx : gd);
+    if (is_x)
+      u[e] = __fmul_rn(l, val);
+    else
+      v[e] = val;
+  }
+}
+
+cudaError_t launch_mean_dequant(const uint8_t* codes_x, const uint8_t* scales_x, const float* gdec_x, int64_t m,
+                                const uint8_t* codes_d, const uint8_t* scales_d, const float* gdec_d, int64_t n,
+                                int64_t l, float* u, float* v, cudaStream_t s, bool pdl) {
+  const int64_t blocks = min64((m + n + 255) / 256, 148);
+  return launch_ex(mean_dequant_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, pdl, codes_x, scales_x,
+                   gdec_x, m, codes_d, scales_d, gdec_d, n, static_cast<float>(l), u, v);
 }
 
 // ---------------------------------------------------------------------------

@@ -100,3 +100,37 @@ def test_mean_energy_ratio_validation(lib):
     assert f(ctypes.c_void_p(24), 1, 256, 128, None, R, ws, 1 << 30, None) == api.AVR_ERR_MISALIGNED
     assert f(ctypes.c_void_p(16), 1, 256, 128, None, R, ws, 64, None) == api.AVR_ERR_WORKSPACE_TOO_SMALL
     assert f(ctypes.c_void_p(16), 9, 256, 128, None, R, ws, 1 << 30, None) == api.AVR_ERR_INVALID_ARG
+
+
+def test_wgrad_validation(lib):
+    """Weight-gradient entry points reject bad arguments before any launch."""
+    from quantized_gemm_column_b200 import api
+    ws = ctypes.c_void_p(256)
+    a = api.avr_nvfp4(16, 16, 16, 128, 320)     # [m = 128, L = 320]
+    b = api.avr_nvfp4(16, 16, 16, 192, 320)
+    mx = api.avr_nvfp4(16, 16, 16, 1, 128)
+    md = api.avr_nvfp4(16, 16, 16, 1, 192)
+    f = lib.averis_wgrad_gemm
+    Y = ctypes.c_void_p(16)
+    # one mean without the other
+    assert f(ctypes.byref(a), ctypes.byref(b), ctypes.byref(mx), None, 300, Y, 0, ws, 1 << 30,
+             None) == api.AVR_ERR_INVALID_ARG
+    # L must be l rounded up to 64
+    assert f(ctypes.byref(a), ctypes.byref(b), ctypes.byref(mx), ctypes.byref(md), 250, Y, 0, ws,
+             1 << 30, None) == api.AVR_ERR_UNSUPPORTED_SHAPE
+    # operands of different token lengths
+    b2 = api.avr_nvfp4(16, 16, 16, 192, 384)
+    assert f(ctypes.byref(a), ctypes.byref(b2), None, None, 300, Y, 0, ws, 1 << 30,
+             None) == api.AVR_ERR_INVALID_ARG
+    # workspace too small
+    assert f(ctypes.byref(a), ctypes.byref(b), ctypes.byref(mx), ctypes.byref(md), 300, Y, 0, ws, 64,
+             None) == api.AVR_ERR_WORKSPACE_TOO_SMALL
+    # whole wgrad: n not a multiple of 64, bad dtype
+    g = lib.averis_linear_wgrad
+    assert g(Y, 1, Y, 1, 300, 128, 100, 1, 0, 0, Y, 0, ws, 1 << 30, None) == api.AVR_ERR_UNSUPPORTED_SHAPE
+    assert g(Y, 5, Y, 1, 300, 128, 128, 1, 0, 0, Y, 0, ws, 1 << 30, None) == api.AVR_ERR_INVALID_ARG
+    # token-axis quantizer: descriptor must be [K, L]
+    q = api.avr_nvfp4(16, 16, 16, 128, 300)
+    assert lib.averis_split_quant_t(Y, 1, 300, 128, 0, 0, 0, 0, None, None, ctypes.byref(q), ws,
+                                    1 << 30, None) == api.AVR_ERR_INVALID_ARG
+    assert api.averis_wgrad_workspace_size(8192, 1024, 4096) > (1024 + 4096) * 8192 // 2
