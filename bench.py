@@ -387,6 +387,25 @@ def run_gpu(args, rank, world, local_rank):
     g_d = avg_us(lambda i: api.nvfp4_gemm(dr, w_dgrad, None, dX, ws, stream))
     gemm_tflops = 2 * L * M * N * 2 / ((g_f + g_d) * 1e-6) / 1e12
 
+    # the weight gradient dW = X^T dY (beyond the timed fwd + dgrad step):
+    # two token-axis splits, the rank-one factors and the GEMM, fp32 dW
+    wws = api.wgrad_workspace(L, M, N, dev)
+    dW = torch.empty((M, N), dtype=torch.float32, device=dev)
+    wg_a = avg_us(lambda i: api.averis_linear_wgrad(Xs[i % copies], Ds[i % copies], "sr", 1, 0, dW, wws, stream))
+    wg_v = avg_us(lambda i: api.nvfp4_linear_wgrad(Xs[i % copies], Ds[i % copies], "sr", 1, 0, dW, wws, stream))
+    Lp = api.padded_tokens(L)
+    xt_q, dt_q = api.NVFP4Tensor(M, Lp, dev), api.NVFP4Tensor(N, Lp, dev)
+    sqt_x = avg_us(lambda i: api.averis_split_quant_t(Xs[i % copies], "sr", 1, 0, False, None, muq, xt_q, ws, stream))
+    sqt_d = avg_us(lambda i: api.averis_split_quant_t(Ds[i % copies], "sr", 1, 0, True, None, dmuq, dt_q, ws, stream))
+    g_w = avg_us(lambda i: api.averis_wgrad_gemm(xt_q, dt_q, muq, dmuq, L, dW, wws, stream))
+    if api.averis_check_status(wws, stream) or api.averis_check_status(ws, stream):
+        raise RuntimeError("device status set by the weight-gradient timing")
+    wgrad = {"dW": f"fp32 [{M}, {N}], contraction over {L} tokens", "averis_us": wg_a, "vanilla_us": wg_v,
+             "averis_overhead_vs_vanilla": wg_a / wg_v - 1.0,
+             "tflops": 2 * L * M * N / (wg_a * 1e-6) / 1e12,
+             "split_quant_t_us": {"X": sqt_x, "dY": sqt_d}, "gemm_us": g_w,
+             "gemm_tflops": 2 * L * M * N / (g_w * 1e-6) / 1e12}
+
     # split-quant algorithmic bytes: read the input twice (reduce, quantize),
     # write codes (1/2 byte per element) and scales (1/16 byte per element)
     def sq_bytes(rows, K):
@@ -468,6 +487,7 @@ def run_gpu(args, rank, world, local_rank):
         "split_quant_gbs": sq_gbs,
         "split_quant_us": {"X": sq_x, "dY": sq_d},
         "gemm_us": {"fwd": g_f, "dgrad": g_d}, "gemm_tflops": gemm_tflops,
+        "wgrad": wgrad,
         "gemm_frac_fp4_peak": gemm_tflops / fp4_peak,
         "vanilla_ms_per_step": ms_van / args.steps,
         "averis_overhead_vs_vanilla": (ms / ms_van) - 1.0,
