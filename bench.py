@@ -203,7 +203,7 @@ def run_reference(args, rank, world):
 # ---------------------------------------------------------------------------
 # measured DRAM traffic (ncu), valid only for the kernel sources it was taken on
 # ---------------------------------------------------------------------------
-KERNEL_SOURCES = ["colreduce.cu", "quant.cu", "gemm.cu", "device.cuh", "internal.h"]
+KERNEL_SOURCES = ["colreduce.cu", "quant.cu", "quant_common.cuh", "split_fused.cu", "gemm.cu", "device.cuh", "internal.h"]
 TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "traffic_qkv_step.md")
 
 
@@ -383,6 +383,9 @@ def run_gpu(args, rank, world, local_rank):
 
     sq_x = avg_us(lambda i: api.averis_split_quant(Xs[i % copies], "sr", 1, 0, False, None, muq, xr, None, ws, stream))
     sq_d = avg_us(lambda i: api.averis_split_quant(Ds[i % copies], "sr", 1, 0, True, None, dmuq, dr, None, ws, stream))
+    # the one-kernel split (same bits), for comparison with the two-kernel chain above
+    fs_x = avg_us(lambda i: api.averis_split_quant_fused(Xs[i % copies], "sr", 1, 0, False, None, muq, xr, ws, stream))
+    fs_d = avg_us(lambda i: api.averis_split_quant_fused(Ds[i % copies], "sr", 1, 0, True, None, dmuq, dr, ws, stream))
     g_f = avg_us(lambda i: api.nvfp4_gemm(xr, w_fwd, None, Y, ws, stream))
     g_d = avg_us(lambda i: api.nvfp4_gemm(dr, w_dgrad, None, dX, ws, stream))
     gemm_tflops = 2 * L * M * N * 2 / ((g_f + g_d) * 1e-6) / 1e12
@@ -486,6 +489,7 @@ def run_gpu(args, rank, world, local_rank):
                          f"{copies * (L * M + L * N) * 2 / 2**20:.0f} MiB > 126 MB L2"},
         "split_quant_gbs": sq_gbs,
         "split_quant_us": {"X": sq_x, "dY": sq_d},
+        "split_quant_fused_us": {"X": fs_x, "dY": fs_d},
         "gemm_us": {"fwd": g_f, "dgrad": g_d}, "gemm_tflops": gemm_tflops,
         "wgrad": wgrad,
         "gemm_frac_fp4_peak": gemm_tflops / fp4_peak,

@@ -150,6 +150,21 @@ avr_status averis_split_quant(const void* X, avr_dtype xt, int64_t l, int64_t K,
 avr_status averis_mean_energy_ratio(const void* X, avr_dtype xt, int64_t l, int64_t K, float* mu,
                                     float* R, void* ws, size_t ws_bytes, avr_stream stream);
 
+/* averis_split_quant as one persistent kernel (the "fewer passes" variant):
+ * the input is read from memory once, each CTA keeping its last 256 x 128
+ * unit in shared memory, with grid-wide barriers between the reduce, the fold
+ * and the quantization instead of a second launch.  Same arguments and the
+ * same output bits as averis_split_quant (no X_R debug output).  On B200 the
+ * two-kernel chain is faster at the benchmark's sizes (its second read of the
+ * input comes from L2), so the linear entry points use that chain.  Every CTA
+ * of the grid must be resident at once: the call uses at most two CTAs per SM
+ * and no other work may hold the GPU's SMs meanwhile, else its barriers time
+ * out (AVR_ERR_DEVICE_TIMEOUT).  Launches 1 kernel (2 when l % 128 != 0). */
+avr_status averis_split_quant_fused(const void* X, avr_dtype xt, int64_t l, int64_t K, avr_round rm,
+                                    uint64_t seed, uint64_t offset, int grad, float* mu,
+                                    const avr_nvfp4* mu_q, const avr_nvfp4* xr_q, void* ws,
+                                    size_t ws_bytes, avr_stream stream);
+
 /* averis_split_quant for callers that cannot allocate.  The paper has no
  * counterpart to this entry point; it exists for the library's users.
  *

@@ -59,6 +59,9 @@ _SIGS = {
     "averis_split_quant": (_c_int, [_c_ptr, _c_int, _c_i64, _c_i64, _c_int, _c_u64, _c_u64, _c_int,
                                     _c_ptr, ctypes.POINTER(avr_nvfp4), ctypes.POINTER(avr_nvfp4),
                                     _c_ptr, _c_ptr, _c_size, _c_ptr]),
+    "averis_split_quant_fused": (_c_int, [_c_ptr, _c_int, _c_i64, _c_i64, _c_int, _c_u64, _c_u64, _c_int,
+                                          _c_ptr, ctypes.POINTER(avr_nvfp4), ctypes.POINTER(avr_nvfp4),
+                                          _c_ptr, _c_size, _c_ptr]),
     "averis_split_quant_t": (_c_int, [_c_ptr, _c_int, _c_i64, _c_i64, _c_int, _c_u64, _c_u64, _c_int,
                                       _c_ptr, ctypes.POINTER(avr_nvfp4), ctypes.POINTER(avr_nvfp4),
                                       _c_ptr, _c_size, _c_ptr]),
@@ -262,6 +265,13 @@ def averis_mean_energy_ratio(X, mu, R, ws, stream=None):
     l, K = X.shape
     _check(load().averis_mean_energy_ratio(_ptr(X), _dtype(X), l, K, _ptr(mu), _ptr(R), _ptr(ws),
                                            ws.numel(), _stream(stream)), "averis_mean_energy_ratio")
+
+
+def averis_split_quant_fused(X, rm, seed, offset, grad, mu, mu_q, xr_q, ws, stream=None):
+    l, K = X.shape
+    _check(load().averis_split_quant_fused(_ptr(X), _dtype(X), l, K, _round(rm), seed, offset, int(grad),
+                                           _ptr(mu), _s(mu_q), _s(xr_q), _ptr(ws), ws.numel(),
+                                           _stream(stream)), "averis_split_quant_fused")
 
 
 def nvfp4_quant(X, rm, seed, offset, grad, out, ws, stream=None):

@@ -192,7 +192,7 @@ static avr_status split_chain(const void* X, avr_dtype xt, int64_t l, int64_t K,
                               avr_round rm, uint64_t seed, uint64_t offset, uint32_t tag,
                               uint32_t tag_mu, float* mu_buf, const avr_nvfp4* mu_q,
                               const avr_nvfp4* xr_q, float* xr_debug, const avr_nvfp4* w,
-                              float* bias, const Ws& ws, cudaStream_t s) {
+                              float* bias, const Ws& ws, cudaStream_t s, bool fused = false) {
   ColReduceArgs ca;
   ca.X = X;
   ca.xt = xt;
@@ -203,7 +203,6 @@ static avr_status split_chain(const void* X, avr_dtype xt, int64_t l, int64_t K,
   ca.energy = 0;
   ca.ws = ws.base;
   ca.lay = &ws.lay;
-  AVR_TRY(cuda_status(launch_colreduce(ca, s, true)));
   QuantArgs qa = {};
   qa.X = X;
   qa.xt = xt;
@@ -235,6 +234,8 @@ static avr_status split_chain(const void* X, avr_dtype xt, int64_t l, int64_t K,
     qa.n_out = w->rows;
     qa.bias = bias;
   }
+  if (fused) return cuda_status(launch_split_fused(ca, qa, s, true));
+  AVR_TRY(cuda_status(launch_colreduce(ca, s, true)));
   return cuda_status(launch_quant(qa, s, true));
 }
 
@@ -327,7 +328,9 @@ avr_status averis_check_status(void* ws, avr_stream stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return AVR_ERR_CUDA;
   uint32_t st = 0;
   if (cudaMemcpy(&st, ws, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return AVR_ERR_CUDA;
-  if (st != 0 && cudaMemset(ws, 0, sizeof(st)) != cudaSuccess) return AVR_ERR_CUDA;
+  // after an error the whole 256-byte status block (status word and the
+  // grid-barrier words of the fused split) starts again from zero
+  if (st != 0 && cudaMemset(ws, 0, 256) != cudaSuccess) return AVR_ERR_CUDA;
   return static_cast<avr_status>(st);
 }
 
@@ -387,6 +390,25 @@ avr_status averis_mean_energy_ratio(const void* X, avr_dtype xt, int64_t l, int6
   ca.lay = &w.lay;
   AVR_TRY(cuda_status(launch_colreduce(ca, stream, true)));
   return cuda_status(launch_energy_ratio(mu_buf, w.at<float>(w.lay.energy), K, l, R, w.status(), stream, true));
+}
+
+avr_status averis_split_quant_fused(const void* X, avr_dtype xt, int64_t l, int64_t K, avr_round rm,
+                                    uint64_t seed, uint64_t offset, int grad, float* mu,
+                                    const avr_nvfp4* mu_q, const avr_nvfp4* xr_q, void* ws,
+                                    size_t ws_bytes, avr_stream stream) {
+  if (!dtype_ok(xt) || !round_ok(rm)) return AVR_ERR_INVALID_ARG;
+  if (!k_ok(K) || !l_ok(l)) return AVR_ERR_UNSUPPORTED_SHAPE;
+  if (l == 0) return AVR_OK;   // no tokens: nothing is read or written
+  if (!X) return AVR_ERR_INVALID_ARG;
+  AVR_TRY(check_nvfp4(xr_q, l, K));
+  if (mu_q) AVR_TRY(check_nvfp4(mu_q, 1, K));
+  if (!aligned16(X) || !aligned16(mu)) return AVR_ERR_MISALIGNED;
+  Ws w;
+  AVR_TRY(make_ws(ws, ws_bytes, l, K, 0, &w));
+  AVR_TRY(device_ok());
+  float* mu_buf = mu ? mu : w.at<float>(w.lay.mu);
+  return split_chain(X, xt, l, K, 1, rm, seed, offset, grad ? 3u : 1u, grad ? 4u : 2u, mu_buf, mu_q,
+                     xr_q, nullptr, nullptr, nullptr, w, stream, true);
 }
 
 avr_status nvfp4_quant(const void* X, avr_dtype xt, int64_t rows, int64_t K, avr_round rm,

@@ -85,6 +85,41 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Wait for the phase with the given parity to complete.  Returns false (and
 // records a timeout in *status) if it has not completed within kWaitLimitNs.
+// Grid-wide barrier for a grid whose CTAs are all resident at once.  Thread 0
+// of each CTA arrives on *count (acquire-release at GPU scope, after a CTA
+// barrier, so it publishes every thread's prior writes); the last of n
+// arrivals resets *count and advances *gen, which the others poll with a
+// bounded wait.  *count is back at 0 after every completed barrier.  Returns
+// false (and records AVR_ERR_DEVICE_TIMEOUT) if the other CTAs never came.
+__device__ __forceinline__ bool grid_barrier(uint32_t* count, uint32_t* gen, uint32_t n, uint32_t* status) {
+  __shared__ uint32_t s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t ok = 1u, g0, old;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g0) : "l"(gen) : "memory");
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(count) : "memory");
+    if (old == n - 1u) {
+      asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(count) : "memory");
+      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(gen) : "memory");
+    } else {
+      const uint64_t t0 = globaltimer_ns();
+      uint32_t spins = 0, g;
+      for (;;) {
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(gen) : "memory");
+        if (g != g0) break;
+        if (((++spins) & 255u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+          raise_status(status, AVR_ERR_DEVICE_TIMEOUT);
+          ok = 0u;
+          break;
+        }
+      }
+    }
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0u;
+}
+
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer_ns();

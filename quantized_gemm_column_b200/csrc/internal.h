@@ -97,6 +97,14 @@ struct QuantArgs {
 };
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s, bool pdl);
 
+// zero the scale bytes of the padding rows [rows, next multiple of 128) (no-op when rows % 128 == 0)
+cudaError_t launch_zero_scale_padding(uint8_t* scales, int64_t rows, int64_t K, cudaStream_t s);
+
+// K1 + K2 as one persistent kernel (one CTA per SM, grid-wide barriers): the
+// same outputs as launch_colreduce followed by launch_quant, without the
+// X_R debug output or the monitor's sums of squares.
+cudaError_t launch_split_fused(const ColReduceArgs& ca, const QuantArgs& qa, cudaStream_t s, bool pdl);
+
 // The same split quantized along the tokens (a.rows = l tokens, a.K
 // features): codes [K][L/2] and scales of a K x L tensor, L = l rounded up to
 // 64, zero padding.  xr_debug and the rank-one row (w_*) are not used.

@@ -30,14 +30,19 @@ def _x(l, K, dtype, seed=0, mean_scale=1.0):
     return torch.from_numpy(x).cuda(), x
 
 
-def _split(api, Xd, rm, seed=7, offset=0, grad=False):
+def _split(api, Xd, rm, seed=7, offset=0, grad=False, debug=True, fused=False):
+    """The two-kernel split, with X_R as well when debug; fused=True runs the
+    one-kernel variant (no X_R)."""
     l, K = Xd.shape
     mu = torch.empty(K, dtype=torch.float32, device="cuda")
     mu_q = api.NVFP4Tensor(1, K)
     xr_q = api.NVFP4Tensor(l, K)
-    xr = torch.empty((l, K), dtype=torch.float32, device="cuda")
+    xr = torch.empty((l, K), dtype=torch.float32, device="cuda") if debug and not fused else None
     ws = api.workspace(l, K)
-    api.averis_split_quant(Xd, rm, seed, offset, grad, mu, mu_q, xr_q, xr, ws)
+    if fused:
+        api.averis_split_quant_fused(Xd, rm, seed, offset, grad, mu, mu_q, xr_q, ws)
+    else:
+        api.averis_split_quant(Xd, rm, seed, offset, grad, mu, mu_q, xr_q, xr, ws)
     assert api.averis_check_status(ws) == 0
     return mu, mu_q, xr_q, xr
 
@@ -49,12 +54,15 @@ SHAPES = [(256, 128, "f32"), (300, 192, "bf16"), (1024, 1024, "bf16"), (4133, 64
 
 @pytest.mark.parametrize("l,K,dt", SHAPES)
 @pytest.mark.parametrize("rm", ["rne", "sr"])
-def test_split_quant_bit_exact(api, l, K, dt, rm):
+@pytest.mark.parametrize("path", ["two-kernel", "two-kernel-no-debug", "fused"])
+def test_split_quant_bit_exact(api, l, K, dt, rm, path):
     Xd, x = _x(l, K, dt, seed=l + K)
-    mu, mu_q, xr_q, xr = _split(api, Xd, rm, seed=1234 + l, offset=99)
+    debug = path == "two-kernel"
+    mu, mu_q, xr_q, xr = _split(api, Xd, rm, seed=1234 + l, offset=99, debug=debug, fused=path == "fused")
     rmu, rxr, rmu_q, rxr_q = oracle.averis_split_quant(x, rm, seed=1234 + l, offset=99)
     assert np.array_equal(mu.cpu().numpy().view(np.uint32), rmu.view(np.uint32))
-    assert np.array_equal(xr.cpu().numpy().view(np.uint32), rxr.view(np.uint32))
+    if debug:
+        assert np.array_equal(xr.cpu().numpy().view(np.uint32), rxr.view(np.uint32))
     assert_nvfp4_equal(xr_q, rxr_q, "X_bar_R")
     assert_nvfp4_equal(mu_q, rmu_q, "mu_bar")
 
@@ -158,3 +166,42 @@ def test_repeat_calls_reuse_workspace(api):
     assert api.averis_check_status(ws) == 0
     for o in outs[1:]:
         assert np.array_equal(o[0], outs[0][0]) and np.array_equal(o[1], outs[0][1])
+
+
+@pytest.mark.parametrize("l,K,dt", [(8192, 1024, "bf16"), (16384, 3072, "bf16"), (32768, 4096, "bf16"),
+                                    (2000, 384, "f32"), (257, 4160, "bf16")])
+def test_fused_split_matches_two_kernel_split(api, l, K, dt):
+    """The persistent one-kernel split (the unit resident in shared memory,
+    the others copied in again) gives the two-kernel chain's bytes, also where
+    every CTA has several units."""
+    Xd, _ = _x(l, K, dt, seed=l + 3 * K)
+    a = _split(api, Xd, "sr", seed=99, offset=5, debug=True)
+    b = _split(api, Xd, "sr", seed=99, offset=5, fused=True)
+    assert torch.equal(a[0], b[0])
+    for qa, qb in ((a[1], b[1]), (a[2], b[2])):
+        assert torch.equal(qa.codes, qb.codes) and torch.equal(qa.scales, qb.scales)
+        assert torch.equal(qa.g_dec, qb.g_dec)
+
+
+def test_fused_split_reuses_workspace_and_reports_nonfinite(api):
+    """The one-kernel split's grid barriers leave the workspace reusable across
+    calls and shapes; a NaN input latches AVR_ERR_NONFINITE, and after the
+    status is read the next call runs clean."""
+    ws = api.workspace(4096, 1024)
+    Xd, x = _x(1024, 512, "bf16", seed=31)
+    Yd, _ = _x(4096, 1024, "bf16", seed=32)
+    ref = oracle.averis_split_quant(x, "sr", seed=3, offset=1)
+    for _ in range(3):
+        q, m = api.NVFP4Tensor(1024, 512), api.NVFP4Tensor(1, 512)
+        api.averis_split_quant_fused(Xd, "sr", 3, 1, False, None, m, q, ws)
+        api.averis_split_quant_fused(Yd, "rne", 3, 1, False, None, None, api.NVFP4Tensor(4096, 1024), ws)
+        assert api.averis_check_status(ws) == 0
+        assert_nvfp4_equal(q, ref[3], "X_bar_R (fused, repeated)")
+    bad = Xd.clone()
+    bad[5, 7] = float("nan")
+    api.averis_split_quant_fused(bad, "rne", 0, 0, False, None, None, api.NVFP4Tensor(1024, 512), ws)
+    assert api.averis_check_status(ws) == api.AVR_ERR_NONFINITE
+    q = api.NVFP4Tensor(1024, 512)
+    api.averis_split_quant_fused(Xd, "sr", 3, 1, False, None, None, q, ws)
+    assert api.averis_check_status(ws) == 0
+    assert_nvfp4_equal(q, ref[3], "X_bar_R (fused, after an error)")
