@@ -68,6 +68,11 @@ from .averis import (
     wgrad_reference,
     averis_wgrad_reference,
     vanilla_wgrad_reference,
+    MOE_ALIGN,
+    moe_offsets,
+    moe_split_quant,
+    moe_quant_weights,
+    moe_linear_reference,
 )
 from . import stats
 

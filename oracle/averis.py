@@ -216,3 +216,72 @@ def vanilla_wgrad_reference(X, D, rounding="sr", seed=0, offset=0):
     xt_q = vanilla_quant_t(X, rounding, seed, offset, grad=False)
     dt_q = vanilla_quant_t(D, rounding, seed, offset, grad=True)
     return wgrad_reference(xt_q, dt_q), dict(xt_q=xt_q, dt_q=dt_q)
+
+
+# ---------------------------------------------------------------------------
+# MoE: one Averis linear per expert over a token buffer permuted by expert
+# ---------------------------------------------------------------------------
+# Readings (the pages name the Qwen3 7B-A1.5B MoE model and nothing more):
+#  * each expert is its own linear layer, so each gets its own split: mu_e is
+#    the mean of the tokens routed to expert e (the same fixed order, chunks
+#    counted from the first token of the segment), with its own tensor scales
+#    for X_bar_R,e and mu_bar_e;
+#  * the tokens of expert e are rows [o_e, o_e + n_e) of the permuted buffer,
+#    o_0 = 0 and o_{e+1} = o_e + n_e rounded up to 128; rows in between are
+#    padding that no statistic sees and whose outputs are undefined;
+#  * random streams: element (r, j) of the buffer counts from offset +
+#    (r K + j) / 16 as in the dense layer; mu_bar_e counts as row e of an
+#    [E, K] tensor (offset + (e K + j) / 16), with the dense layer's tags.
+
+MOE_ALIGN = 128
+
+
+def moe_offsets(counts):
+    """Row offsets o_e of the expert segments and the buffer's padded length."""
+    o, r = [], 0
+    for n in counts:
+        o.append(r)
+        r += (int(n) + MOE_ALIGN - 1) // MOE_ALIGN * MOE_ALIGN
+    return o, r
+
+
+def moe_split_quant(X, counts, rounding="sr", seed=0, offset=0, grad=False):
+    """Per-expert split of the permuted buffer X [L, K]: lists (per expert) of
+    mu_e, X_R,e, mu_bar_e, X_bar_R,e (the latter quantized as rows o_e .. of
+    the buffer)."""
+    X = _as_f32(X)
+    K = X.shape[1]
+    offs, L = moe_offsets(counts)
+    assert X.shape[0] >= L
+    t_r, t_mu = (TAGS["d_r"], TAGS["mu_d"]) if grad else (TAGS["x_r"], TAGS["mu_x"])
+    out = []
+    for e, (o, n) in enumerate(zip(offs, counts)):
+        if n == 0:
+            out.append(None)
+            continue
+        Xe = X[o:o + n]
+        _check_finite(Xe)
+        mu, XR, A = column_mean_and_residual_amax(Xe)
+        xr_q = nvfp4_quantize(XR, rounding, seed, offset + (o * K) // 16, t_r, amax=A)
+        mu_q = nvfp4_quantize(mu[None, :], rounding, seed, offset + (e * K) // 16, t_mu)
+        out.append(dict(mu=mu, xr=XR, mu_q=mu_q, xr_q=xr_q, row0=o, rows=n))
+    return out
+
+
+def moe_quant_weights(Ws):
+    """Per-expert (W_bar_fwd, W_bar_dgrad), each with its own tensor scale."""
+    return [quant_weight(W) for W in Ws]
+
+
+def moe_linear_reference(X, counts, w_qs, rounding="sr", seed=0, offset=0, grad=False):
+    """fp64 output rows of every expert's segment: Y[o_e + i] for i < n_e, the
+    Averis product of expert e (w_qs[e] = W_bar_fwd,e, or W_bar_dgrad,e for
+    grad=True).  Returns (dict row -> output row block, the split)."""
+    split = moe_split_quant(X, counts, rounding, seed, offset, grad)
+    Y = {}
+    for e, s in enumerate(split):
+        if s is None:
+            continue
+        b = bias_row(s["mu_q"], w_qs[e])
+        Y[e] = gemm_reference(s["xr_q"], w_qs[e], b)
+    return Y, split
