@@ -310,6 +310,63 @@ avr_status nvfp4_linear_wgrad(const void* X, avr_dtype xt, const void* D, avr_dt
                               void* dW, avr_dtype wt, void* ws, size_t ws_bytes, avr_stream stream);
 
 /* -------------------------------------------------------------------------
+ * Mixture of experts [Abs], [RAv]
+ *
+ * The pages train a Qwen3 7B-A1.5B MoE model with Averis and say no more.
+ * Reading: every expert is its own linear layer with its own split.  The
+ * tokens routed to expert e are rows [o_e, o_e + n_e) of a buffer permuted by
+ * expert, o_0 = 0 and o_{e+1} = o_e + n_e rounded up to 128 (rows in between
+ * are padding: no statistic sees them and their outputs are undefined).  mu_e
+ * is the mean of the expert's rows in the dense layer's fixed order (chunks
+ * from o_e); X_bar_R,e and mu_bar_e have per-expert tensor scales.  The counts
+ * n_e are a device array (int32 [E]), e.g. from a router; the buffer has
+ * l_cap rows (a multiple of 128, at least sum_e n_e rounded up per expert).
+ * Random streams: row r of the buffer as in the dense layer; mu_bar_e as row
+ * e of an [E, K] tensor.  Limits: E <= 1024, E * ceil(K / 128) <= 4096,
+ * N % 128 == 0.  A segment table that does not fit l_cap latches
+ * AVR_ERR_INVALID_ARG and nothing is computed.
+ * NVFP4 tensors of the MoE calls hold E decode scales (g_dec[E]):
+ *   xr_q [l_cap, K]: rows of expert e scaled by g_dec[e];
+ *   mu_q [E, K]: row e is mu_bar_e;
+ *   w_fwd [E * n, m/2] and w_dgrad [E * m, n/2]: the experts stacked.
+ * ------------------------------------------------------------------------- */
+
+/* Workspace bytes of the MoE calls (N = output features per expert; 0 for
+ * averis_moe_split_quant). */
+size_t averis_moe_workspace_size(int64_t l_cap, int64_t K, int64_t N, int E);
+
+/* Per-expert quantization of W [E][m][n] (each expert's own tensor scale),
+ * RNE, into the stacked w_fwd / w_dgrad.  ws: averis_workspace_size(m, n, n).
+ * m % 128 == 0 and n % 128 == 0. */
+avr_status averis_moe_quant_weights(const void* W, avr_dtype wt, int E, int64_t m, int64_t n,
+                                    const avr_nvfp4* w_fwd, const avr_nvfp4* w_dgrad, void* ws,
+                                    size_t ws_bytes, avr_stream stream);
+
+/* Per-expert split of X [l_cap, K]: mu [E][K] (nullable), mu_q (nullable),
+ * xr_q (padding rows: zero codes and scales).  grad selects the stream tags
+ * as in averis_split_quant.  Launches 3 kernels (table, reduce, quantize). */
+avr_status averis_moe_split_quant(const void* X, avr_dtype xt, int64_t l_cap, const int32_t* counts, int E,
+                                  int64_t K, avr_round rm, uint64_t seed, uint64_t offset, int grad, float* mu,
+                                  const avr_nvfp4* mu_q, const avr_nvfp4* xr_q, void* ws, size_t ws_bytes,
+                                  avr_stream stream);
+
+/* Forward of the MoE layer: Y[o_e + i] = 1 (mu_bar_e W_bar_e) + X_bar_R,e W_bar_e
+ * for every expert, one grouped block-scaled GEMM over all segments.
+ * X [l_cap, m], Y [l_cap, n].  Launches 5 kernels (table, reduce, quantize,
+ * rank-one rows, grouped GEMM). */
+avr_status averis_moe_linear_fwd(const void* X, avr_dtype xt, int64_t l_cap, const int32_t* counts, int E,
+                                 int64_t m, int64_t n, const avr_nvfp4* w_fwd, avr_round rm, uint64_t seed,
+                                 uint64_t offset, void* Y, avr_dtype yt, void* ws, size_t ws_bytes,
+                                 avr_stream stream);
+
+/* Dgrad of the MoE layer: dX[o_e + i] from D [l_cap, n] and w_dgrad, as the
+ * forward with the split of D (stream tags 3 and 4). */
+avr_status averis_moe_linear_dgrad(const void* D, avr_dtype dt, int64_t l_cap, const int32_t* counts, int E,
+                                   int64_t m, int64_t n, const avr_nvfp4* w_dgrad, avr_round rm, uint64_t seed,
+                                   uint64_t offset, void* dX, avr_dtype xt, void* ws, size_t ws_bytes,
+                                   avr_stream stream);
+
+/* -------------------------------------------------------------------------
  * Diagnostics (used by the tests to pin the number formats on the device)
  * ------------------------------------------------------------------------- */
 

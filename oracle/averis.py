@@ -245,10 +245,11 @@ def moe_offsets(counts):
     return o, r
 
 
-def moe_split_quant(X, counts, rounding="sr", seed=0, offset=0, grad=False):
+def moe_split_quant(X, counts, rounding="sr", seed=0, offset=0, grad=False, experts=None):
     """Per-expert split of the permuted buffer X [L, K]: lists (per expert) of
     mu_e, X_R,e, mu_bar_e, X_bar_R,e (the latter quantized as rows o_e .. of
-    the buffer)."""
+    the buffer).  `experts` restricts the work to those experts (the others
+    are None)."""
     X = _as_f32(X)
     K = X.shape[1]
     offs, L = moe_offsets(counts)
@@ -256,7 +257,7 @@ def moe_split_quant(X, counts, rounding="sr", seed=0, offset=0, grad=False):
     t_r, t_mu = (TAGS["d_r"], TAGS["mu_d"]) if grad else (TAGS["x_r"], TAGS["mu_x"])
     out = []
     for e, (o, n) in enumerate(zip(offs, counts)):
-        if n == 0:
+        if n == 0 or (experts is not None and e not in experts):
             out.append(None)
             continue
         Xe = X[o:o + n]
@@ -273,11 +274,11 @@ def moe_quant_weights(Ws):
     return [quant_weight(W) for W in Ws]
 
 
-def moe_linear_reference(X, counts, w_qs, rounding="sr", seed=0, offset=0, grad=False):
+def moe_linear_reference(X, counts, w_qs, rounding="sr", seed=0, offset=0, grad=False, experts=None):
     """fp64 output rows of every expert's segment: Y[o_e + i] for i < n_e, the
     Averis product of expert e (w_qs[e] = W_bar_fwd,e, or W_bar_dgrad,e for
     grad=True).  Returns (dict row -> output row block, the split)."""
-    split = moe_split_quant(X, counts, rounding, seed, offset, grad)
+    split = moe_split_quant(X, counts, rounding, seed, offset, grad, experts)
     Y = {}
     for e, s in enumerate(split):
         if s is None:

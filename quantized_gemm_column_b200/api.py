@@ -59,6 +59,18 @@ _SIGS = {
     "averis_split_quant": (_c_int, [_c_ptr, _c_int, _c_i64, _c_i64, _c_int, _c_u64, _c_u64, _c_int,
                                     _c_ptr, ctypes.POINTER(avr_nvfp4), ctypes.POINTER(avr_nvfp4),
                                     _c_ptr, _c_ptr, _c_size, _c_ptr]),
+    "averis_moe_workspace_size": (_c_size, [_c_i64, _c_i64, _c_i64, _c_int]),
+    "averis_moe_quant_weights": (_c_int, [_c_ptr, _c_int, _c_int, _c_i64, _c_i64, ctypes.POINTER(avr_nvfp4),
+                                          ctypes.POINTER(avr_nvfp4), _c_ptr, _c_size, _c_ptr]),
+    "averis_moe_split_quant": (_c_int, [_c_ptr, _c_int, _c_i64, _c_ptr, _c_int, _c_i64, _c_int, _c_u64, _c_u64,
+                                        _c_int, _c_ptr, ctypes.POINTER(avr_nvfp4), ctypes.POINTER(avr_nvfp4),
+                                        _c_ptr, _c_size, _c_ptr]),
+    "averis_moe_linear_fwd": (_c_int, [_c_ptr, _c_int, _c_i64, _c_ptr, _c_int, _c_i64, _c_i64,
+                                       ctypes.POINTER(avr_nvfp4), _c_int, _c_u64, _c_u64, _c_ptr, _c_int, _c_ptr,
+                                       _c_size, _c_ptr]),
+    "averis_moe_linear_dgrad": (_c_int, [_c_ptr, _c_int, _c_i64, _c_ptr, _c_int, _c_i64, _c_i64,
+                                         ctypes.POINTER(avr_nvfp4), _c_int, _c_u64, _c_u64, _c_ptr, _c_int,
+                                         _c_ptr, _c_size, _c_ptr]),
     "averis_split_quant_fused": (_c_int, [_c_ptr, _c_int, _c_i64, _c_i64, _c_int, _c_u64, _c_u64, _c_int,
                                           _c_ptr, ctypes.POINTER(avr_nvfp4), ctypes.POINTER(avr_nvfp4),
                                           _c_ptr, _c_size, _c_ptr]),
@@ -265,6 +277,58 @@ def averis_mean_energy_ratio(X, mu, R, ws, stream=None):
     l, K = X.shape
     _check(load().averis_mean_energy_ratio(_ptr(X), _dtype(X), l, K, _ptr(mu), _ptr(R), _ptr(ws),
                                            ws.numel(), _stream(stream)), "averis_mean_energy_ratio")
+
+
+class NVFP4Group(NVFP4Tensor):
+    """An NVFP4 tensor [rows, K] with one decode scale per expert (MoE calls)."""
+
+    def __init__(self, rows, K, groups, device="cuda"):
+        super().__init__(rows, K, device)
+        self.g_dec = torch.empty(groups, dtype=torch.float32, device=device)
+
+
+def moe_padded_rows(counts):
+    """Rows the permuted buffer needs: every expert's count rounded up to 128."""
+    return sum((int(c) + 127) // 128 * 128 for c in counts)
+
+
+def averis_moe_workspace_size(l_cap, K, N, E):
+    return int(load().averis_moe_workspace_size(l_cap, K, N, E))
+
+
+def moe_workspace(l_cap, K, N, E, device="cuda", stream=None):
+    ws = torch.empty(averis_moe_workspace_size(l_cap, K, N, E), dtype=torch.uint8, device=device)
+    averis_workspace_init(ws, stream)
+    return ws
+
+
+def averis_moe_quant_weights(W, w_fwd, w_dgrad, ws, stream=None):
+    E, m, n = W.shape
+    _check(load().averis_moe_quant_weights(_ptr(W), _dtype(W), E, m, n, _s(w_fwd), _s(w_dgrad), _ptr(ws),
+                                           ws.numel(), _stream(stream)), "averis_moe_quant_weights")
+
+
+def averis_moe_split_quant(X, counts, rm, seed, offset, grad, mu, mu_q, xr_q, ws, stream=None):
+    l_cap, K = X.shape
+    _check(load().averis_moe_split_quant(_ptr(X), _dtype(X), l_cap, _ptr(counts), counts.numel(), K, _round(rm),
+                                         seed, offset, int(grad), _ptr(mu), _s(mu_q), _s(xr_q), _ptr(ws),
+                                         ws.numel(), _stream(stream)), "averis_moe_split_quant")
+
+
+def averis_moe_linear_fwd(X, counts, w_fwd, rm, seed, offset, Y, ws, stream=None):
+    l_cap, m = X.shape
+    n = Y.shape[1]
+    _check(load().averis_moe_linear_fwd(_ptr(X), _dtype(X), l_cap, _ptr(counts), counts.numel(), m, n,
+                                        _s(w_fwd), _round(rm), seed, offset, _ptr(Y), _dtype(Y), _ptr(ws),
+                                        ws.numel(), _stream(stream)), "averis_moe_linear_fwd")
+
+
+def averis_moe_linear_dgrad(D, counts, w_dgrad, rm, seed, offset, dX, ws, stream=None):
+    l_cap, n = D.shape
+    m = dX.shape[1]
+    _check(load().averis_moe_linear_dgrad(_ptr(D), _dtype(D), l_cap, _ptr(counts), counts.numel(), m, n,
+                                          _s(w_dgrad), _round(rm), seed, offset, _ptr(dX), _dtype(dX), _ptr(ws),
+                                          ws.numel(), _stream(stream)), "averis_moe_linear_dgrad")
 
 
 def averis_split_quant_fused(X, rm, seed, offset, grad, mu, mu_q, xr_q, ws, stream=None):

@@ -682,6 +682,230 @@ avr_status nvfp4_linear_wgrad(const void* X, avr_dtype xt, const void* D, avr_dt
   return linear_wgrad(X, xt, D, dt, l, m, n, 0, rm, seed, offset, dW, wt, ws, ws_bytes, stream);
 }
 
+// ---------------------------------------------------------------------------
+// mixture of experts
+// ---------------------------------------------------------------------------
+static int moe_c_max(int64_t l_cap, int E) {
+  return static_cast<int>((l_cap + kChunkRows - 1) / kChunkRows) + E;
+}
+
+// status, tickets and slots at the fixed offsets of WsLayout, then the
+// grouped reduce's partials, the segment table, the per-expert means, their
+// NVFP4 form, the rank-one rows and the split residual
+struct MoeLayout {
+  WsLayout base;              // status, tickets, slots, partials [3][c_max][K]
+  size_t seg = 0, totals = 0, chunk_expert = 0, block_expert = 0;
+  size_t mu = 0, mu_codes = 0, mu_scales = 0, mu_gdec = 0, xr_gdec = 0, bias = 0;
+  size_t xr_codes = 0, xr_scales = 0;
+  size_t total = 0;
+};
+
+static MoeLayout moe_layout(int64_t l_cap, int64_t K, int64_t N, int E) {
+  MoeLayout w;
+  const size_t C = static_cast<size_t>(moe_c_max(l_cap, E));
+  const size_t Ks = static_cast<size_t>(K), Ns = static_cast<size_t>(N), Es = static_cast<size_t>(E);
+  size_t off = round_up(w.base.slots + 2 * sizeof(float) * kMaxColTiles, 256);
+  w.base.partials = off; off = round_up(off + 3 * C * Ks * sizeof(float), 256);
+  w.seg = off;           off = round_up(off + Es * sizeof(MoeSeg), 256);
+  w.totals = off;        off += 256;
+  w.chunk_expert = off;  off = round_up(off + C * sizeof(int32_t), 256);
+  w.block_expert = off;  off = round_up(off + static_cast<size_t>(l_cap / 128) * sizeof(int32_t), 256);
+  w.mu = off;            off = round_up(off + Es * Ks * sizeof(float), 256);
+  w.mu_codes = off;      off = round_up(off + Es * Ks / 2, 256);
+  w.mu_scales = off;     off = round_up(off + scales_bytes(E, K), 256);
+  w.mu_gdec = off;       off = round_up(off + Es * sizeof(float), 256);
+  w.xr_gdec = off;       off = round_up(off + Es * sizeof(float), 256);
+  w.bias = off;          off = round_up(off + Es * Ns * sizeof(float), 256);
+  w.xr_codes = off;      off = round_up(off + static_cast<size_t>(l_cap) * Ks / 2, 256);
+  w.xr_scales = off;     off = round_up(off + scales_bytes(l_cap, K), 256);
+  w.total = off;
+  return w;
+}
+
+static bool moe_shape_ok(int64_t l_cap, int E, int64_t K) {
+  return l_cap >= 0 && l_cap % 128 == 0 && l_cap <= kMaxDim && E >= 1 && E <= 1024 && k_ok(K) &&
+         static_cast<int64_t>(E) * ((K + kColTile - 1) / kColTile) <= kMaxColTiles;
+}
+
+static avr_status make_moe_ws(void* ws, size_t ws_bytes, int64_t l_cap, int64_t K, int64_t N, int E,
+                              MoeLayout* lay, Ws* w) {
+  if (!ws) return AVR_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return AVR_ERR_MISALIGNED;
+  *lay = moe_layout(l_cap, K, N, E);
+  if (ws_bytes < lay->total) return AVR_ERR_WORKSPACE_TOO_SMALL;
+  w->base = static_cast<char*>(ws);
+  w->lay = lay->base;
+  return AVR_OK;
+}
+
+// segment table, grouped reduce and grouped quantizer (the per-expert split)
+static avr_status moe_split_chain(const void* X, avr_dtype xt, int64_t l_cap, const int32_t* counts, int E,
+                                  int64_t K, avr_round rm, uint64_t seed, uint64_t offset, uint32_t tag,
+                                  uint32_t tag_mu, float* mu, const avr_nvfp4* mu_q, const avr_nvfp4* xr_q,
+                                  const Ws& w, const MoeLayout& lay, cudaStream_t s) {
+  const int c_max = moe_c_max(l_cap, E);
+  MoeSeg* seg = w.at<MoeSeg>(lay.seg);
+  int32_t* totals = w.at<int32_t>(lay.totals);
+  int32_t* chunk_expert = w.at<int32_t>(lay.chunk_expert);
+  int32_t* block_expert = w.at<int32_t>(lay.block_expert);
+  AVR_TRY(cuda_status(launch_moe_table(counts, E, l_cap, c_max, seg, chunk_expert, block_expert, totals,
+                                       w.status(), s, true)));
+  ColReduceArgs ca;
+  ca.X = X;
+  ca.xt = xt;
+  ca.l = l_cap;
+  ca.K = K;
+  ca.split = 1;
+  ca.mu_out = mu;
+  ca.energy = 0;
+  ca.ws = w.base;
+  ca.lay = &w.lay;
+  ca.seg = seg;
+  ca.chunk_expert = chunk_expert;
+  ca.totals = totals;
+  ca.c_max = c_max;
+  AVR_TRY(cuda_status(launch_colreduce(ca, s, true)));
+  MoeQuantArgs qa = {};
+  qa.X = X;
+  qa.xt = xt;
+  qa.l_cap = l_cap;
+  qa.K = K;
+  qa.E = E;
+  qa.seg = seg;
+  qa.block_expert = block_expert;
+  qa.totals = totals;
+  qa.mu = mu;
+  qa.slot_xr = w.slot_xr();
+  qa.slot_mu = w.slot_mu();
+  qa.codes = xr_q->codes;
+  qa.scales = xr_q->scales;
+  qa.g_dec = xr_q->g_dec;
+  if (mu_q) {
+    qa.mu_codes = mu_q->codes;
+    qa.mu_scales = mu_q->scales;
+    qa.mu_gdec = mu_q->g_dec;
+  }
+  qa.seed = seed;
+  qa.offset = offset;
+  qa.tag = tag;
+  qa.tag_mu = tag_mu;
+  qa.sr = rm == AVR_SR;
+  qa.status = w.status();
+  return cuda_status(launch_moe_quant(qa, s, true));
+}
+
+size_t averis_moe_workspace_size(int64_t l_cap, int64_t K, int64_t N, int E) {
+  if (!moe_shape_ok(l_cap, E, K) || N < 0) return 0;
+  return moe_layout(l_cap, K, N, E).total;
+}
+
+avr_status averis_moe_split_quant(const void* X, avr_dtype xt, int64_t l_cap, const int32_t* counts, int E,
+                                  int64_t K, avr_round rm, uint64_t seed, uint64_t offset, int grad, float* mu,
+                                  const avr_nvfp4* mu_q, const avr_nvfp4* xr_q, void* ws, size_t ws_bytes,
+                                  avr_stream stream) {
+  if (!dtype_ok(xt) || !round_ok(rm)) return AVR_ERR_INVALID_ARG;
+  if (!moe_shape_ok(l_cap, E, K)) return AVR_ERR_UNSUPPORTED_SHAPE;
+  if (!X || !counts || !xr_q || !xr_q->g_dec) return AVR_ERR_INVALID_ARG;
+  AVR_TRY(check_nvfp4(xr_q, l_cap, K));
+  if (mu_q) AVR_TRY(check_nvfp4(mu_q, E, K));
+  if (!aligned16(X) || !aligned16(mu) || (reinterpret_cast<uintptr_t>(counts) & 3u)) return AVR_ERR_MISALIGNED;
+  MoeLayout lay;
+  Ws w;
+  AVR_TRY(make_moe_ws(ws, ws_bytes, l_cap, K, 0, E, &lay, &w));
+  AVR_TRY(device_ok());
+  if (l_cap == 0) return AVR_OK;
+  return moe_split_chain(X, xt, l_cap, counts, E, K, rm, seed, offset, grad ? 3u : 1u, grad ? 4u : 2u,
+                         mu ? mu : w.at<float>(lay.mu), mu_q, xr_q, w, lay, stream);
+}
+
+avr_status averis_moe_quant_weights(const void* W, avr_dtype wt, int E, int64_t m, int64_t n,
+                                    const avr_nvfp4* w_fwd, const avr_nvfp4* w_dgrad, void* ws, size_t ws_bytes,
+                                    avr_stream stream) {
+  if (!W || !dtype_ok(wt) || E < 1 || E > 1024) return AVR_ERR_INVALID_ARG;
+  if (!k_ok(m) || !k_ok(n) || m % 128 || n % 128) return AVR_ERR_UNSUPPORTED_SHAPE;
+  AVR_TRY(check_nvfp4(w_fwd, static_cast<int64_t>(E) * n, m));
+  AVR_TRY(check_nvfp4(w_dgrad, static_cast<int64_t>(E) * m, n));
+  const size_t elem = wt == AVR_BF16 ? 2 : 4;
+  for (int e = 0; e < E; ++e) {
+    // expert e's slices: its W [m, n], rows e n .. of W_bar_fwd, e m .. of W_bar_dgrad
+    const avr_nvfp4 f = {w_fwd->codes + static_cast<size_t>(e) * n * (m / 2),
+                         w_fwd->scales + static_cast<size_t>(e) * scales_bytes(n, m), w_fwd->g_dec + e, n, m};
+    const avr_nvfp4 d = {w_dgrad->codes + static_cast<size_t>(e) * m * (n / 2),
+                         w_dgrad->scales + static_cast<size_t>(e) * scales_bytes(m, n), w_dgrad->g_dec + e, m, n};
+    AVR_TRY(averis_quant_weight(static_cast<const char*>(W) + static_cast<size_t>(e) * m * n * elem, wt, m, n, &f,
+                                &d, ws, ws_bytes, stream));
+  }
+  return AVR_OK;
+}
+
+static avr_status moe_linear(const void* X, avr_dtype xt, int64_t l_cap, const int32_t* counts, int E, int64_t K,
+                             int64_t N, const avr_nvfp4* wq, avr_round rm, uint64_t seed, uint64_t offset,
+                             uint32_t tag, uint32_t tag_mu, void* Y, avr_dtype yt, void* ws, size_t ws_bytes,
+                             avr_stream stream) {
+  if (!dtype_ok(xt) || !dtype_ok(yt) || !round_ok(rm)) return AVR_ERR_INVALID_ARG;
+  if (!moe_shape_ok(l_cap, E, K) || !n_ok(N) || N % 128) return AVR_ERR_UNSUPPORTED_SHAPE;
+  if (!X || !Y || !counts) return AVR_ERR_INVALID_ARG;
+  AVR_TRY(check_nvfp4(wq, static_cast<int64_t>(E) * N, K));
+  if (!aligned16(X) || !aligned16(Y) || (reinterpret_cast<uintptr_t>(counts) & 3u)) return AVR_ERR_MISALIGNED;
+  MoeLayout lay;
+  Ws w;
+  AVR_TRY(make_moe_ws(ws, ws_bytes, l_cap, K, N, E, &lay, &w));
+  AVR_TRY(device_ok());
+  if (l_cap == 0) return AVR_OK;
+  const avr_nvfp4 xr = {w.at<uint8_t>(lay.xr_codes), w.at<uint8_t>(lay.xr_scales), w.at<float>(lay.xr_gdec),
+                        l_cap, K};
+  const avr_nvfp4 muq = {w.at<uint8_t>(lay.mu_codes), w.at<uint8_t>(lay.mu_scales), w.at<float>(lay.mu_gdec),
+                         E, K};
+  AVR_TRY(moe_split_chain(X, xt, l_cap, counts, E, K, rm, seed, offset, tag, tag_mu, w.at<float>(lay.mu), &muq,
+                          &xr, w, lay, stream));
+  MoeBiasArgs ba;
+  ba.seg = w.at<MoeSeg>(lay.seg);
+  ba.totals = w.at<int32_t>(lay.totals);
+  ba.E = E;
+  ba.K = K;
+  ba.N = N;
+  ba.mu_codes = muq.codes;
+  ba.mu_scales = muq.scales;
+  ba.mu_gdec = muq.g_dec;
+  ba.w_codes = wq->codes;
+  ba.w_scales = wq->scales;
+  ba.w_gdec = wq->g_dec;
+  ba.bias = w.at<float>(lay.bias);
+  AVR_TRY(cuda_status(launch_moe_bias(ba, stream, true)));
+  GemmArgs g;
+  g.a_codes = xr.codes;
+  g.a_scales = xr.scales;
+  g.a_gdec = xr.g_dec;
+  g.b_codes = wq->codes;
+  g.b_scales = wq->scales;
+  g.b_gdec = wq->g_dec;
+  g.M = l_cap;
+  g.N = N;
+  g.K = K;
+  g.bias = ba.bias;
+  g.Y = Y;
+  g.yt = yt;
+  g.status = w.status();
+  g.groups = E;
+  g.block_expert = w.at<int32_t>(lay.block_expert);
+  g.totals = ba.totals;
+  return cuda_status(launch_gemm(g, stream, true));
+}
+
+avr_status averis_moe_linear_fwd(const void* X, avr_dtype xt, int64_t l_cap, const int32_t* counts, int E,
+                                 int64_t m, int64_t n, const avr_nvfp4* w_fwd, avr_round rm, uint64_t seed,
+                                 uint64_t offset, void* Y, avr_dtype yt, void* ws, size_t ws_bytes,
+                                 avr_stream stream) {
+  return moe_linear(X, xt, l_cap, counts, E, m, n, w_fwd, rm, seed, offset, 1u, 2u, Y, yt, ws, ws_bytes, stream);
+}
+
+avr_status averis_moe_linear_dgrad(const void* D, avr_dtype dt, int64_t l_cap, const int32_t* counts, int E,
+                                   int64_t m, int64_t n, const avr_nvfp4* w_dgrad, avr_round rm, uint64_t seed,
+                                   uint64_t offset, void* dX, avr_dtype xt, void* ws, size_t ws_bytes,
+                                   avr_stream stream) {
+  return moe_linear(D, dt, l_cap, counts, E, n, m, w_dgrad, rm, seed, offset, 3u, 4u, dX, xt, ws, ws_bytes, stream);
+}
+
 avr_status averis_probe_convert(const float* in, uint8_t* e4m3, uint8_t* e2m1, int64_t n,
                                 avr_stream stream) {
   if (!in || n < 0) return AVR_ERR_INVALID_ARG;

@@ -33,9 +33,15 @@ struct ColReduceParams {
   float* part_e;          // [C][K]: sum of squares (energy pass only)
   float* energy;          // [K] column sums of squares, chunks in order (energy pass only)
   uint32_t* status;
+  // grouped (MoE) mode: blockIdx.y is a global chunk index; chunk_expert maps it
+  // to its expert, whose segment, chunk range, mean and slots it uses (null: dense)
+  const MoeSeg* seg;
+  const int32_t* chunk_expert;
+  const int32_t* totals;  // [1]: chunks in use
+  int T;                  // column tiles (slot and ticket stride per expert)
 };
 
-template <bool kBf16, bool kEnergy>
+template <bool kBf16, bool kEnergy, bool kGrouped>
 __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_constant__ CUtensorMap map,
                                                              const ColReduceParams p) {
   extern __shared__ __align__(1024) uint8_t tile[];
@@ -45,10 +51,26 @@ __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_consta
 
   const int tid = threadIdx.x;
   const int t = blockIdx.x;
-  const int c = blockIdx.y;
+  const int c = blockIdx.y;                    // chunk index into the partials
   const int64_t col = static_cast<int64_t>(t) * kColTile + tid;
-  const int64_t row0 = static_cast<int64_t>(c) * kChunkRows;
-  const int rows = static_cast<int>(min64(kChunkRows, p.l - row0));
+  // this chunk's rows, the chunks folded with it, the slot and mean it feeds
+  int64_t row0 = static_cast<int64_t>(c) * kChunkRows;
+  int64_t n_rows = p.l;                        // rows of the (expert's) matrix
+  int c_first = 0, c_count = p.C, slot = t;
+  float* mu_out = p.mu_out;
+  if (kGrouped) {
+    pdl_wait_prior_grid();                     // the segment table comes from the previous launch
+    if (c >= __ldcg(p.totals)) return;         // a chunk past the last expert's
+    const int e = __ldcg(p.chunk_expert + c);
+    const MoeSeg sg = p.seg[e];
+    c_first = sg.chunk0;
+    c_count = sg.chunks;
+    row0 = sg.row0 + static_cast<int64_t>(c - sg.chunk0) * kChunkRows;
+    n_rows = sg.rows;
+    slot = e * p.T + t;
+    mu_out = p.mu_out + static_cast<int64_t>(e) * p.K;
+  }
+  const int rows = static_cast<int>(min64(kChunkRows, n_rows - static_cast<int64_t>(c - c_first) * kChunkRows));
   constexpr uint32_t kElem = kBf16 ? 2u : 4u;
   constexpr uint32_t kTileBytes = kChunkRows * kColTile * kElem;
 
@@ -107,8 +129,8 @@ __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_consta
   // barrier) and, for the last CTA, makes every other CTA's partials visible
   // to the fold below (acquire, passed on by the second barrier).
   __syncthreads();
-  if (tid == 0) s_last = ticket_inc_acq_rel(&p.tickets[t], static_cast<uint32_t>(p.C - 1)) ==
-                         static_cast<uint32_t>(p.C - 1);
+  if (tid == 0) s_last = ticket_inc_acq_rel(&p.tickets[slot], static_cast<uint32_t>(c_count - 1)) ==
+                         static_cast<uint32_t>(c_count - 1);
   __syncthreads();
   if (!s_last) return;
 
@@ -120,12 +142,12 @@ __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_consta
   if (col < p.K) {
     constexpr int kBatch = 16;
     const int64_t plane = static_cast<int64_t>(p.C) * p.K;
-    for (int c0 = 0; c0 < p.C; c0 += kBatch) {
+    for (int c0 = 0; c0 < c_count; c0 += kBatch) {
       float ps[kBatch], px[kBatch], pn[kBatch];
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
-        if (c0 + u < p.C) {
-          const int64_t o = static_cast<int64_t>(c0 + u) * p.K + col;
+        if (c0 + u < c_count) {
+          const int64_t o = static_cast<int64_t>(c_first + c0 + u) * p.K + col;
           ps[u] = __ldcg(&p.part[o]);
           px[u] = __ldcg(&p.part[plane + o]);
           pn[u] = __ldcg(&p.part[2 * plane + o]);
@@ -133,7 +155,7 @@ __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_consta
       }
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
-        if (c0 + u < p.C) {
+        if (c0 + u < c_count) {
           S = __fadd_rn(S, ps[u]);
           cmax = fmaxf(cmax, px[u]);
           cmin = fminf(cmin, pn[u]);
@@ -158,11 +180,11 @@ __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_consta
   if (col < p.K) {
     if (!isfinite(S)) raise_status(p.status, AVR_ERR_NONFINITE);
     if (p.split) {
-      const float mu = __fdiv_rn(S, static_cast<float>(p.l));
+      const float mu = __fdiv_rn(S, static_cast<float>(n_rows));
       if (!isfinite(mu)) raise_status(p.status, AVR_ERR_NONFINITE);
       a_xr = fmaxf(__fsub_rn(cmax, mu), __fsub_rn(mu, cmin));
       a_mu = fabsf(mu);
-      p.mu_out[col] = mu;
+      mu_out[col] = mu;
     } else {
       a_xr = fmaxf(cmax, -cmin);
     }
@@ -184,18 +206,18 @@ __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_consta
       x = fmaxf(x, s_red[0][w]);
       m = fmaxf(m, s_red[1][w]);
     }
-    p.slot_xr[t] = x;
-    p.slot_mu[t] = m;
+    p.slot_xr[slot] = x;
+    p.slot_mu[slot] = m;
   }
 }
 
-template <bool kBf16, bool kEnergy>
+template <bool kBf16, bool kEnergy, bool kGrouped>
 static cudaError_t launch_colreduce_t(const CUtensorMap& map, const ColReduceParams& p, dim3 grid, size_t smem,
                                       cudaStream_t s, bool pdl) {
-  const void* fn = reinterpret_cast<const void*>(colreduce_kernel<kBf16, kEnergy>);
+  const void* fn = reinterpret_cast<const void*>(colreduce_kernel<kBf16, kEnergy, kGrouped>);
   cudaError_t e = set_max_dynamic_smem(fn, smem);
   if (e != cudaSuccess) return e;
-  return launch_ex(colreduce_kernel<kBf16, kEnergy>, grid, dim3(kColTile), smem, s, pdl, map, p);
+  return launch_ex(colreduce_kernel<kBf16, kEnergy, kGrouped>, grid, dim3(kColTile), smem, s, pdl, map, p);
 }
 
 cudaError_t launch_colreduce(const ColReduceArgs& a, cudaStream_t s, bool pdl) {
@@ -209,7 +231,7 @@ cudaError_t launch_colreduce(const ColReduceArgs& a, cudaStream_t s, bool pdl) {
   ColReduceParams p;
   p.l = a.l;
   p.K = a.K;
-  p.C = static_cast<int>((a.l + kChunkRows - 1) / kChunkRows);
+  p.C = a.seg ? a.c_max : static_cast<int>((a.l + kChunkRows - 1) / kChunkRows);
   p.split = a.split;
   p.part = reinterpret_cast<float*>(a.ws + a.lay->partials);
   p.tickets = reinterpret_cast<uint32_t*>(a.ws + a.lay->tickets);
@@ -219,15 +241,23 @@ cudaError_t launch_colreduce(const ColReduceArgs& a, cudaStream_t s, bool pdl) {
   p.part_e = reinterpret_cast<float*>(a.ws + a.lay->energy_partials);
   p.energy = reinterpret_cast<float*>(a.ws + a.lay->energy);
   p.status = reinterpret_cast<uint32_t*>(a.ws + a.lay->status);
+  p.seg = a.seg;
+  p.chunk_expert = a.chunk_expert;
+  p.totals = a.totals;
   const int T = static_cast<int>((a.K + kColTile - 1) / kColTile);
+  p.T = T;
+  if (p.C < 1) return cudaSuccess;
   const size_t smem = static_cast<size_t>(kChunkRows) * kColTile * elem;
   const dim3 grid(T, p.C);
+  if (a.seg != nullptr)   // grouped (MoE): no energy pass
+    return bf16 ? launch_colreduce_t<true, false, true>(map, p, grid, smem, s, pdl)
+                : launch_colreduce_t<false, false, true>(map, p, grid, smem, s, pdl);
   if (a.energy) {
-    return bf16 ? launch_colreduce_t<true, true>(map, p, grid, smem, s, pdl)
-                : launch_colreduce_t<false, true>(map, p, grid, smem, s, pdl);
+    return bf16 ? launch_colreduce_t<true, true, false>(map, p, grid, smem, s, pdl)
+                : launch_colreduce_t<false, true, false>(map, p, grid, smem, s, pdl);
   }
-  return bf16 ? launch_colreduce_t<true, false>(map, p, grid, smem, s, pdl)
-              : launch_colreduce_t<false, false>(map, p, grid, smem, s, pdl);
+  return bf16 ? launch_colreduce_t<true, false, false>(map, p, grid, smem, s, pdl)
+              : launch_colreduce_t<false, false, false>(map, p, grid, smem, s, pdl);
 }
 
 // ---------------------------------------------------------------------------

@@ -102,6 +102,12 @@ struct GemmParams {
   const float* bias;
   const float* row_scale;   // rank-one epilogue only: Y = alpha acc + row_scale[i] bias[j]
   uint32_t* status;
+  // grouped (MoE) mode, null for one GEMM: A's 128-row block b belongs to
+  // expert block_expert[b], whose B rows start at e * N (experts stacked), and
+  // whose decode scales and bias row are gdec_a[e], gdec_b[e], bias + e * N;
+  // totals[1] = the rows in use (a multiple of 128)
+  const int32_t* block_expert;
+  const int32_t* totals;
 };
 
 // The contiguous run of tiles [first, first + count) of this CTA; tile t is
@@ -116,7 +122,7 @@ struct TileRun {
   }
 };
 
-template <int BN, bool kBf16Out, bool kRank1>
+template <int BN, bool kBf16Out, bool kRank1, bool kGrouped>
 __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                       const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
@@ -146,7 +152,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_kst = static_cast<int>((p.K + Cfg::kStageK - 1) / Cfg::kStageK);
   const bool res = p.sfb_resident != 0;
-  const TileRun run(p.num_tiles);
+  constexpr bool grouped = kGrouped;
 
   if (threadIdx.x == 0) {
     prefetch_tensormap(&map_a);
@@ -176,6 +182,14 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   pdl_wait_prior_grid();
   pdl_allow_next_grid();
+  // grouped: only the blocks of the experts' segments are tiles (a device count)
+  int tiles_m = p.tiles_m, num_tiles = p.num_tiles;
+  if (grouped) {
+    tiles_m = __ldcg(p.totals + 1) / Cfg::kBM;
+    num_tiles = tiles_m * (p.num_tiles / p.tiles_m);
+  }
+  const TileRun run(num_tiles);
+  auto expert_of = [&](int32_t m0) { return grouped ? __ldg(p.block_expert + m0 / Cfg::kBM) : 0; };
 
   if (warp >= 1 && warp <= 4) {
     if (lane == 0) {
@@ -185,7 +199,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
         // B's scales for all of K, once per column block
         int n_prev = -1, uses = 0;
         for (int i = 0; i < run.count; ++i) {
-          const int n_blk = (run.first + i) / p.tiles_m;
+          const int n_blk = (run.first + i) / tiles_m;
           if (n_blk == n_prev) continue;
           n_prev = n_blk;
           if (uses >= 1 && !mbar_wait(res_empty, static_cast<uint32_t>(uses - 1) & 1u, p.status)) break;
@@ -200,8 +214,9 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
         bool ok = true;
         for (int i = 0; i < run.count && ok; ++i) {
           const int tile = run.first + i;
-          const int32_t m0 = (tile % p.tiles_m) * Cfg::kBM;
-          const int32_t n0 = (tile / p.tiles_m) * Cfg::kBN;
+          const int32_t m0 = (tile % tiles_m) * Cfg::kBM;
+          const int32_t n0 = (tile / tiles_m) * Cfg::kBN;
+          const int32_t nb0 = n0 + (grouped ? expert_of(m0) * static_cast<int32_t>(p.N) : 0);   // B's first row
           for (int ks = 0; ks < n_kst; ++ks, ++it) {
             if (it >= Cfg::kStages && !mbar_wait(&empty[st], ph ^ 1u, p.status)) {
               ok = false;
@@ -212,14 +227,14 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
               tma_load_2d(sA + st * Cfg::kABytes, &map_a, &full[st], ks * Cfg::kRowBytes, m0);
             } else if (role == 1) {
               mbar_arrive_expect_tx(&full[st], Cfg::kBBytes);
-              tma_load_2d(sB + st * Cfg::kBBytes, &map_b, &full[st], ks * Cfg::kRowBytes, n0);
+              tma_load_2d(sB + st * Cfg::kBBytes, &map_b, &full[st], ks * Cfg::kRowBytes, nb0);
             } else if (role == 2) {
               // 4 atoms (2 KB) of the tile's 128-row group, as 256 eight-byte elements
               mbar_arrive_expect_tx(&full[st], Cfg::kSfaBytes);
               tma_load_2d(sSfa + st * Cfg::kSfaBytes, &map_sfa, &full[st], ks * 256, m0 / 128);
             } else {
               mbar_arrive_expect_tx(&full[st], Cfg::kSfbBytes);
-              tma_load_2d(sSfb + st * Cfg::kSfbBytes, &map_sfb, &full[st], ks * 256, n0 / 128);
+              tma_load_2d(sSfb + st * Cfg::kSfbBytes, &map_sfb, &full[st], ks * 256, nb0 / 128);
             }
             if (++st == Cfg::kStages) {
               st = 0;
@@ -256,9 +271,9 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
         const int ab = i % Cfg::kAccBufs;
         const int use = i / Cfg::kAccBufs;
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(ab * Cfg::kAccCols);
-        if (res && tile / p.tiles_m != n_prev) {
+        if (res && tile / tiles_m != n_prev) {
           // a new column block: its B scales, all of K, into tensor memory
-          n_prev = tile / p.tiles_m;
+          n_prev = tile / tiles_m;
           if (!mbar_wait(res_full, static_cast<uint32_t>(res_uses) & 1u, p.status)) break;
           tc_fence_after();
           const uint64_t r_d = smem_desc(smem_u32(sRes), 0, 128, kLayoutSwizzleNone);
@@ -337,19 +352,25 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
     const int h = ew / 4;                      // which 128-column half (BN = 256)
     const int r = 32 * q + lane;               // row of the tile
     const bool leader = (ew == 0 && lane == 0);
-    const float alpha = __ldg(p.gdec_a) * __ldg(p.gdec_b);
+    float alpha = __ldg(p.gdec_a) * __ldg(p.gdec_b);
     for (int i = 0; i < run.count; ++i) {
       const int tile = run.first + i;
       const int ab = i % Cfg::kAccBufs;
-      const int64_t m0 = static_cast<int64_t>(tile % p.tiles_m) * Cfg::kBM;
-      const int64_t n0 = static_cast<int64_t>(tile / p.tiles_m) * Cfg::kBN;
+      const int64_t m0 = static_cast<int64_t>(tile % tiles_m) * Cfg::kBM;
+      const int64_t n0 = static_cast<int64_t>(tile / tiles_m) * Cfg::kBN;
+      const float* bias = p.bias;
+      if (grouped) {
+        const int e = expert_of(static_cast<int32_t>(m0));
+        alpha = __ldg(p.gdec_a + e) * __ldg(p.gdec_b + e);
+        if (bias != nullptr) bias += static_cast<int64_t>(e) * p.N;
+      }
       // lane l holds the bias of column 32 cc + l of each of its chunks, fetched
       // before the accumulator is ready so the load hides behind the mainloop
       float bias_l[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int64_t col = n0 + 32 * (4 * h + c) + lane;
-        bias_l[c] = (p.bias != nullptr && col < p.N) ? __ldg(p.bias + col) : 0.0f;
+        bias_l[c] = (bias != nullptr && col < p.N) ? __ldg(bias + col) : 0.0f;
       }
       // rank-one epilogue: this thread's row factor (the bias row becomes the column factor)
       float u_r = 1.0f;
@@ -452,7 +473,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
   }
 }
 
-template <int BN, bool kBf16Out, bool kRank1>
+template <int BN, bool kBf16Out, bool kRank1, bool kGrouped>
 static cudaError_t launch_gemm_t(const GemmArgs& a, cudaStream_t s, bool pdl) {
   using Cfg = GemmCfg<BN, kBf16Out>;
   constexpr CUtensorMapSwizzle kOpSwizzle = CU_TENSOR_MAP_SWIZZLE_128B;
@@ -460,7 +481,8 @@ static cudaError_t launch_gemm_t(const GemmArgs& a, cudaStream_t s, bool pdl) {
   if (!make_tensor_map_2d(&ma, a.a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(a.M),
                           static_cast<uint64_t>(a.K / 2), Cfg::kBM, Cfg::kRowBytes, kOpSwizzle))
     return cudaErrorInvalidValue;
-  if (!make_tensor_map_2d(&mb, a.b_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(a.N),
+  const uint64_t b_rows = static_cast<uint64_t>(a.N) * static_cast<uint64_t>(a.groups);   // experts stacked
+  if (!make_tensor_map_2d(&mb, a.b_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, b_rows,
                           static_cast<uint64_t>(a.K / 2), Cfg::kBN, Cfg::kRowBytes, kOpSwizzle))
     return cudaErrorInvalidValue;
   // scale atoms as a [row groups, K/64 * 64] array of 8-byte elements; a box of
@@ -469,7 +491,7 @@ static cudaError_t launch_gemm_t(const GemmArgs& a, cudaStream_t s, bool pdl) {
   if (!make_tensor_map_2d(&msa, a.a_scales, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, static_cast<uint64_t>((a.M + 127) / 128),
                           sf_cols, 1, 256, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
-  if (!make_tensor_map_2d(&msb, a.b_scales, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, static_cast<uint64_t>((a.N + 127) / 128),
+  if (!make_tensor_map_2d(&msb, a.b_scales, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, (b_rows + 127) / 128,
                           sf_cols, Cfg::kBN / 128, 256, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   if (!make_tensor_map_2d(&my, a.Y, kBf16Out ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
@@ -480,16 +502,18 @@ static cudaError_t launch_gemm_t(const GemmArgs& a, cudaStream_t s, bool pdl) {
   p.M = a.M;
   p.N = a.N;
   p.K = a.K;
+  p.block_expert = a.block_expert;
+  p.totals = a.totals;
   p.tiles_m = static_cast<int>((a.M + Cfg::kBM - 1) / Cfg::kBM);
   p.num_tiles = p.tiles_m * static_cast<int>((a.N + Cfg::kBN - 1) / Cfg::kBN);
   const int64_t n_kst = (a.K + Cfg::kStageK - 1) / Cfg::kStageK;
-  p.sfb_resident = (Cfg::kResMaxStages > 0 && n_kst <= Cfg::kResMaxStages) ? 1 : 0;
+  p.sfb_resident = (Cfg::kResMaxStages > 0 && n_kst <= Cfg::kResMaxStages && a.block_expert == nullptr) ? 1 : 0;
   p.gdec_a = a.a_gdec;
   p.gdec_b = a.b_gdec;
   p.bias = a.bias;
   p.row_scale = a.row_scale;
   p.status = a.status;
-  auto kern = gemm_nvfp4_kernel<BN, kBf16Out, kRank1>;
+  auto kern = gemm_nvfp4_kernel<BN, kBf16Out, kRank1, kGrouped>;
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kern), Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
@@ -498,10 +522,15 @@ static cudaError_t launch_gemm_t(const GemmArgs& a, cudaStream_t s, bool pdl) {
 
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, bool pdl) {
   if (a.row_scale != nullptr) {
-    if (a.bias == nullptr) return cudaErrorInvalidValue;
-    return a.yt == AVR_BF16 ? launch_gemm_t<256, true, true>(a, s, pdl) : launch_gemm_t<128, false, true>(a, s, pdl);
+    if (a.bias == nullptr || a.block_expert != nullptr) return cudaErrorInvalidValue;
+    return a.yt == AVR_BF16 ? launch_gemm_t<256, true, true, false>(a, s, pdl)
+                            : launch_gemm_t<128, false, true, false>(a, s, pdl);
   }
-  return a.yt == AVR_BF16 ? launch_gemm_t<256, true, false>(a, s, pdl) : launch_gemm_t<128, false, false>(a, s, pdl);
+  if (a.block_expert != nullptr)
+    return a.yt == AVR_BF16 ? launch_gemm_t<256, true, false, true>(a, s, pdl)
+                            : launch_gemm_t<128, false, false, true>(a, s, pdl);
+  return a.yt == AVR_BF16 ? launch_gemm_t<256, true, false, false>(a, s, pdl)
+                          : launch_gemm_t<128, false, false, false>(a, s, pdl);
 }
 
 }  // namespace avr

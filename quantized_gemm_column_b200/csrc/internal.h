@@ -51,15 +51,28 @@ WgLayout wgrad_layout(int64_t l, int64_t m, int64_t n);
 size_t scales_bytes(int64_t rows, int64_t K);
 
 // ---------------- K1: fixed-order column reduce ----------------
+// One expert's segment of a token buffer permuted by expert (MoE): rows
+// [row0, row0 + rows) of the buffer, its chunks of 256 rows numbered
+// chunk0 .. chunk0 + chunks - 1 among all experts' chunks.
+struct MoeSeg {
+  int32_t row0, rows, chunk0, chunks;
+};
+
 struct ColReduceArgs {
   const void* X;
   avr_dtype xt;
   int64_t l, K;
   int split;              // 1: mean + residual amax; 0: amax of X only (vanilla)
-  float* mu_out;          // [K], written when split (nullable otherwise)
+  float* mu_out;          // [K] ([E][K] grouped), written when split (nullable otherwise)
   int energy;             // 1: also the column sums of squares (the R monitor)
   char* ws;               // workspace base
   const WsLayout* lay;
+  // grouped (MoE) mode, null for a dense matrix: per-expert segments, the
+  // expert of every chunk, the number of chunks in use; c_max chunks launched
+  const MoeSeg* seg = nullptr;
+  const int32_t* chunk_expert = nullptr;
+  const int32_t* totals = nullptr;
+  int c_max = 0;
 };
 cudaError_t launch_colreduce(const ColReduceArgs& a, cudaStream_t s, bool pdl);
 
@@ -110,6 +123,51 @@ cudaError_t launch_split_fused(const ColReduceArgs& ca, const QuantArgs& qa, cud
 // 64, zero padding.  xr_debug and the rank-one row (w_*) are not used.
 cudaError_t launch_quant_tokens(const QuantArgs& a, cudaStream_t s, bool pdl);
 
+// ---------------- mixture of experts (moe.cu) ----------------
+// segment table from the per-expert token counts (device), see moe.cu
+cudaError_t launch_moe_table(const int32_t* counts, int E, int64_t l_cap, int c_max, MoeSeg* seg,
+                             int32_t* chunk_expert, int32_t* block_expert, int32_t* totals, uint32_t* status,
+                             cudaStream_t s, bool pdl);
+
+struct MoeQuantArgs {
+  const void* X;
+  avr_dtype xt;
+  int64_t l_cap, K;
+  int E;
+  const MoeSeg* seg;
+  const int32_t* block_expert;
+  const int32_t* totals;
+  const float* mu;              // [E][K] (null: vanilla)
+  const float* slot_xr;         // [E][T] (T = K / 128 rounded up)
+  const float* slot_mu;
+  uint8_t* codes;               // [l_cap][K/2]
+  uint8_t* scales;
+  float* g_dec;                 // [E]
+  uint8_t* mu_codes;            // [E][K/2] (null: no mean quantization)
+  uint8_t* mu_scales;
+  float* mu_gdec;               // [E]
+  uint64_t seed, offset;
+  uint32_t tag, tag_mu;
+  int sr;
+  uint32_t* status;
+};
+cudaError_t launch_moe_quant(const MoeQuantArgs& a, cudaStream_t s, bool pdl);
+
+struct MoeBiasArgs {
+  const MoeSeg* seg;
+  const int32_t* totals;
+  int E;
+  int64_t K, N;                 // mean length; output features per expert
+  const uint8_t* mu_codes;      // [E][K/2] with scales and mu_gdec [E]
+  const uint8_t* mu_scales;
+  const float* mu_gdec;
+  const uint8_t* w_codes;       // [E * N][K/2], experts stacked
+  const uint8_t* w_scales;
+  const float* w_gdec;          // [E]
+  float* bias;                  // [E][N]
+};
+cudaError_t launch_moe_bias(const MoeBiasArgs& a, cudaStream_t s, bool pdl);
+
 // u = l * deq(mu_bar_X) [m], v = deq(mu_bar_D) [n]
 cudaError_t launch_mean_dequant(const uint8_t* codes_x, const uint8_t* scales_x, const float* gdec_x, int64_t m,
                                 const uint8_t* codes_d, const uint8_t* scales_d, const float* gdec_d, int64_t n,
@@ -152,6 +210,12 @@ struct GemmArgs {
   int64_t M, N, K;
   const float* bias;   // nullable
   const float* row_scale = nullptr;   // nullable: Y = alpha acc + row_scale[i] * bias[j] (rank-one term)
+  // grouped (MoE): B holds `groups` experts' [N, K] matrices stacked; a_gdec,
+  // b_gdec and bias are per expert; A's 128-row blocks map to experts through
+  // block_expert, and totals[1] rows are in use (null: one GEMM)
+  int64_t groups = 1;
+  const int32_t* block_expert = nullptr;
+  const int32_t* totals = nullptr;
   void* Y;
   avr_dtype yt;
   uint32_t* status;

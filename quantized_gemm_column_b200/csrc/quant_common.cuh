@@ -253,11 +253,9 @@ static __device__ void bias_window(const uint16_t* s_mu16, float* s_part, int64_
   }
 }
 
-// 16 floats of a 64-byte aligned row (plain loads: cached in L1, so the
-// warps of an SM that read the same columns share one L2 request).
-// 16 fp32 values; kL2: through L2 only, for data other CTAs of the same grid
-// wrote (L1 does not see their stores).  The plain form lets the warps of an
-// SM that read the same mean share L1 lines.
+// 16 fp32 values of a 64-byte aligned row; kL2: through L2 only, for data
+// other CTAs of the same grid wrote (L1 does not see their stores).  The
+// plain form lets the warps of an SM that read the same mean share L1 lines.
 template <bool kL2 = false>
 __device__ __forceinline__ void load_f32x16(const float* p, float (&v)[16]) {
   const float4* q = reinterpret_cast<const float4*>(p);

@@ -142,3 +142,38 @@ def workload3(c, l=16384, m=2048, n=2048, seed_tag=0):
                            mean_scale=c)
     W = weight(rng_for(3, 2 + seed_tag), m, n)
     return to_bf16(X), to_bf16(W)
+
+
+def moe_counts(E, tokens, top_k, seed=0, alpha=1.0):
+    """Tokens routed to each of E experts when every token picks top_k
+    distinct experts, drawn with expert popularities p ~ Dirichlet(alpha): a
+    skewed load like a trained router's.  Returns a list of E ints summing to
+    tokens * top_k."""
+    rng = rng_for(4, 100 + seed)
+    p = rng.dirichlet(np.full(E, alpha))
+    counts = np.zeros(E, dtype=np.int64)
+    for _ in range(tokens):
+        counts[rng.choice(E, top_k, replace=False, p=p)] += 1
+    return [int(c) for c in counts]
+
+
+def workload_moe(E=64, tokens=4096, top_k=8, m=2048, n=1024, seed_tag=0):
+    """A mixture-of-experts linear: the permuted activation buffer [l_cap, m]
+    (expert e's tokens carry their own planted mean, spike and noise; rows of
+    the 128-row padding are zero), the per-expert counts, the expert weights
+    [E, m, n] and an output gradient in the same segments."""
+    counts = moe_counts(E, tokens, top_k, seed_tag)
+    rng = rng_for(5, 1 + seed_tag)
+    offs, l_cap = [], 0
+    for c in counts:
+        offs.append(l_cap)
+        l_cap += (c + 127) // 128 * 128
+    X = np.zeros((l_cap, m))
+    D = np.zeros((l_cap, n))
+    for e, (o, c) in enumerate(zip(offs, counts)):
+        if c:
+            X[o:o + c] = spiked_activations(rng, c, m, rank=2, s=(8.0, 4.0), n_hot=m // 100,
+                                            mean_scale=1.0 + (e % 4) / 2)
+            D[o:o + c] = output_gradient(rng, c, n)
+    W = np.stack([weight(rng, m, n) for _ in range(E)])
+    return counts, to_bf16(X), to_bf16(W), to_bf16(D)
