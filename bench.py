@@ -135,6 +135,37 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# the MoE variant (beyond the timed step)
+# ---------------------------------------------------------------------------
+def moe_timing(dev, stream, avg_us):
+    """Forward and dgrad of one MoE linear: 64 experts, 4096 tokens routed to 8
+    experts each (skewed counts), hidden 2048 -> 1024 per expert; the permuted
+    buffer (151 MB) is larger than L2."""
+    import torch
+    from quantized_gemm_column_b200 import api, inputs
+    counts, Xm, Wm, Dm = inputs.workload_moe()
+    E, m, n = Wm.shape
+    l_cap = Xm.shape[0]
+    cnt = torch.tensor(counts, dtype=torch.int32, device=dev)
+    w_fwd, w_dgrad = api.NVFP4Group(E * n, m, E, dev), api.NVFP4Group(E * m, n, E, dev)
+    wq_ws = api.workspace(m, n, n, dev)
+    api.averis_moe_quant_weights(Wm.to(dev), w_fwd, w_dgrad, wq_ws, stream)
+    mws = api.moe_workspace(l_cap, max(m, n), max(m, n), E, dev)
+    Xd, Dd = Xm.to(dev), Dm.to(dev)
+    Y = torch.empty((l_cap, n), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((l_cap, m), dtype=torch.bfloat16, device=dev)
+    fwd = avg_us(lambda i: api.averis_moe_linear_fwd(Xd, cnt, w_fwd, "sr", 1 + i, 0, Y, mws, stream))
+    dgr = avg_us(lambda i: api.averis_moe_linear_dgrad(Dd, cnt, w_dgrad, "sr", 1 + i, 0, dX, mws, stream))
+    if api.averis_check_status(mws, stream) or api.averis_check_status(wq_ws, stream):
+        raise RuntimeError("device status set by the MoE timing")
+    tokens = sum(counts)
+    flops = 2.0 * tokens * m * n
+    return {"experts": E, "tokens_routed": tokens, "rows_padded": l_cap, "m": m, "n": n,
+            "fwd_us": fwd, "dgrad_us": dgr, "tflops": 2 * flops / ((fwd + dgr) * 1e-6) / 1e12,
+            "launches_per_pass": 5}
+
+
+# ---------------------------------------------------------------------------
 # CPU oracle baseline
 # ---------------------------------------------------------------------------
 def oracle_step(x, d, w_fwd_q, w_dgrad_q):
@@ -409,6 +440,8 @@ def run_gpu(args, rank, world, local_rank):
              "split_quant_t_us": {"X": sqt_x, "dY": sqt_d}, "gemm_us": g_w,
              "gemm_tflops": 2 * L * M * N / (g_w * 1e-6) / 1e12}
 
+    moe = moe_timing(dev, stream, avg_us)
+
     # split-quant algorithmic bytes: read the input twice (reduce, quantize),
     # write codes (1/2 byte per element) and scales (1/16 byte per element)
     def sq_bytes(rows, K):
@@ -492,6 +525,7 @@ def run_gpu(args, rank, world, local_rank):
         "split_quant_fused_us": {"X": fs_x, "dY": fs_d},
         "gemm_us": {"fwd": g_f, "dgrad": g_d}, "gemm_tflops": gemm_tflops,
         "wgrad": wgrad,
+        "moe": moe,
         "gemm_frac_fp4_peak": gemm_tflops / fp4_peak,
         "vanilla_ms_per_step": ms_van / args.steps,
         "averis_overhead_vs_vanilla": (ms / ms_van) - 1.0,

@@ -174,13 +174,18 @@ __global__ void __launch_bounds__(kQuantThreads) moe_quant_kernel(const MoeQuant
 
   // tasks: (512-column strip, 32-row group) with every row of the group in
   // one expert's segment (or past all of them)
+  // each warp takes a contiguous range of tasks, so that consecutive tasks
+  // mostly share the expert (and its tensor scale and reciprocal table)
   const int n_ctas = static_cast<int>(gridDim.x) - p.n_aux;
   const int64_t n_groups = p.l_cap / kGroupRows;
   const int64_t n_tasks = n_groups * p.n_strips;
+  const int64_t n_warps = static_cast<int64_t>(n_ctas) * kQuantWarps;
   const int64_t gw0 = static_cast<int64_t>(static_cast<int>(blockIdx.x) - p.n_aux) * kQuantWarps + warp;
+  const int64_t t_per = (n_tasks + n_warps - 1) / n_warps;
+  const int64_t t_end = min64(n_tasks, (gw0 + 1) * t_per);
   int cached_e = -1;
   TensorScale ts = {1.0f, 1.0f};
-  for (int64_t task = gw0; task < n_tasks; task += static_cast<int64_t>(n_ctas) * kQuantWarps) {
+  for (int64_t task = gw0 * t_per; task < t_end; ++task) {
     const int strip = static_cast<int>(task % p.n_strips);
     const int64_t r_first = (task / p.n_strips) * kGroupRows;
     const int e = __ldg(p.block_expert + r_first / 128);
@@ -203,31 +208,44 @@ __global__ void __launch_bounds__(kQuantThreads) moe_quant_kernel(const MoeQuant
     if (strip == 0 && r_first == sg.row0 && lane == 0) p.g_dec[e] = ts.g_dec;
     const int64_t r_end = static_cast<int64_t>(sg.row0) + sg.rows;   // rows past it are padding
     const uint32_t c16 = static_cast<uint32_t>(col0 / 16);
-    Raw16<kBf16> cur;
-    load16<kBf16>(p.X, r_first * p.K + col0, active && r_first < r_end, cur);
-#pragma unroll 1
-    for (int i = 0; i < kGroupRows; ++i) {
-      const int64_t r = r_first + i;
-      Raw16<kBf16> nxt;
-      if (i + 1 < kGroupRows) load16<kBf16>(p.X, (r + 1) * p.K + col0, active && r + 1 < r_end, nxt);
-      const bool real = r < r_end;
-      float xr[16];
-      sub_mu16<kBf16>(cur, mu, xr);
-      if (!real) {
+    // rows kRowsInFlight at a time, the next ones loading meanwhile (the
+    // buffer is usually read from HBM: it does not fit in L2 with the reduce's pass)
+    constexpr int kRowsInFlight = 2;
+    Raw16<kBf16> cur[kRowsInFlight], nxt[kRowsInFlight];
 #pragma unroll
-        for (int q = 0; q < 16; ++q) xr[q] = 0.0f;     // padding rows: zero codes and scales
+    for (int q = 0; q < kRowsInFlight; ++q)
+      load16<kBf16>(p.X, (r_first + q) * p.K + col0, active && r_first + q < r_end, cur[q]);
+#pragma unroll 1
+    for (int i = 0; i < kGroupRows; i += kRowsInFlight) {
+      if (i + kRowsInFlight < kGroupRows) {
+#pragma unroll
+        for (int q = 0; q < kRowsInFlight; ++q) {
+          const int64_t rn = r_first + i + kRowsInFlight + q;
+          load16<kBf16>(p.X, rn * p.K + col0, active && rn < r_end, nxt[q]);
+        }
       }
-      const uint4 rw = kSR ? philox_keyed(p.offset + static_cast<uint64_t>((r * p.K + col0) / 16), p.tag, keys)
-                           : make_uint4(0u, 0u, 0u, 0u);
-      uint32_t S;
-      const uint2 packed = quant16<kSR>(xr, ts.g_enc, r_tab, rw, &S);
-      const uint32_t sw = gather_scale_word(S);
-      if (active) {
-        *reinterpret_cast<uint2*>(p.codes + r * (p.K / 2) + col0 / 2) = packed;
-        if ((lane & 3) == 0)
-          *reinterpret_cast<uint32_t*>(p.scales + scale_offset(static_cast<uint64_t>(r), c16, n_kb64)) = sw;
+#pragma unroll
+      for (int q = 0; q < kRowsInFlight; ++q) {
+        const int64_t r = r_first + i + q;
+        float xr[16];
+        sub_mu16<kBf16>(cur[q], mu, xr);
+        if (r >= r_end) {
+#pragma unroll
+          for (int t = 0; t < 16; ++t) xr[t] = 0.0f;   // padding rows: zero codes and scales
+        }
+        const uint4 rw = kSR ? philox_keyed(p.offset + static_cast<uint64_t>((r * p.K + col0) / 16), p.tag, keys)
+                             : make_uint4(0u, 0u, 0u, 0u);
+        uint32_t S;
+        const uint2 packed = quant16<kSR>(xr, ts.g_enc, r_tab, rw, &S);
+        const uint32_t sw = gather_scale_word(S);
+        if (active) {
+          *reinterpret_cast<uint2*>(p.codes + r * (p.K / 2) + col0 / 2) = packed;
+          if ((lane & 3) == 0)
+            *reinterpret_cast<uint32_t*>(p.scales + scale_offset(static_cast<uint64_t>(r), c16, n_kb64)) = sw;
+        }
       }
-      if (i + 1 < kGroupRows) cur = nxt;
+#pragma unroll
+      for (int q = 0; q < kRowsInFlight; ++q) cur[q] = nxt[q];
     }
   }
 }
@@ -281,22 +299,34 @@ cudaError_t launch_moe_quant(const MoeQuantArgs& a, cudaStream_t s, bool pdl) {
 }
 
 // ---------------------------------------------------------------------------
-// rank-one rows b_e = mu_bar_e W_bar_e, one CTA per (32-row group, expert)
+// rank-one rows b_e = mu_bar_e W_bar_e: a warp per output row, so the 32 lanes
+// read the row's codes with coalesced 16-byte loads (32 elements per lane per
+// step); products of E2M1 x (E2M1 x E4M3) values are exact in f16 and summed
+// in fp32 per 16-element block, scaled by the block's E4M3 scale, then the
+// lanes' partial sums are added by a shuffle tree.  CTA (x, e) takes rows
+// 64 x .. 64 x + 63 of expert e.
 // ---------------------------------------------------------------------------
+constexpr int kBiasRowsPerCta = 64;
+
 __global__ void __launch_bounds__(kQuantThreads) moe_bias_kernel(const MoeBiasArgs a) {
-  extern __shared__ uint16_t s_mu16[];
-  __shared__ float s_part[kQuantWarps * kRowGroup];
+  extern __shared__ uint16_t s_mu16[];         // mu_bar_e as f16, one window of K
   pdl_wait_prior_grid();
   pdl_allow_next_grid();
   const int e = static_cast<int>(blockIdx.y);
   if (__ldcg(a.totals + 2) == 0) return;       // the segments did not fit
   if (a.seg[e].rows == 0) return;             // no tokens: the GEMM has no tile of this expert
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t n_kb64 = static_cast<uint32_t>(a.K / 64);
   const float gprod = __ldcg(a.mu_gdec + e) * __ldg(a.w_gdec + e);
   const uint8_t* w_codes = a.w_codes + static_cast<int64_t>(e) * a.N * (a.K / 2);
   const uint8_t* w_scales = a.w_scales + static_cast<int64_t>(e) * a.N * (a.K / 16);
+  const int64_t j0 = static_cast<int64_t>(blockIdx.x) * kBiasRowsPerCta;
+  float acc[kBiasRowsPerCta / kQuantWarps];
+#pragma unroll
+  for (int r = 0; r < kBiasRowsPerCta / kQuantWarps; ++r) acc[r] = 0.0f;
   for (int64_t k_lo = 0; k_lo < a.K; k_lo += kBiasWindow) {
     const int64_t k_hi = min64(a.K, k_lo + kBiasWindow);
+    __syncthreads();                            // the previous window is no longer read
     for (int64_t k = k_lo + threadIdx.x; k < k_hi; k += kQuantThreads) {
       const uint32_t byte = a.mu_codes[static_cast<int64_t>(e) * (a.K / 2) + k / 2];
       const uint32_t code = (k & 1) ? (byte >> 4) : (byte & 0xFu);
@@ -305,15 +335,63 @@ __global__ void __launch_bounds__(kQuantThreads) moe_bias_kernel(const MoeBiasAr
       s_mu16[k - k_lo] = __half_as_ushort(__float2half_rn(v));
     }
     __syncthreads();
-    bias_window(s_mu16, s_part, k_lo, k_hi, a.K, w_codes, w_scales, gprod, a.N, static_cast<int>(blockIdx.x),
-                static_cast<int>(gridDim.x), a.bias + static_cast<int64_t>(e) * a.N);
-    __syncthreads();
+    // per 1024-column step: the codes and scales of all this warp's rows are
+    // requested before any product, so a warp keeps 8 row loads in flight
+    for (int64_t ks = k_lo; ks < k_hi; ks += 32 * 32) {
+      const int64_t k = ks + lane * 32;
+      const bool kv = k < k_hi;
+      uint4 c[kBiasRowsPerCta / kQuantWarps];
+      uint32_t sc[kBiasRowsPerCta / kQuantWarps];
+#pragma unroll
+      for (int r = 0; r < kBiasRowsPerCta / kQuantWarps; ++r) {
+        const int64_t j = j0 + r * kQuantWarps + warp;
+        c[r] = make_uint4(0u, 0u, 0u, 0u);
+        sc[r] = 0u;
+        if (kv && j < a.N) {
+          c[r] = __ldg(reinterpret_cast<const uint4*>(w_codes + j * (a.K / 2) + k / 2));   // 32 codes
+          sc[r] = __ldg(reinterpret_cast<const uint16_t*>(
+              w_scales + scale_offset(static_cast<uint64_t>(j), static_cast<uint32_t>(k / 16), n_kb64)));
+        }
+      }
+      if (!kv) continue;
+      uint32_t mv[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 m = *reinterpret_cast<const uint4*>(s_mu16 + (k - k_lo) + 8 * q);
+        mv[4 * q] = m.x;
+        mv[4 * q + 1] = m.y;
+        mv[4 * q + 2] = m.z;
+        mv[4 * q + 3] = m.w;
+      }
+#pragma unroll
+      for (int r = 0; r < kBiasRowsPerCta / kQuantWarps; ++r) {
+        const uint32_t words[4] = {c[r].x, c[r].y, c[r].z, c[r].w};
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {           // two 16-element blocks
+          float part = 0.0f;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t byte = (words[2 * b + q / 4] >> (8 * (q % 4))) & 0xFFu;
+            part = fma2_f16_f32(e2m1x2_to_f16x2(byte), mv[8 * b + q], part);
+          }
+          acc[r] = fmaf(part, e4m3_value((sc[r] >> (8 * b)) & 0xFFu), acc[r]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < kBiasRowsPerCta / kQuantWarps; ++r) {
+    float v = acc[r];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    const int64_t j = j0 + r * kQuantWarps + warp;
+    if (lane == 0 && j < a.N) a.bias[static_cast<int64_t>(e) * a.N + j] = v * gprod;
   }
 }
 
 cudaError_t launch_moe_bias(const MoeBiasArgs& a, cudaStream_t s, bool pdl) {
   const size_t smem = static_cast<size_t>(min64(a.K, kBiasWindow)) * sizeof(uint16_t);
-  const dim3 grid(static_cast<unsigned>((a.N + kRowGroup - 1) / kRowGroup), static_cast<unsigned>(a.E));
+  const dim3 grid(static_cast<unsigned>((a.N + kBiasRowsPerCta - 1) / kBiasRowsPerCta), static_cast<unsigned>(a.E));
   return launch_ex(moe_bias_kernel, grid, dim3(kQuantThreads), smem, s, pdl, a);
 }
 
