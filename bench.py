@@ -46,7 +46,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="averis", choices=["averis", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--cpu-sample-rows", type=int, default=1024)
+    p.add_argument("--cpu-sample-rows", type=int, default=4096)
+    p.add_argument("--cpu-sample-steps", type=int, default=2)
     p.add_argument("--copies", type=int, default=4, help="input copies rotated between steps")
     return p.parse_args()
 
@@ -135,6 +136,86 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# the 28-layer Qwen3-0.6B linear stack (beyond the timed step)
+# ---------------------------------------------------------------------------
+STACK_SHAPES = (("qkv", 1024, 4096), ("o_proj", 2048, 1024), ("gate_up", 1024, 6144), ("down", 3072, 1024))
+
+
+def stack_timing(dev, stream, layers=28, tokens=32768, steps=2):
+    """Forward + dgrad through the 4 linears of each of `layers` layers at
+    `tokens` tokens, Averis and vanilla NVFP4, CUDA-graph replay of one layer.
+    Inputs are drawn on the device (seeded): activations = per-column mean
+    N(0, 0.5) with 1% of channels x20 + N(0, 1) (the down projection's input:
+    silu(a) b with a, b ~ N(0.2, 1)); output gradients 1e-3 (N(0, 1) + per-column
+    N(0, 0.3)); weights N(0, 1/sqrt(m)), one per shape for all layers."""
+    import torch
+    from quantized_gemm_column_b200 import api
+    g = torch.Generator(device=dev)
+    g.manual_seed(20)
+    bufs = []
+    for name, m, n in STACK_SHAPES:
+        if name == "down":
+            a = torch.randn(tokens, m, generator=g, device=dev) + 0.2
+            b = torch.randn(tokens, m, generator=g, device=dev) + 0.2
+            X = (torch.nn.functional.silu(a) * b).to(torch.bfloat16)
+            del a, b
+        else:
+            mu = torch.randn(m, generator=g, device=dev) * 0.5
+            hot = torch.randperm(m, generator=g, device=dev)[: m // 100]
+            mu[hot] *= 20.0
+            X = (torch.randn(tokens, m, generator=g, device=dev) + mu).to(torch.bfloat16)
+        D = ((torch.randn(tokens, n, generator=g, device=dev) + torch.randn(n, generator=g, device=dev) * 0.3)
+             * 1e-3).to(torch.bfloat16)
+        W = (torch.randn(m, n, generator=g, device=dev) / m ** 0.5).to(torch.bfloat16)
+        w_fwd, w_dgrad = api.NVFP4Tensor(n, m, dev), api.NVFP4Tensor(m, n, dev)
+        ws = api.workspace(tokens, max(m, n), max(m, n), dev)
+        torch.cuda.synchronize(dev)            # drawn on the default stream, consumed on `stream`
+        api.averis_quant_weight(W, w_fwd, w_dgrad, ws, stream)
+        Y = torch.empty((tokens, n), dtype=torch.bfloat16, device=dev)
+        dX = torch.empty((tokens, m), dtype=torch.bfloat16, device=dev)
+        bufs.append((X, D, w_fwd, w_dgrad, ws, Y, dX))
+
+    def layer(vanilla):
+        for X, D, w_fwd, w_dgrad, ws, Y, dX in bufs:
+            if vanilla:
+                api.nvfp4_linear_fwd(X, w_fwd, "sr", 1, 0, Y, ws, stream=stream)
+                api.nvfp4_linear_dgrad(D, w_dgrad, "sr", 2, 0, dX, ws, stream=stream)
+            else:
+                api.averis_linear_fwd(X, w_fwd, "sr", 1, 0, Y, ws, stream=stream)
+                api.averis_linear_dgrad(D, w_dgrad, "sr", 2, 0, dX, ws, stream=stream)
+
+    torch.cuda.synchronize(dev)
+    out = {}
+    for vanilla in (False, True):
+        with torch.cuda.stream(stream):
+            layer(vanilla)
+            torch.cuda.synchronize(dev)
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                layer(vanilla)
+            for _ in range(layers):
+                gr.replay()
+            torch.cuda.synchronize(dev)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(steps * layers):
+                gr.replay()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+        out["vanilla_ms" if vanilla else "averis_ms"] = a.elapsed_time(b) / steps
+        del gr
+    for _, _, _, _, ws, _, _ in bufs:
+        if api.averis_check_status(ws, stream):
+            raise RuntimeError("device status set by the stack timing")
+    flops = sum(2.0 * tokens * m * n * 2 for _, m, n in STACK_SHAPES) * layers
+    return {"layers": layers, "tokens": tokens, "shapes": {s[0]: [s[1], s[2]] for s in STACK_SHAPES},
+            "averis_ms_per_step": out["averis_ms"], "vanilla_ms_per_step": out["vanilla_ms"],
+            "averis_overhead_vs_vanilla": out["averis_ms"] / out["vanilla_ms"] - 1.0,
+            "tflops": flops / (out["averis_ms"] * 1e-3) / 1e12,
+            "data": "synthetic, drawn on the device (seeded)"}
+
+
+# ---------------------------------------------------------------------------
 # the MoE variant (beyond the timed step)
 # ---------------------------------------------------------------------------
 def moe_timing(dev, stream, avg_us):
@@ -149,15 +230,17 @@ def moe_timing(dev, stream, avg_us):
     cnt = torch.tensor(counts, dtype=torch.int32, device=dev)
     w_fwd, w_dgrad = api.NVFP4Group(E * n, m, E, dev), api.NVFP4Group(E * m, n, E, dev)
     wq_ws = api.workspace(m, n, n, dev)
-    api.averis_moe_quant_weights(Wm.to(dev), w_fwd, w_dgrad, wq_ws, stream)
+    Wd, Xd, Dd = Wm.to(dev), Xm.to(dev), Dm.to(dev)
+    torch.cuda.synchronize(dev)                # copied on the default stream, consumed on `stream`
+    api.averis_moe_quant_weights(Wd, w_fwd, w_dgrad, wq_ws, stream)
     mws = api.moe_workspace(l_cap, max(m, n), max(m, n), E, dev)
-    Xd, Dd = Xm.to(dev), Dm.to(dev)
     Y = torch.empty((l_cap, n), dtype=torch.bfloat16, device=dev)
     dX = torch.empty((l_cap, m), dtype=torch.bfloat16, device=dev)
     fwd = avg_us(lambda i: api.averis_moe_linear_fwd(Xd, cnt, w_fwd, "sr", 1 + i, 0, Y, mws, stream))
     dgr = avg_us(lambda i: api.averis_moe_linear_dgrad(Dd, cnt, w_dgrad, "sr", 1 + i, 0, dX, mws, stream))
     if api.averis_check_status(mws, stream) or api.averis_check_status(wq_ws, stream):
         raise RuntimeError("device status set by the MoE timing")
+    del Wd
     tokens = sum(counts)
     flops = 2.0 * tokens * m * n
     return {"experts": E, "tokens_routed": tokens, "rows_padded": l_cap, "m": m, "n": n,
@@ -203,7 +286,11 @@ def cpu_baseline(rows, steps=1):
     flops = 2 * (2 * rows * M * N)
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"first {rows} of {L} tokens of X and dY (column mean, split, NVFP4 SR "
-                      f"quantization and fp64 product of the sample), {dt:.1f} s per fwd+dgrad"}
+                      f"quantization and fp64 product of the sample), {steps} fwd+dgrad passes of "
+                      f"{dt:.1f} s each"}
+
+
+REF_WARMUP_S, REF_TIMED_S = 20.0, 120.0
 
 
 def run_reference(args, rank, world):
@@ -211,21 +298,31 @@ def run_reference(args, rank, world):
         return
     rows = 128
     x, d, wf, wd = oracle_operands(rows)
-    for _ in range(args.warmup):
-        oracle_step(x, d, wf, wd)
+    # the oracle takes ~0.4 s a step (it decodes the weight every call): warm-up and timed steps
+    # stop at a wall-clock budget so that a run with the GPU arm's step count still ends in minutes
     t0 = time.perf_counter()
-    for _ in range(args.steps):
+    warm = 0
+    while warm < args.warmup and (warm == 0 or time.perf_counter() - t0 < REF_WARMUP_S):
         oracle_step(x, d, wf, wd)
-    dt = (time.perf_counter() - t0) / args.steps
+        warm += 1
+    t0 = time.perf_counter()
+    timed = 0
+    while timed < args.steps and (timed == 0 or time.perf_counter() - t0 < REF_TIMED_S):
+        oracle_step(x, d, wf, wd)
+        timed += 1
+    dt = (time.perf_counter() - t0) / timed
     value = 2 * (2 * rows * M * N) / dt / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "steps": timed, "steps_requested": args.steps, "warmup": warm, "warmup_requested": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64 product of e2m1 x e4m3 operands",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample_rows": rows},
+        "config": {"workload": WORKLOAD, "l": L, "m": M, "n": N, "rounding": "philox-sr",
+                   "parallelism": "single host process (rank 0)", "sample_rows": rows},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-                         "sample": f"first {rows} of {L} tokens per step"},
+                         "sample": f"first {rows} of {L} tokens per step, {timed} timed steps "
+                                   f"(at most {REF_TIMED_S:.0f} s of steps)"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -307,6 +404,7 @@ def run_gpu(args, rank, world, local_rank):
     Y = torch.empty((L, N), dtype=torch.bfloat16, device=dev)
     dX = torch.empty((L, M), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.Stream(dev)
+    torch.cuda.synchronize(dev)                # staged on the default stream, consumed on `stream`
 
     def step(i, s=None):
         api.averis_linear_fwd(Xs[i % copies], w_fwd, "sr", 1 + i, 0, Y, ws, stream=s)
@@ -441,6 +539,7 @@ def run_gpu(args, rank, world, local_rank):
              "gemm_tflops": 2 * L * M * N / (g_w * 1e-6) / 1e12}
 
     moe = moe_timing(dev, stream, avg_us)
+    stack = stack_timing(dev, stream)
 
     # split-quant algorithmic bytes: read the input twice (reduce, quantize),
     # write codes (1/2 byte per element) and scales (1/16 byte per element)
@@ -533,7 +632,7 @@ def run_gpu(args, rank, world, local_rank):
         return
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        cpu = cpu_baseline(args.cpu_sample_rows)
+        cpu = cpu_baseline(args.cpu_sample_rows, args.cpu_sample_steps)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
@@ -550,6 +649,7 @@ def run_gpu(args, rank, world, local_rank):
         "gemm_us": {"fwd": g_f, "dgrad": g_d}, "gemm_tflops": gemm_tflops,
         "wgrad": wgrad,
         "moe": moe,
+        "stack": stack,
         "gemm_frac_fp4_peak": gemm_tflops / fp4_peak,
         "vanilla_ms_per_step": ms_van / args.steps,
         "averis_overhead_vs_vanilla": (ms / ms_van) - 1.0,
