@@ -328,9 +328,10 @@ avr_status averis_check_status(void* ws, avr_stream stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return AVR_ERR_CUDA;
   uint32_t st = 0;
   if (cudaMemcpy(&st, ws, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return AVR_ERR_CUDA;
-  // after an error the whole 256-byte status block (status word and the
-  // grid-barrier words of the fused split) starts again from zero
-  if (st != 0 && cudaMemset(ws, 0, 256) != cudaSuccess) return AVR_ERR_CUDA;
+  // after an error the 256-byte status block (status word and the grid-barrier
+  // words of the fused split) and the reduce's tickets, which a kernel that
+  // gave up may have left part-counted, start again from zero
+  if (st != 0 && cudaMemset(ws, 0, WsLayout{}.slots) != cudaSuccess) return AVR_ERR_CUDA;
   return static_cast<avr_status>(st);
 }
 

@@ -41,102 +41,83 @@ struct ColReduceParams {
   int T;                  // column tiles (slot and ticket stride per expert)
 };
 
-template <bool kBf16, bool kEnergy, bool kGrouped>
-__global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_constant__ CUtensorMap map,
-                                                             const ColReduceParams p) {
-  extern __shared__ __align__(1024) uint8_t tile[];
-  __shared__ uint64_t bar;
-  __shared__ uint32_t s_last, s_ok;
-  __shared__ float s_red[2][kColTile / 32];
+// Sequential fp32 sum, max and min (and sum of squares) of column `tid` of a
+// 256 x 128 chunk in shared memory, rows in order.  The shared-memory loads
+// of kRowBatch rows are issued before the first add of the batch, so the
+// thread waits for one load latency per batch, not per row.
+constexpr int kRowBatch = 16;
 
-  const int tid = threadIdx.x;
-  const int t = blockIdx.x;
-  const int c = blockIdx.y;                    // chunk index into the partials
-  const int64_t col = static_cast<int64_t>(t) * kColTile + tid;
-  // this chunk's rows, the chunks folded with it, the slot and mean it feeds
-  int64_t row0 = static_cast<int64_t>(c) * kChunkRows;
-  int64_t n_rows = p.l;                        // rows of the (expert's) matrix
-  int c_first = 0, c_count = p.C, slot = t;
-  float* mu_out = p.mu_out;
-  if (kGrouped) {
-    pdl_wait_prior_grid();                     // the segment table comes from the previous launch
-    if (c >= __ldcg(p.totals)) return;         // a chunk past the last expert's
-    const int e = __ldcg(p.chunk_expert + c);
-    const MoeSeg sg = p.seg[e];
-    c_first = sg.chunk0;
-    c_count = sg.chunks;
-    row0 = sg.row0 + static_cast<int64_t>(c - sg.chunk0) * kChunkRows;
-    n_rows = sg.rows;
-    slot = e * p.T + t;
-    mu_out = p.mu_out + static_cast<int64_t>(e) * p.K;
-  }
-  const int rows = static_cast<int>(min64(kChunkRows, n_rows - static_cast<int64_t>(c - c_first) * kChunkRows));
-  constexpr uint32_t kElem = kBf16 ? 2u : 4u;
-  constexpr uint32_t kTileBytes = kChunkRows * kColTile * kElem;
+__device__ __forceinline__ void stats_step(float x, float& s, float& mx, float& mn) {
+  s = __fadd_rn(s, x);
+  mx = fmaxf(mx, x);
+  mn = fminf(mn, x);
+}
 
-  if (tid == 0) {
-    prefetch_tensormap(&map);
-    mbar_init(&bar, 1);
-    fence_mbarrier_init();
-  }
-  __syncthreads();
-  pdl_wait_prior_grid();
-  pdl_allow_next_grid();
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&bar, kTileBytes);
-    tma_load_2d(tile, &map, &bar, t * kColTile, static_cast<int32_t>(row0));
-    s_ok = mbar_wait(&bar, 0, p.status) ? 1u : 0u;
-    if (!s_ok) mbar_wait(&bar, 0, nullptr);   // a second bounded wait for the copy in flight
-  }
-  __syncthreads();
-  if (!s_ok) return;
-
-  // Sequential fp32 sum of this column over the chunk, plus max and min.
-  if (col < p.K) {
-    float s = 0.0f, mx = -INFINITY, mn = INFINITY, e = 0.0f;
-    if (kBf16) {
-      const uint16_t* v = reinterpret_cast<const uint16_t*>(tile) + tid;
-#pragma unroll 8
-      for (int i = 0; i < rows; ++i) {
-        const float x = __uint_as_float(static_cast<uint32_t>(v[i * kColTile]) << 16);
-        s = __fadd_rn(s, x);
-        mx = fmaxf(mx, x);
-        mn = fminf(mn, x);
-        if (kEnergy) e = __fmaf_rn(x, x, e);
-      }
-    } else {
-      const float* v = reinterpret_cast<const float*>(tile) + tid;
-#pragma unroll 8
-      for (int i = 0; i < rows; ++i) {
-        const float x = v[i * kColTile];
-        s = __fadd_rn(s, x);
-        mx = fmaxf(mx, x);
-        mn = fminf(mn, x);
+template <bool kBf16, bool kEnergy>
+__device__ __forceinline__ void chunk_column_stats(const uint8_t* tile, int tid, int rows, float& s, float& mx,
+                                                   float& mn, float& e) {
+  s = 0.0f;
+  mx = -INFINITY;
+  mn = INFINITY;
+  e = 0.0f;
+  int i = 0;
+  if (kBf16) {
+    const uint16_t* v = reinterpret_cast<const uint16_t*>(tile) + tid;
+    for (; i + kRowBatch <= rows; i += kRowBatch) {
+      uint32_t w[kRowBatch];
+#pragma unroll
+      for (int k = 0; k < kRowBatch; ++k) w[k] = v[(i + k) * kColTile];
+#pragma unroll
+      for (int k = 0; k < kRowBatch; ++k) {
+        const float x = __uint_as_float(w[k] << 16);
+        stats_step(x, s, mx, mn);
         if (kEnergy) e = __fmaf_rn(x, x, e);
       }
     }
-    if (kEnergy) p.part_e[static_cast<int64_t>(c) * p.K + col] = e;
-    const int64_t o = static_cast<int64_t>(c) * p.K + col;
-    const int64_t plane = static_cast<int64_t>(p.C) * p.K;
-    p.part[o] = s;
-    p.part[plane + o] = mx;
-    p.part[2 * plane + o] = mn;
+    for (; i < rows; ++i) {
+      const float x = __uint_as_float(static_cast<uint32_t>(v[i * kColTile]) << 16);
+      stats_step(x, s, mx, mn);
+      if (kEnergy) e = __fmaf_rn(x, x, e);
+    }
+  } else {
+    const float* v = reinterpret_cast<const float*>(tile) + tid;
+    for (; i + kRowBatch <= rows; i += kRowBatch) {
+      float w[kRowBatch];
+#pragma unroll
+      for (int k = 0; k < kRowBatch; ++k) w[k] = v[(i + k) * kColTile];
+#pragma unroll
+      for (int k = 0; k < kRowBatch; ++k) {
+        stats_step(w[k], s, mx, mn);
+        if (kEnergy) e = __fmaf_rn(w[k], w[k], e);
+      }
+    }
+    for (; i < rows; ++i) {
+      const float x = v[i * kColTile];
+      stats_step(x, s, mx, mn);
+      if (kEnergy) e = __fmaf_rn(x, x, e);
+    }
   }
+}
 
-  // Last CTA of this column tile finalizes it.  The CTA barrier orders every
-  // thread's partial stores before thread 0's ticket, an acquire-release
-  // increment at GPU scope: it publishes them (release, cumulative over the
-  // barrier) and, for the last CTA, makes every other CTA's partials visible
-  // to the fold below (acquire, passed on by the second barrier).
-  __syncthreads();
-  if (tid == 0) s_last = ticket_inc_acq_rel(&p.tickets[slot], static_cast<uint32_t>(c_count - 1)) ==
-                         static_cast<uint32_t>(c_count - 1);
-  __syncthreads();
-  if (!s_last) return;
+template <bool kEnergy>
+__device__ __forceinline__ void store_partials(const ColReduceParams& p, int c, int64_t col, float s, float mx,
+                                               float mn, float e) {
+  if (kEnergy) p.part_e[static_cast<int64_t>(c) * p.K + col] = e;
+  const int64_t o = static_cast<int64_t>(c) * p.K + col;
+  const int64_t plane = static_cast<int64_t>(p.C) * p.K;
+  p.part[o] = s;
+  p.part[plane + o] = mx;
+  p.part[2 * plane + o] = mn;
+}
 
-  // Each thread folds its column's chunk partials in chunk order; the loads
-  // of a batch of kBatch chunks (three planes) are all issued before the
-  // first add, so the fold waits for one L2 round trip per batch.
+// The fold of one column tile, run by every thread of the CTA that took the
+// tile's last ticket: each thread sums its column's chunk partials in chunk
+// order (the loads of a batch of kBatch chunks, three planes, all issued
+// before the first add, so the fold waits for one L2 round trip per batch),
+// writes mu and, through a CTA max, the tile's two amax slots.
+template <bool kEnergy>
+__device__ __forceinline__ void fold_tile(const ColReduceParams& p, int tid, int64_t col, int c_first, int c_count,
+                                          int64_t n_rows, float* mu_out, int slot, float (*s_red)[kColTile / 32]) {
   float a_xr = 0.0f, a_mu = 0.0f;
   float S = 0.0f, cmax = -INFINITY, cmin = INFINITY;
   if (col < p.K) {
@@ -209,6 +190,77 @@ __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_consta
     p.slot_xr[slot] = x;
     p.slot_mu[slot] = m;
   }
+}
+
+template <bool kBf16, bool kEnergy, bool kGrouped>
+__global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_constant__ CUtensorMap map,
+                                                             const ColReduceParams p) {
+  extern __shared__ __align__(1024) uint8_t tile[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t s_last, s_ok;
+  __shared__ float s_red[2][kColTile / 32];
+
+  const int tid = threadIdx.x;
+  const int t = blockIdx.x;
+  const int c = blockIdx.y;                    // chunk index into the partials
+  const int64_t col = static_cast<int64_t>(t) * kColTile + tid;
+  // this chunk's rows, the chunks folded with it, the slot and mean it feeds
+  int64_t row0 = static_cast<int64_t>(c) * kChunkRows;
+  int64_t n_rows = p.l;                        // rows of the (expert's) matrix
+  int c_first = 0, c_count = p.C, slot = t;
+  float* mu_out = p.mu_out;
+  if (kGrouped) {
+    pdl_wait_prior_grid();                     // the segment table comes from the previous launch
+    if (c >= __ldcg(p.totals)) return;         // a chunk past the last expert's
+    const int e = __ldcg(p.chunk_expert + c);
+    const MoeSeg sg = p.seg[e];
+    c_first = sg.chunk0;
+    c_count = sg.chunks;
+    row0 = sg.row0 + static_cast<int64_t>(c - sg.chunk0) * kChunkRows;
+    n_rows = sg.rows;
+    slot = e * p.T + t;
+    mu_out = p.mu_out + static_cast<int64_t>(e) * p.K;
+  }
+  const int rows = static_cast<int>(min64(kChunkRows, n_rows - static_cast<int64_t>(c - c_first) * kChunkRows));
+  constexpr uint32_t kElem = kBf16 ? 2u : 4u;
+  constexpr uint32_t kTileBytes = kChunkRows * kColTile * kElem;
+
+  if (tid == 0) {
+    prefetch_tensormap(&map);
+    mbar_init(&bar, 1);
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  pdl_wait_prior_grid();
+  pdl_allow_next_grid();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bar, kTileBytes);
+    tma_load_2d(tile, &map, &bar, t * kColTile, static_cast<int32_t>(row0));
+    s_ok = mbar_wait(&bar, 0, p.status) ? 1u : 0u;
+    if (!s_ok) mbar_wait(&bar, 0, nullptr);   // a second bounded wait for the copy in flight
+  }
+  __syncthreads();
+  if (!s_ok) return;
+
+  // Sequential fp32 sum of this column over the chunk, plus max and min.
+  if (col < p.K) {
+    float sum, mx, mn, e;
+    chunk_column_stats<kBf16, kEnergy>(tile, tid, rows, sum, mx, mn, e);
+    store_partials<kEnergy>(p, c, col, sum, mx, mn, e);
+  }
+
+  // Last CTA of this column tile finalizes it.  The CTA barrier orders every
+  // thread's partial stores before thread 0's ticket, an acquire-release
+  // increment at GPU scope: it publishes them (release, cumulative over the
+  // barrier) and, for the last CTA, makes every other CTA's partials visible
+  // to the fold below (acquire, passed on by the second barrier).
+  __syncthreads();
+  if (tid == 0) s_last = ticket_inc_acq_rel(&p.tickets[slot], static_cast<uint32_t>(c_count - 1)) ==
+                         static_cast<uint32_t>(c_count - 1);
+  __syncthreads();
+  if (!s_last) return;
+
+  fold_tile<kEnergy>(p, tid, col, c_first, c_count, n_rows, mu_out, slot, s_red);
 }
 
 template <bool kBf16, bool kEnergy, bool kGrouped>

@@ -50,7 +50,8 @@ def _dev(X, dt):
 
 @pytest.mark.parametrize("l,K,dt,mean_scale", [
     (256, 128, "f32", 1.0), (300, 192, "bf16", 1.0), (4133, 640, "bf16", 2.0),
-    (8192, 1024, "bf16", 1.0), (1024, 4096, "bf16", 0.25), (77, 8256, "bf16", 1.0)])
+    (8192, 1024, "bf16", 1.0), (1024, 4096, "bf16", 0.25), (77, 8256, "bf16", 1.0),
+    (5000, 2112, "bf16", 0.5)])     # ragged column tile and chunk
 def test_ratio_matches_oracle(api, l, K, dt, mean_scale):
     rng = inputs.rng_for(61, l + K)
     X = inputs.spiked_activations(rng, l, K, rank=2, s=(8.0, 4.0), n_hot=max(1, K // 100),

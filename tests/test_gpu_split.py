@@ -49,7 +49,8 @@ def _split(api, Xd, rm, seed=7, offset=0, grad=False, debug=True, fused=False):
 
 SHAPES = [(256, 128, "f32"), (300, 192, "bf16"), (1024, 1024, "bf16"), (4133, 640, "bf16"),
           (512, 6144, "bf16"), (64, 64, "f32"), (1, 256, "bf16"),
-          (40, 8256, "bf16")]     # K above the 8192-column window of the mean quantizer
+          (40, 8256, "bf16"),     # K above the 8192-column window of the mean quantizer
+          (5000, 2112, "bf16")]   # 17 x 20 reduce units, a ragged column tile and a ragged chunk
 
 
 @pytest.mark.parametrize("l,K,dt", SHAPES)
@@ -166,6 +167,28 @@ def test_repeat_calls_reuse_workspace(api):
     assert api.averis_check_status(ws) == 0
     for o in outs[1:]:
         assert np.array_equal(o[0], outs[0][0]) and np.array_equal(o[1], outs[0][1])
+
+
+def test_alternating_shapes_share_tickets(api):
+    """Reduces of different grids (4 x 4 and 17 x 20 units) count on the same
+    tickets; alternating them on one workspace gives the same bytes every time."""
+    ws = api.workspace(5000, 2112)
+    Xd, _ = _x(1024, 512, "bf16", seed=23)
+    Yd, _ = _x(5000, 2112, "bf16", seed=24)
+    outs = []
+    for _ in range(3):
+        got = []
+        for src, (l, K) in ((Xd, (1024, 512)), (Yd, (5000, 2112)), (Xd, (1024, 512))):
+            mu = torch.empty(K, device="cuda")
+            q = api.NVFP4Tensor(l, K)
+            api.averis_split_quant(src, "sr", 2, 0, False, mu, None, q, None, ws)
+            got.append((mu.cpu().numpy(), q.codes.cpu().numpy(), q.g_dec.item()))
+        outs.append(got)
+    assert api.averis_check_status(ws) == 0
+    for o in outs[1:]:
+        for (m0, c0, g0), (m1, c1, g1) in zip(o, outs[0]):
+            assert np.array_equal(m0, m1) and np.array_equal(c0, c1) and g0 == g1
+    assert np.array_equal(outs[0][0][0], outs[0][2][0]) and np.array_equal(outs[0][0][1], outs[0][2][1])
 
 
 @pytest.mark.parametrize("l,K,dt", [(8192, 1024, "bf16"), (16384, 3072, "bf16"), (32768, 4096, "bf16"),
