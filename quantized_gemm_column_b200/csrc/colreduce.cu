@@ -111,52 +111,62 @@ __device__ __forceinline__ void store_partials(const ColReduceParams& p, int c, 
 }
 
 // The fold of one column tile, run by every thread of the CTA that took the
-// tile's last ticket: each thread sums its column's chunk partials in chunk
-// order (the loads of a batch of kBatch chunks, three planes, all issued
-// before the first add, so the fold waits for one L2 round trip per batch),
-// writes mu and, through a CTA max, the tile's two amax slots.
+// tile's last ticket.  The tile's chunk partials (three planes) come into the
+// CTA's now idle tile buffer by TMA, kFoldRows chunks of each plane per round,
+// one round trip per round; each thread then sums its column's partials in
+// chunk order from shared memory, writes mu and, through a CTA max, the
+// tile's two amax slots.  `phase` is the parity of the tile barrier's next
+// phase.  Returns false if a copy never landed (status set).
+constexpr int kFoldRows = 40;                      // 3 planes x 40 x 128 fp32 = 60 KB of the tile buffer
+constexpr uint32_t kFoldPlaneBytes = kFoldRows * kColTile * 4;
+
 template <bool kEnergy>
-__device__ __forceinline__ void fold_tile(const ColReduceParams& p, int tid, int64_t col, int c_first, int c_count,
-                                          int64_t n_rows, float* mu_out, int slot, float (*s_red)[kColTile / 32]) {
+__device__ __forceinline__ bool fold_tile(const ColReduceParams& p, int tid, int64_t col, int t, int c_first,
+                                          int c_count, int64_t n_rows, float* mu_out, int slot,
+                                          float (*s_red)[kColTile / 32], uint8_t* tile, uint64_t* bar,
+                                          const CUtensorMap* pmap, uint32_t phase, uint32_t* s_ok) {
   float a_xr = 0.0f, a_mu = 0.0f;
   float S = 0.0f, cmax = -INFINITY, cmin = INFINITY;
-  if (col < p.K) {
+  const float* sp = reinterpret_cast<const float*>(tile);
+  for (int c0 = 0; c0 < c_count; c0 += kFoldRows) {
+    const int n = c_count - c0 < kFoldRows ? c_count - c0 : kFoldRows;
+    __syncthreads();                                // the buffer's previous contents are no longer read
+    if (tid == 0) {
+      fence_proxy_async_smem();                     // ... before the copies overwrite it
+      fence_proxy_async_global();                   // the acquired partials, for the copy engine
+      mbar_arrive_expect_tx(bar, 3 * kFoldPlaneBytes);
+#pragma unroll
+      for (int pl = 0; pl < 3; ++pl)
+        tma_load_2d(tile + pl * kFoldPlaneBytes, pmap, bar, t * kColTile, pl * p.C + c_first + c0);
+      *s_ok = mbar_wait(bar, phase, p.status) ? 1u : 0u;
+      if (!*s_ok) mbar_wait(bar, phase, nullptr);   // a second bounded wait for the copies in flight
+    }
+    __syncthreads();
+    if (!*s_ok) return false;
+    phase ^= 1u;
+    if (col < p.K) {
+#pragma unroll 8
+      for (int u = 0; u < n; ++u) {
+        S = __fadd_rn(S, sp[u * kColTile + tid]);
+        cmax = fmaxf(cmax, sp[(kFoldRows + u) * kColTile + tid]);
+        cmin = fminf(cmin, sp[(2 * kFoldRows + u) * kColTile + tid]);
+      }
+    }
+  }
+  if (col < p.K && kEnergy) {
+    // the column's sum of squares, chunks in order
     constexpr int kBatch = 16;
-    const int64_t plane = static_cast<int64_t>(p.C) * p.K;
-    for (int c0 = 0; c0 < c_count; c0 += kBatch) {
-      float ps[kBatch], px[kBatch], pn[kBatch];
+    float E = 0.0f;
+    for (int c0 = 0; c0 < p.C; c0 += kBatch) {
+      float pe[kBatch];
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        if (c0 + u < c_count) {
-          const int64_t o = static_cast<int64_t>(c_first + c0 + u) * p.K + col;
-          ps[u] = __ldcg(&p.part[o]);
-          px[u] = __ldcg(&p.part[plane + o]);
-          pn[u] = __ldcg(&p.part[2 * plane + o]);
-        }
-      }
+      for (int u = 0; u < kBatch; ++u)
+        if (c0 + u < p.C) pe[u] = __ldcg(&p.part_e[static_cast<int64_t>(c0 + u) * p.K + col]);
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        if (c0 + u < c_count) {
-          S = __fadd_rn(S, ps[u]);
-          cmax = fmaxf(cmax, px[u]);
-          cmin = fminf(cmin, pn[u]);
-        }
-      }
+      for (int u = 0; u < kBatch; ++u)
+        if (c0 + u < p.C) E = __fadd_rn(E, pe[u]);
     }
-    if (kEnergy) {
-      // the column's sum of squares, chunks in order
-      float E = 0.0f;
-      for (int c0 = 0; c0 < p.C; c0 += kBatch) {
-        float pe[kBatch];
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u)
-          if (c0 + u < p.C) pe[u] = __ldcg(&p.part_e[static_cast<int64_t>(c0 + u) * p.K + col]);
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u)
-          if (c0 + u < p.C) E = __fadd_rn(E, pe[u]);
-      }
-      p.energy[col] = E;
-    }
+    p.energy[col] = E;
   }
   if (col < p.K) {
     if (!isfinite(S)) raise_status(p.status, AVR_ERR_NONFINITE);
@@ -190,10 +200,12 @@ __device__ __forceinline__ void fold_tile(const ColReduceParams& p, int tid, int
     p.slot_xr[slot] = x;
     p.slot_mu[slot] = m;
   }
+  return true;
 }
 
 template <bool kBf16, bool kEnergy, bool kGrouped>
 __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_constant__ CUtensorMap map,
+                                                             const __grid_constant__ CUtensorMap pmap,
                                                              const ColReduceParams p) {
   extern __shared__ __align__(1024) uint8_t tile[];
   __shared__ uint64_t bar;
@@ -260,16 +272,17 @@ __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_consta
   __syncthreads();
   if (!s_last) return;
 
-  fold_tile<kEnergy>(p, tid, col, c_first, c_count, n_rows, mu_out, slot, s_red);
+  if (tid == 0) prefetch_tensormap(&pmap);
+  fold_tile<kEnergy>(p, tid, col, t, c_first, c_count, n_rows, mu_out, slot, s_red, tile, &bar, &pmap, 1u, &s_ok);
 }
 
 template <bool kBf16, bool kEnergy, bool kGrouped>
-static cudaError_t launch_colreduce_t(const CUtensorMap& map, const ColReduceParams& p, dim3 grid, size_t smem,
-                                      cudaStream_t s, bool pdl) {
+static cudaError_t launch_colreduce_t(const CUtensorMap& map, const CUtensorMap& pmap, const ColReduceParams& p,
+                                      dim3 grid, size_t smem, cudaStream_t s, bool pdl) {
   const void* fn = reinterpret_cast<const void*>(colreduce_kernel<kBf16, kEnergy, kGrouped>);
   cudaError_t e = set_max_dynamic_smem(fn, smem);
   if (e != cudaSuccess) return e;
-  return launch_ex(colreduce_kernel<kBf16, kEnergy, kGrouped>, grid, dim3(kColTile), smem, s, pdl, map, p);
+  return launch_ex(colreduce_kernel<kBf16, kEnergy, kGrouped>, grid, dim3(kColTile), smem, s, pdl, map, pmap, p);
 }
 
 cudaError_t launch_colreduce(const ColReduceArgs& a, cudaStream_t s, bool pdl) {
@@ -299,17 +312,23 @@ cudaError_t launch_colreduce(const ColReduceArgs& a, cudaStream_t s, bool pdl) {
   const int T = static_cast<int>((a.K + kColTile - 1) / kColTile);
   p.T = T;
   if (p.C < 1) return cudaSuccess;
+  // the partials as a [3 C, K] fp32 array, for the fold's copies
+  CUtensorMap pmap;
+  if (!make_tensor_map_2d(&pmap, p.part, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 3 * static_cast<uint64_t>(p.C),
+                          static_cast<uint64_t>(a.K), kFoldRows, kColTile, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
   const size_t smem = static_cast<size_t>(kChunkRows) * kColTile * elem;
+  static_assert(3 * kFoldPlaneBytes <= kChunkRows * kColTile * 2, "fold rounds fit the bf16 tile buffer");
   const dim3 grid(T, p.C);
   if (a.seg != nullptr)   // grouped (MoE): no energy pass
-    return bf16 ? launch_colreduce_t<true, false, true>(map, p, grid, smem, s, pdl)
-                : launch_colreduce_t<false, false, true>(map, p, grid, smem, s, pdl);
+    return bf16 ? launch_colreduce_t<true, false, true>(map, pmap, p, grid, smem, s, pdl)
+                : launch_colreduce_t<false, false, true>(map, pmap, p, grid, smem, s, pdl);
   if (a.energy) {
-    return bf16 ? launch_colreduce_t<true, true, false>(map, p, grid, smem, s, pdl)
-                : launch_colreduce_t<false, true, false>(map, p, grid, smem, s, pdl);
+    return bf16 ? launch_colreduce_t<true, true, false>(map, pmap, p, grid, smem, s, pdl)
+                : launch_colreduce_t<false, true, false>(map, pmap, p, grid, smem, s, pdl);
   }
-  return bf16 ? launch_colreduce_t<true, false, false>(map, p, grid, smem, s, pdl)
-              : launch_colreduce_t<false, false, false>(map, p, grid, smem, s, pdl);
+  return bf16 ? launch_colreduce_t<true, false, false>(map, pmap, p, grid, smem, s, pdl)
+              : launch_colreduce_t<false, false, false>(map, pmap, p, grid, smem, s, pdl);
 }
 
 // ---------------------------------------------------------------------------
