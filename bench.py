@@ -46,7 +46,7 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="averis", choices=["averis", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--cpu-sample-rows", type=int, default=4096)
+    p.add_argument("--cpu-sample-rows", type=int, default=8192)
     p.add_argument("--cpu-sample-steps", type=int, default=2)
     p.add_argument("--copies", type=int, default=4, help="input copies rotated between steps")
     return p.parse_args()
