@@ -566,10 +566,10 @@ def run_gpu(args, rank, world, local_rank):
                 "traffic_unit": "DRAM bytes per step (fwd + dgrad launches)",
                 "peak_source": f"{peak_src} bf16 x 4 (nominal FP4:BF16 ratio)"}
     else:
-        roof = {"bound": "hbm", "kernel": "colreduce_kernel + quant_kernel (split-quant, X and dY)",
+        roof = {"bound": "hbm", "kernel": "colreduce_kernel + fold_kernel + quant_kernel (split-quant, X and dY)",
                 "achieved": sq_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": sq_gbs / hbm_peak,
                 "traffic": measured_traffic("split-quant"),
-                "traffic_unit": "DRAM bytes per step (4 launches: reduce and quantize, X and dY)",
+                "traffic_unit": "DRAM bytes per step (6 launches: reduce, fold and quantize, X and dY)",
                 "algorithmic_bytes_per_step": sq_bytes(L, M) + sq_bytes(L, N),
                 "peak_source": f"{peak_src} HBM copy"}
 

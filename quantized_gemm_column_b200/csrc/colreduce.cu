@@ -203,7 +203,7 @@ __device__ __forceinline__ bool fold_tile(const ColReduceParams& p, int tid, int
   return true;
 }
 
-template <bool kBf16, bool kEnergy, bool kGrouped>
+template <bool kBf16, bool kEnergy, bool kGrouped, bool kDeferFold>
 __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_constant__ CUtensorMap map,
                                                              const __grid_constant__ CUtensorMap pmap,
                                                              const ColReduceParams p) {
@@ -261,6 +261,8 @@ __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_consta
     store_partials<kEnergy>(p, c, col, sum, mx, mn, e);
   }
 
+  if (kDeferFold) return;   // fold_kernel, the next launch, folds every tile
+
   // Last CTA of this column tile finalizes it.  The CTA barrier orders every
   // thread's partial stores before thread 0's ticket, an acquire-release
   // increment at GPU scope: it publishes them (release, cumulative over the
@@ -276,13 +278,42 @@ __global__ void __launch_bounds__(kColTile) colreduce_kernel(const __grid_consta
   fold_tile<kEnergy>(p, tid, col, t, c_first, c_count, n_rows, mu_out, slot, s_red, tile, &bar, &pmap, 1u, &s_ok);
 }
 
-template <bool kBf16, bool kEnergy, bool kGrouped>
+// The fold as its own launch, one CTA per column tile, after a reduce that
+// took no tickets (the dense split and vanilla amax): the partials are
+// complete once the reduce grid is, so its CTAs hold their SM slots only for
+// the copy and the sum.
+__global__ void __launch_bounds__(kColTile) fold_kernel(const __grid_constant__ CUtensorMap pmap,
+                                                        const ColReduceParams p) {
+  extern __shared__ __align__(1024) uint8_t buf[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t s_ok;
+  __shared__ float s_red[2][kColTile / 32];
+  const int tid = threadIdx.x, t = blockIdx.x;
+  if (tid == 0) {
+    prefetch_tensormap(&pmap);
+    mbar_init(&bar, 1);
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  pdl_wait_prior_grid();
+  pdl_allow_next_grid();
+  fold_tile<false>(p, tid, static_cast<int64_t>(t) * kColTile + tid, t, 0, p.C, p.l, p.mu_out, t, s_red, buf, &bar,
+                   &pmap, 0u, &s_ok);
+}
+
+template <bool kBf16, bool kEnergy, bool kGrouped, bool kDeferFold = false>
 static cudaError_t launch_colreduce_t(const CUtensorMap& map, const CUtensorMap& pmap, const ColReduceParams& p,
                                       dim3 grid, size_t smem, cudaStream_t s, bool pdl) {
-  const void* fn = reinterpret_cast<const void*>(colreduce_kernel<kBf16, kEnergy, kGrouped>);
+  const void* fn = reinterpret_cast<const void*>(colreduce_kernel<kBf16, kEnergy, kGrouped, kDeferFold>);
   cudaError_t e = set_max_dynamic_smem(fn, smem);
   if (e != cudaSuccess) return e;
-  return launch_ex(colreduce_kernel<kBf16, kEnergy, kGrouped>, grid, dim3(kColTile), smem, s, pdl, map, pmap, p);
+  e = launch_ex(colreduce_kernel<kBf16, kEnergy, kGrouped, kDeferFold>, grid, dim3(kColTile), smem, s, pdl, map,
+                pmap, p);
+  if (e != cudaSuccess || !kDeferFold) return e;
+  const size_t fold_smem = 3 * static_cast<size_t>(kFoldPlaneBytes);
+  e = set_max_dynamic_smem(reinterpret_cast<const void*>(fold_kernel), fold_smem);
+  if (e != cudaSuccess) return e;
+  return launch_ex(fold_kernel, dim3(grid.x), dim3(kColTile), fold_smem, s, true, pmap, p);
 }
 
 cudaError_t launch_colreduce(const ColReduceArgs& a, cudaStream_t s, bool pdl) {
@@ -327,8 +358,8 @@ cudaError_t launch_colreduce(const ColReduceArgs& a, cudaStream_t s, bool pdl) {
     return bf16 ? launch_colreduce_t<true, true, false>(map, pmap, p, grid, smem, s, pdl)
                 : launch_colreduce_t<false, true, false>(map, pmap, p, grid, smem, s, pdl);
   }
-  return bf16 ? launch_colreduce_t<true, false, false>(map, pmap, p, grid, smem, s, pdl)
-              : launch_colreduce_t<false, false, false>(map, pmap, p, grid, smem, s, pdl);
+  return bf16 ? launch_colreduce_t<true, false, false, true>(map, pmap, p, grid, smem, s, pdl)
+              : launch_colreduce_t<false, false, false, true>(map, pmap, p, grid, smem, s, pdl);
 }
 
 // ---------------------------------------------------------------------------
