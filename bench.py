@@ -4,8 +4,9 @@
 
 One step = one forward and one dgrad pass of the Qwen3-0.6B fused-QKV
 projection (X bf16 [8192, 1024], W [1024, 4096], dY bf16 [8192, 4096],
-Philox stochastic rounding): column reduce, split quantizer (+ mean quantizer
-and rank-one row) and tcgen05 FP4 GEMM for each pass, six kernel launches.
+Philox stochastic rounding): column reduce, fold, split quantizer (+ mean
+quantizer and rank-one row) and tcgen05 FP4 GEMM for each pass, eight kernel
+launches.
 The weight quantization is done once before timing (it runs once per weight
 update, not per linear) and is reported on its own.
 
@@ -661,7 +662,8 @@ def run_gpu(args, rank, world, local_rank):
                 "ms_per_step": e2e_ms,
                 "copies": "pinned host <-> device every step, overlapping the neighbouring steps' kernels "
                           "(upload, compute and download streams; double-buffered)"},
-        "gpu_launches": 6 * args.steps,
+        # per step: column reduce, fold, quantizer and GEMM, for the forward and for the dgrad
+        "gpu_launches": 8 * args.steps,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)

@@ -227,7 +227,7 @@ avr_status nvfp4_gemm(const avr_nvfp4* a, const avr_nvfp4* b, const float* bias,
 /* Forward: Y [l, n] = 1 (Q_4(mu_X) W_bar) + Q_4(X - 1 mu_X) W_bar for
  * X [l, m] and w_fwd = Q_4(W^T) [n, m].  save_xr / save_mu (nullable)
  * receive the quantized operands for a later weight-gradient pass; when
- * NULL they live in the workspace.  Three launches: column reduce,
+ * NULL they live in the workspace.  Four launches: column reduce, fold,
  * split-quantize (+ mean quantize + rank-one row), GEMM. */
 avr_status averis_linear_fwd(const void* X, avr_dtype xt, int64_t l, int64_t m, int64_t n,
                              const avr_nvfp4* w_fwd, avr_round rm, uint64_t seed,
@@ -243,7 +243,8 @@ avr_status averis_linear_dgrad(const void* D, avr_dtype dt, int64_t l, int64_t m
                                size_t ws_bytes, avr_stream stream);
 
 /* Vanilla NVFP4 forward / dgrad ([R3.1], [Abs] "vanilla NVFP4"): Y = Q_4(X)
- * W_bar, dX = Q_4(D) W_bar^T, the same three launches without the split. */
+ * W_bar, dX = Q_4(D) W_bar^T, the same four launches without the split
+ * (the reduce and the fold then give the amax only). */
 avr_status nvfp4_linear_fwd(const void* X, avr_dtype xt, int64_t l, int64_t m, int64_t n,
                             const avr_nvfp4* w_fwd, avr_round rm, uint64_t seed, uint64_t offset,
                             void* Y, avr_dtype yt, void* ws, size_t ws_bytes, avr_stream stream);
