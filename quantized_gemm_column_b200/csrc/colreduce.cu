@@ -6,16 +6,19 @@
 //   p[c][j] = (((+0 + x[256c][j]) + x[256c+1][j]) + ...)    rows of chunk c in order
 //   S[j]    = (((+0 + p[0][j]) + p[1][j]) + ...)              chunks in order
 //   mu[j]   = S[j] / l                                        IEEE division
-// The same pass keeps the column max and min, so the last CTA of a column tile
+// The same pass keeps the column max and min, so the fold of a column tile
 // can also give max_i |fl(x_ij - mu_j)| = max(fl(colmax - mu), fl(mu - colmin))
 // (rounded subtraction is monotone), the amax the residual's tensor scale
 // needs, without a third pass over X.
 //
-// Grid (column tiles of 128, chunks of 256 rows).  One TMA copy brings the
-// 256 x 128 tile into shared memory; thread j then runs the sequential sum of
-// column j over the chunk.  Partials go to the workspace; the CTA that takes
-// the last ticket of its column tile (atomicInc wraps the ticket back to 0)
-// sums the partials in chunk order and writes mu and the tile's amax slots.
+// colreduce_kernel: grid (column tiles of 128, chunks of 256 rows).  One TMA
+// copy brings the 256 x 128 tile into shared memory; thread j then runs the
+// sequential sum of column j over the chunk, and the partials go to the
+// workspace.  The tile's fold (the partials summed in chunk order, mu and the
+// tile's amax slots) is then either a separate fold_kernel launch (the dense
+// split and vanilla amax: the reduce takes no tickets), or run by the CTA
+// that takes the tile's last ticket (the R monitor's and the MoE layer's
+// reduces; atomicInc wraps the ticket back to 0).
 #include "device.cuh"
 #include "internal.h"
 
@@ -110,9 +113,9 @@ __device__ __forceinline__ void store_partials(const ColReduceParams& p, int c, 
   p.part[2 * plane + o] = mn;
 }
 
-// The fold of one column tile, run by every thread of the CTA that took the
-// tile's last ticket.  The tile's chunk partials (three planes) come into the
-// CTA's now idle tile buffer by TMA, kFoldRows chunks of each plane per round,
+// The fold of one column tile, run by every thread of a fold_kernel CTA or of
+// the CTA that took the tile's last ticket.  The tile's chunk partials (three
+// planes) come into the CTA's shared buffer by TMA, kFoldRows chunks of each plane per round,
 // one round trip per round; each thread then sums its column's partials in
 // chunk order from shared memory, writes mu and, through a CTA max, the
 // tile's two amax slots.  `phase` is the parity of the tile barrier's next
