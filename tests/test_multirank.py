@@ -97,3 +97,23 @@ def test_measured_traffic_follows_kernel_sources(tmp_path, monkeypatch):
     assert bench.measured_traffic("gemm") is None
     prof.write_text("    traffic-digest: 0000000000000000\n    traffic-split-quant-bytes-per-step: 123\n")
     assert bench.measured_traffic("split-quant") is None
+
+
+def test_reference_arm_stops_at_its_time_budget(monkeypatch, capsys):
+    """The oracle arm times at most its wall-clock budget of steps, whatever
+    step count it is given, and says how many it timed beside the request;
+    its config is the GPU arm's workload."""
+    import argparse
+    import bench
+    monkeypatch.setattr(bench, "REF_WARMUP_S", 0.05)
+    monkeypatch.setattr(bench, "REF_TIMED_S", 0.2)
+    args = argparse.Namespace(gpus=1, steps=10**6, warmup=10**6)
+    bench.run_reference(args, 0, 1)
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert 1 <= d["steps"] < d["steps_requested"] == 10**6
+    assert 1 <= d["warmup"] < d["warmup_requested"] == 10**6
+    assert d["config"]["workload"] == bench.WORKLOAD
+    assert (d["config"]["l"], d["config"]["m"], d["config"]["n"]) == (bench.L, bench.M, bench.N)
+    assert d["value"] > 0 and d["cpu_baseline"]["value"] == d["value"]
