@@ -134,3 +134,47 @@ def test_wgrad_validation(lib):
     assert lib.averis_split_quant_t(Y, 1, 300, 128, 0, 0, 0, 0, None, None, ctypes.byref(q), ws,
                                     1 << 30, None) == api.AVR_ERR_INVALID_ARG
     assert api.averis_wgrad_workspace_size(8192, 1024, 4096) > (1024 + 4096) * 8192 // 2
+
+
+def test_moe_validation(lib):
+    """The MoE entry points reject bad arguments before any launch: the
+    buffer's row count, the expert-count and tile limits, null or misaligned
+    pointers, descriptors that disagree with the call, a short workspace."""
+    from quantized_gemm_column_b200 import api
+    ws = ctypes.c_void_p(256)
+    X = ctypes.c_void_p(16)
+    cnt = ctypes.c_void_p(64)
+    E, l_cap, K = 4, 512, 256
+    xr = api.avr_nvfp4(16, 16, 16, l_cap, K)
+    f = lib.averis_moe_split_quant
+    args = lambda **kw: [kw.get("X", X), kw.get("xt", 1), kw.get("l_cap", l_cap), kw.get("cnt", cnt),
+                         kw.get("E", E), kw.get("K", K), 0, 0, 0, 0, None, None, ctypes.byref(kw.get("xr", xr)),
+                         ws, kw.get("ws_bytes", 1 << 40), None]
+    assert f(*args(xt=7)) == api.AVR_ERR_INVALID_ARG
+    assert f(*args(l_cap=300, xr=api.avr_nvfp4(16, 16, 16, 300, K))) == api.AVR_ERR_UNSUPPORTED_SHAPE
+    assert f(*args(E=0)) == api.AVR_ERR_UNSUPPORTED_SHAPE
+    assert f(*args(E=1025)) == api.AVR_ERR_UNSUPPORTED_SHAPE
+    # E x ceil(K / 128) column tiles above the 4096 slots
+    assert f(*args(E=1024, K=640, xr=api.avr_nvfp4(16, 16, 16, l_cap, 640))) == api.AVR_ERR_UNSUPPORTED_SHAPE
+    assert f(*args(K=96, xr=api.avr_nvfp4(16, 16, 16, l_cap, 96))) == api.AVR_ERR_UNSUPPORTED_SHAPE
+    assert f(*args(cnt=None)) == api.AVR_ERR_INVALID_ARG
+    assert f(*args(xr=api.avr_nvfp4(16, 16, 16, 384, K))) == api.AVR_ERR_INVALID_ARG
+    assert f(*args(X=ctypes.c_void_p(24))) == api.AVR_ERR_MISALIGNED
+    assert f(*args(cnt=ctypes.c_void_p(66))) == api.AVR_ERR_MISALIGNED
+    assert f(*args(ws_bytes=64)) == api.AVR_ERR_WORKSPACE_TOO_SMALL
+    # linear: N must be a multiple of 128, the stacked weights [E n, m]
+    m, n = 256, 384
+    w = api.avr_nvfp4(16, 16, 16, E * n, m)
+    g = lib.averis_moe_linear_fwd
+    Y = ctypes.c_void_p(16)
+    assert g(X, 1, l_cap, cnt, E, m, 320, ctypes.byref(api.avr_nvfp4(16, 16, 16, E * 320, m)), 1, 0, 0, Y, 1,
+             ws, 1 << 40, None) == api.AVR_ERR_UNSUPPORTED_SHAPE
+    assert g(X, 1, l_cap, cnt, E, m, n, ctypes.byref(api.avr_nvfp4(16, 16, 16, n, m)), 1, 0, 0, Y, 1, ws,
+             1 << 40, None) == api.AVR_ERR_INVALID_ARG
+    assert g(X, 1, l_cap, cnt, E, m, n, ctypes.byref(w), 1, 0, 0, None, 1, ws, 1 << 40,
+             None) == api.AVR_ERR_INVALID_ARG
+    assert g(X, 1, l_cap, cnt, E, m, n, ctypes.byref(w), 1, 0, 0, Y, 1, ws, 64,
+             None) == api.AVR_ERR_WORKSPACE_TOO_SMALL
+    # the workspace grows with the experts and the buffer
+    assert api.averis_moe_workspace_size(l_cap, K, 0, 8) > api.averis_moe_workspace_size(l_cap, K, 0, 4)
+    assert api.averis_moe_workspace_size(2 * l_cap, K, 0, 4) > api.averis_moe_workspace_size(l_cap, K, 0, 4)
