@@ -178,3 +178,59 @@ def test_moe_validation(lib):
     # the workspace grows with the experts and the buffer
     assert api.averis_moe_workspace_size(l_cap, K, 0, 8) > api.averis_moe_workspace_size(l_cap, K, 0, 4)
     assert api.averis_moe_workspace_size(2 * l_cap, K, 0, 4) > api.averis_moe_workspace_size(l_cap, K, 0, 4)
+
+
+def test_linear_and_weight_validation(lib):
+    """The linear, weight, one-kernel-split and rank-one-row entry points
+    reject bad arguments before any launch; l = 0 is a no-op."""
+    from quantized_gemm_column_b200 import api
+    ws = ctypes.c_void_p(256)
+    X, Y = ctypes.c_void_p(16), ctypes.c_void_p(32)
+    l, m, n = 256, 128, 192
+    wf = api.avr_nvfp4(16, 16, 16, n, m)          # w_fwd [n, m]
+    wd = api.avr_nvfp4(16, 16, 16, m, n)          # w_dgrad [m, n]
+    fwd = lambda **kw: lib.averis_linear_fwd(kw.get("X", X), kw.get("xt", 1), kw.get("l", l), kw.get("m", m),
+                                             kw.get("n", n), ctypes.byref(kw.get("w", wf)), 1, 0, 0,
+                                             kw.get("Y", Y), kw.get("yt", 1), kw.get("save_xr"), None, ws,
+                                             kw.get("ws_bytes", 1 << 40), None)
+    assert fwd(xt=3) == api.AVR_ERR_INVALID_ARG
+    assert fwd(yt=3) == api.AVR_ERR_INVALID_ARG
+    assert fwd(m=96, w=api.avr_nvfp4(16, 16, 16, n, 96)) == api.AVR_ERR_UNSUPPORTED_SHAPE
+    assert fwd(n=100, w=api.avr_nvfp4(16, 16, 16, 100, m)) == api.AVR_ERR_UNSUPPORTED_SHAPE
+    assert fwd(w=wd) == api.AVR_ERR_INVALID_ARG                      # [m, n] given for [n, m]
+    assert fwd(save_xr=ctypes.byref(api.avr_nvfp4(16, 16, 16, l, n))) == api.AVR_ERR_INVALID_ARG
+    assert fwd(Y=ctypes.c_void_p(40)) == api.AVR_ERR_MISALIGNED
+    assert fwd(ws_bytes=64) == api.AVR_ERR_WORKSPACE_TOO_SMALL
+    assert fwd(l=0) == api.AVR_OK
+    assert lib.averis_linear_dgrad(X, 1, l, m, n, ctypes.byref(wf), 1, 0, 0, Y, 1, ws, 1 << 40,
+                                   None) == api.AVR_ERR_INVALID_ARG       # w_fwd given for w_dgrad
+    # weights: both dimensions multiples of 64, descriptors [n, m] and [m, n]
+    qw = lib.averis_quant_weight
+    assert qw(X, 1, m, 100, ctypes.byref(wf), ctypes.byref(wd), ws, 1 << 40, None) == api.AVR_ERR_UNSUPPORTED_SHAPE
+    assert qw(X, 1, m, n, ctypes.byref(wd), ctypes.byref(wf), ws, 1 << 40, None) == api.AVR_ERR_INVALID_ARG
+    assert qw(ctypes.c_void_p(24), 1, m, n, ctypes.byref(wf), ctypes.byref(wd), ws, 1 << 40,
+              None) == api.AVR_ERR_MISALIGNED
+    # one-kernel split
+    xr = api.avr_nvfp4(16, 16, 16, l, m)
+    fu = lib.averis_split_quant_fused
+    assert fu(X, 1, l, 100, 0, 0, 0, 0, None, None, ctypes.byref(xr), ws, 1 << 40, None) == api.AVR_ERR_UNSUPPORTED_SHAPE
+    assert fu(X, 1, l, m, 0, 0, 0, 0, None, None, ctypes.byref(wf), ws, 1 << 40, None) == api.AVR_ERR_INVALID_ARG
+    assert fu(X, 1, 0, m, 0, 0, 0, 0, None, None, ctypes.byref(xr), ws, 1 << 40, None) == api.AVR_OK
+    # rank-one row: mu_bar [1, K] against W_bar [N, K]
+    mq = api.avr_nvfp4(16, 16, 16, 1, m)
+    assert lib.averis_bias_row(None, ctypes.byref(wf), Y, ws, 1 << 40, None) == api.AVR_ERR_INVALID_ARG
+    assert lib.averis_bias_row(ctypes.byref(mq), ctypes.byref(wd), Y, ws, 1 << 40, None) == api.AVR_ERR_INVALID_ARG
+
+
+def test_valid_call_without_a_device_fails_loudly(lib):
+    """A call that passes every host check returns AVR_ERR_NO_DEVICE when no
+    sm_100 device is current: there is no CPU path to fall back to.  (Skipped
+    where a GPU is visible: the pointers here are not device memory.)"""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is visible; this check is for a host without one")
+    from quantized_gemm_column_b200 import api
+    wf = api.avr_nvfp4(16, 16, 16, 192, 128)
+    st = lib.averis_linear_fwd(ctypes.c_void_p(16), 1, 256, 128, 192, ctypes.byref(wf), 1, 0, 0,
+                               ctypes.c_void_p(32), 1, None, None, ctypes.c_void_p(256), 1 << 40, None)
+    assert st == api.AVR_ERR_NO_DEVICE
