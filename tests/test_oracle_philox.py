@@ -77,3 +77,45 @@ def test_sr_is_unbiased_over_seeds():
     tol = 5 * sd / math.sqrt(S) + 2.0 * step * scale / 65536 + 1e-12
     assert np.all(np.abs(mean - T)[inside] <= tol[inside])
     assert inside.sum() > 200
+
+
+def test_group_values_uniform_and_round_ups_uncorrelated():
+    """Pin of the random-value-to-element map (``group_values16``): it does
+    not come from the pages, and a mistake in it (two elements of a group
+    drawing the same bits, a byte lost or repeated) would leave every
+    bit-exact test of the oracle against itself green.  So check what any
+    correct map must give, on 2^20 groups of four elements:
+
+    - each of the four 16-bit values is uniform: chi^2 of its high byte and
+      of its low byte over 256 bins below the 1e-6 quantile of chi^2(255);
+    - the round-up decisions of ``e2m1_sr`` for every pair of elements in a
+      group are uncorrelated (|corr| < 5 standard errors, 5 / sqrt(2^20)) and
+      each happens with the probability the rounding rule fixes, at p = 0.5
+      (y = 1.25, halfway between 1 and 1.5) and p = 0.3 (y = 1.15).
+
+    A group draws 32 random bits for its four elements, so the values of a
+    pair are not independent as a whole; what stochastic rounding needs is
+    that the decisions are, and enumerating all 2^16 values of a pair sharing
+    one half-word gives |corr| < 5e-4 at every p tried -- well inside the
+    bound -- while a pair reading the same bits gives corr = 1."""
+    n = 1 << 20
+    r = random_bits16(seed=0x5EED0001, offset=7, tag=3, n_elements=4 * n).reshape(n, 4)
+    for k in range(4):
+        for part in (r[:, k] >> 8, r[:, k] & 0xFF):
+            counts = np.bincount(part, minlength=256)
+            chi2 = float(np.sum((counts - n / 256) ** 2 / (n / 256)))
+            assert chi2 < 370, (k, chi2)
+    bound = 5.0 / math.sqrt(n)
+    for y in (1.25, 1.15):
+        codes = oracle.e2m1_sr(np.full((n, 4), y, dtype=np.float32), r)
+        assert set(np.unique(codes)) <= {2, 3}            # 1.0 or 1.5
+        up = (codes == 3).astype(np.float64)
+        F = math.floor((np.float32(y) - np.float32(1.0)) / np.float32(0.5) * 65536.0)
+        p = F / 65536.0
+        se = math.sqrt(p * (1 - p) / n)
+        for k in range(4):
+            assert abs(up[:, k].mean() - p) < 5 * se, (y, k, up[:, k].mean(), p)
+        for i in range(4):
+            for j in range(i + 1, 4):
+                corr = np.corrcoef(up[:, i], up[:, j])[0, 1]
+                assert abs(corr) < bound, (y, i, j, corr)
