@@ -109,8 +109,25 @@ size_t averis_workspace_size(int64_t l, int64_t K, int64_t N);
 avr_status averis_workspace_init(void* ws, size_t ws_bytes, avr_stream stream);
 
 /* Synchronize `stream`, return the first device-side error latched in the
- * workspace status word since the last check (AVR_OK if none) and clear it. */
+ * workspace status word since the last check (AVR_OK if none) and clear it.
+ * After an error the whole 256-byte status block is cleared (the status
+ * word, the one-kernel split's grid-barrier words, which a kernel that gave
+ * up may have left part-counted, and the wait limit below), so the workspace
+ * is ready for the next call. */
 avr_status averis_check_status(void* ws, avr_stream stream);
+
+/* Bound, in nanoseconds, of the waits in which a CTA waits for other CTAs
+ * (the grid-wide barriers of averis_split_quant_fused); 0 restores the
+ * default of 2 s.  Written in stream order into the workspace's status block
+ * (a zero-filled workspace has the default); averis_check_status resets it
+ * to the default after an error.  A wait that runs out records
+ * AVR_ERR_DEVICE_TIMEOUT and its kernel returns with no copy in flight; the
+ * waits for a CTA's own copies keep the 2 s bound.  This is failure
+ * detection (a grid that cannot be co-resident, a stuck CTA), not a tuning
+ * knob.  Errors: AVR_ERR_INVALID_ARG (null ws), AVR_ERR_MISALIGNED (ws not
+ * 256-byte aligned), AVR_ERR_WORKSPACE_TOO_SMALL (ws_bytes < 256),
+ * AVR_ERR_NO_DEVICE. */
+avr_status averis_set_wait_limit(void* ws, size_t ws_bytes, uint64_t limit_ns, avr_stream stream);
 
 /* Static description of a status code. */
 const char* averis_status_string(avr_status status);
@@ -184,10 +201,16 @@ avr_status averis_split_quant_fused(const void* X, avr_dtype xt, int64_t l, int6
  *   0; the first device-side error of the call (AVR_ERR_NONFINITE,
  *   AVR_ERR_DEVICE_TIMEOUT) is stored there.
  *   The first call on each device looks up the array's device address (with
- *   that device current) and keeps it; make that first call before any
- *   stream capture.  Every call shares the array, so calls that may overlap
- *   on the GPU (other streams, other threads) race: issue them in one stream
- *   order.  Each call clears the parts of the array that must start at zero. */
+ *   that device current) and keeps it for as long as the device's context
+ *   lives; make that first call before any stream capture.  A
+ *   cudaDeviceReset ends the context, and with it the array: the next call
+ *   sees a new context and looks the address up again, so it, too, belongs
+ *   before any capture.  Every call shares the array, so calls that may
+ *   overlap on the GPU (other streams, other threads) race: issue them in one
+ *   stream order.  Each call clears the parts of the array that must start
+ *   at zero.  Validation is averis_split_quant's (the same codes for the same
+ *   bad arguments), and a host without an sm_100 device gets
+ *   AVR_ERR_NO_DEVICE. */
 avr_status averis_split_quant_noalloc(const void* X, avr_dtype xt, int64_t l, int64_t K,
                                       avr_round rm, uint64_t seed, uint64_t offset, int grad,
                                       float* mu, const avr_nvfp4* mu_q, const avr_nvfp4* xr_q,

@@ -55,6 +55,7 @@ _SIGS = {
     "averis_workspace_size": (_c_size, [_c_i64, _c_i64, _c_i64]),
     "averis_workspace_init": (_c_int, [_c_ptr, _c_size, _c_ptr]),
     "averis_check_status": (_c_int, [_c_ptr, _c_ptr]),
+    "averis_set_wait_limit": (_c_int, [_c_ptr, _c_size, _c_u64, _c_ptr]),
     "averis_status_string": (ctypes.c_char_p, [_c_int]),
     "averis_split_quant": (_c_int, [_c_ptr, _c_int, _c_i64, _c_i64, _c_int, _c_u64, _c_u64, _c_int,
                                     _c_ptr, ctypes.POINTER(avr_nvfp4), ctypes.POINTER(avr_nvfp4),
@@ -214,6 +215,12 @@ def averis_workspace_init(ws, stream=None):
 def averis_check_status(ws, stream=None):
     """Synchronize and return the latched device status (0 = ok)."""
     return int(load().averis_check_status(_ptr(ws), _stream(stream)))
+
+
+def averis_set_wait_limit(ws, limit_ns, stream=None):
+    """Bound (ns) of the waits on other CTAs; 0 restores the default 2 s."""
+    _check(load().averis_set_wait_limit(_ptr(ws), ws.numel(), int(limit_ns), _stream(stream)),
+           "averis_set_wait_limit")
 
 
 def averis_split_quant(X, rm, seed, offset, grad, mu, mu_q, xr_q, xr_debug, ws, stream=None):

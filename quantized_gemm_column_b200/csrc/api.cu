@@ -92,6 +92,19 @@ bool make_tensor_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType 
   return r == CUDA_SUCCESS;
 }
 
+bool make_tensor_map_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, const uint64_t dims[3],
+                        const uint64_t strides[2], const uint32_t box[3]) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+  cuuint64_t st[2] = {strides[0], strides[1]};
+  cuuint32_t b[3] = {box[0], box[1], box[2]};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, dtype, 3, const_cast<void*>(base), d, st, b, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 cudaError_t set_max_dynamic_smem(const void* func, size_t bytes) {
   static std::mutex mu;
   static std::map<std::pair<int, const void*>, size_t> done;   // largest size set so far
@@ -134,15 +147,7 @@ int sm_count() {
 // ---------------------------------------------------------------------------
 // validation helpers
 // ---------------------------------------------------------------------------
-static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-static bool dtype_ok(avr_dtype t) { return t == AVR_F32 || t == AVR_BF16; }
-static bool round_ok(avr_round r) { return r == AVR_RNE || r == AVR_SR; }
-constexpr int64_t kMaxDim = (int64_t{1} << 31) - 1;
-static bool k_ok(int64_t K) { return K > 0 && K % 64 == 0 && K <= int64_t{kColTile} * kMaxColTiles; }
-static bool l_ok(int64_t l) { return l >= 0 && l <= kMaxDim; }
-static bool n_ok(int64_t N) { return N > 0 && N % 64 == 0 && N <= kMaxDim; }
-
-static avr_status device_ok() {
+avr_status device_ok() {
   int dev = 0, major = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return AVR_ERR_NO_DEVICE;
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
@@ -150,31 +155,13 @@ static avr_status device_ok() {
   return major == 10 ? AVR_OK : AVR_ERR_NO_DEVICE;
 }
 
-static avr_status check_nvfp4(const avr_nvfp4* t, int64_t rows, int64_t K) {
+avr_status check_nvfp4(const avr_nvfp4* t, int64_t rows, int64_t K) {
   if (!t || !t->codes || !t->scales || !t->g_dec) return AVR_ERR_INVALID_ARG;
   if (t->rows != rows || t->K != K) return AVR_ERR_INVALID_ARG;
   if (!aligned16(t->codes) || !aligned16(t->scales) || (reinterpret_cast<uintptr_t>(t->g_dec) & 3u))
     return AVR_ERR_MISALIGNED;
   return AVR_OK;
 }
-
-static avr_status cuda_status(cudaError_t e) { return e == cudaSuccess ? AVR_OK : AVR_ERR_CUDA; }
-
-#define AVR_TRY(expr)                  \
-  do {                                 \
-    avr_status st_ = (expr);           \
-    if (st_ != AVR_OK) return st_;     \
-  } while (0)
-
-struct Ws {
-  char* base;
-  WsLayout lay;
-  uint32_t* status() const { return reinterpret_cast<uint32_t*>(base + lay.status); }
-  float* slot_xr() const { return reinterpret_cast<float*>(base + lay.slots); }
-  float* slot_mu() const { return slot_xr() + kMaxColTiles; }
-  template <typename T>
-  T* at(size_t off) const { return reinterpret_cast<T*>(base + off); }
-};
 
 static avr_status make_ws(void* ws, size_t ws_bytes, int64_t l, int64_t K, int64_t N, Ws* out) {
   if (!ws) return AVR_ERR_INVALID_ARG;
@@ -188,11 +175,10 @@ static avr_status make_ws(void* ws, size_t ws_bytes, int64_t l, int64_t K, int64
 static int n_tiles(int64_t K) { return static_cast<int>((K + kColTile - 1) / kColTile); }
 
 // K1 + K2 (+ mean quantizer and rank-one row when mu_q / w are given)
-static avr_status split_chain(const void* X, avr_dtype xt, int64_t l, int64_t K, int split,
-                              avr_round rm, uint64_t seed, uint64_t offset, uint32_t tag,
-                              uint32_t tag_mu, float* mu_buf, const avr_nvfp4* mu_q,
-                              const avr_nvfp4* xr_q, float* xr_debug, const avr_nvfp4* w,
-                              float* bias, const Ws& ws, cudaStream_t s, bool fused = false) {
+avr_status split_chain(const void* X, avr_dtype xt, int64_t l, int64_t K, int split, avr_round rm,
+                       uint64_t seed, uint64_t offset, uint32_t tag, uint32_t tag_mu, float* mu_buf,
+                       const avr_nvfp4* mu_q, const avr_nvfp4* xr_q, float* xr_debug, const avr_nvfp4* w,
+                       float* bias, const Ws& ws, cudaStream_t s, bool fused, bool pdl) {
   ColReduceArgs ca;
   ca.X = X;
   ca.xt = xt;
@@ -234,9 +220,9 @@ static avr_status split_chain(const void* X, avr_dtype xt, int64_t l, int64_t K,
     qa.n_out = w->rows;
     qa.bias = bias;
   }
-  if (fused) return cuda_status(launch_split_fused(ca, qa, s, true));
-  AVR_TRY(cuda_status(launch_colreduce(ca, s, true)));
-  return cuda_status(launch_quant(qa, s, true));
+  if (fused) return cuda_status(launch_split_fused(ca, qa, s, pdl));
+  AVR_TRY(cuda_status(launch_colreduce(ca, s, pdl)));
+  return cuda_status(launch_quant(qa, s, pdl));
 }
 
 // K1 + K2 along the tokens (+ mean quantizer when mu_q is given), for the
@@ -306,6 +292,9 @@ static avr_status gemm(const avr_nvfp4* a, const avr_nvfp4* b, const float* bias
 
 using namespace avr;
 
+// one 64-bit word written in stream order (a launch, so it can be captured)
+__global__ void set_word64_kernel(uint64_t* dst, uint64_t value) { *dst = value; }
+
 extern "C" {
 
 size_t avr_nvfp4_scales_bytes(int64_t rows, int64_t K) {
@@ -321,6 +310,16 @@ size_t averis_workspace_size(int64_t l, int64_t K, int64_t N) {
 avr_status averis_workspace_init(void* ws, size_t ws_bytes, avr_stream stream) {
   if (!ws) return AVR_ERR_INVALID_ARG;
   return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, stream));
+}
+
+avr_status averis_set_wait_limit(void* ws, size_t ws_bytes, uint64_t limit_ns, avr_stream stream) {
+  if (!ws) return AVR_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return AVR_ERR_MISALIGNED;
+  if (ws_bytes < WsLayout{}.tickets) return AVR_ERR_WORKSPACE_TOO_SMALL;
+  AVR_TRY(device_ok());
+  set_word64_kernel<<<1, 1, 0, stream>>>(reinterpret_cast<uint64_t*>(static_cast<char*>(ws) + kWaitLimitOffset),
+                                         limit_ns);
+  return cuda_status(cudaGetLastError());
 }
 
 avr_status averis_check_status(void* ws, avr_stream stream) {

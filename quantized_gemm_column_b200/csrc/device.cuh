@@ -86,15 +86,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete.  Returns false (and
-// records a timeout in *status) if it has not completed within kWaitLimitNs.
 // Grid-wide barrier for a grid whose CTAs are all resident at once.  Thread 0
 // of each CTA arrives on *count (acquire-release at GPU scope, after a CTA
 // barrier, so it publishes every thread's prior writes); the last of n
-// arrivals resets *count and advances *gen, which the others poll with a
-// bounded wait.  *count is back at 0 after every completed barrier.  Returns
-// false (and records AVR_ERR_DEVICE_TIMEOUT) if the other CTAs never came.
-__device__ __forceinline__ bool grid_barrier(uint32_t* count, uint32_t* gen, uint32_t n, uint32_t* status) {
+// arrivals resets *count and advances *gen, which the others poll, reading
+// the clock after every poll, for at most limit_ns (0: kWaitLimitNs).  *count
+// is back at 0 after every completed barrier.  Returns false (and records
+// AVR_ERR_DEVICE_TIMEOUT) if the other CTAs did not come in time; *count is
+// then left part-way and the caller's status block must be cleared before
+// the next barrier.
+__device__ __forceinline__ bool grid_barrier(uint32_t* count, uint32_t* gen, uint32_t n, uint32_t* status,
+                                             uint64_t limit_ns) {
+  const uint64_t limit = limit_ns != 0 ? limit_ns : kWaitLimitNs;
   __shared__ uint32_t s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -106,11 +109,11 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* count, uint32_t* gen, uin
       asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(gen) : "memory");
     } else {
       const uint64_t t0 = globaltimer_ns();
-      uint32_t spins = 0, g;
+      uint32_t g;
       for (;;) {
         asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(gen) : "memory");
         if (g != g0) break;
-        if (((++spins) & 255u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit) {   // one clock read per poll: a poll is an L2 round trip
           raise_status(status, AVR_ERR_DEVICE_TIMEOUT);
           ok = 0u;
           break;
@@ -123,6 +126,8 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* count, uint32_t* gen, uin
   return s_ok != 0u;
 }
 
+// Wait for the phase with the given parity to complete.  Returns false (and
+// records a timeout in *status) if it has not completed within kWaitLimitNs.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
   if (mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer_ns();
@@ -175,8 +180,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-
-
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x, int32_t y,
+                                            int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+        "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -1,0 +1,603 @@
+// K3 on CTA pairs: the block-scaled FP4 GEMM with 2-CTA tcgen05 MMAs, for
+// bf16 output.
+//
+// Y = 1 (mu_bar W_bar) + X_bar_R W_bar (Lighthouse review of "The Curse and
+// Blessing of Mean Bias in FP4-Quantized LLM Training", section 二 "Averis
+// 方法"): the product X_bar_R W_bar on E2M1 operands with E4M3 per-16 scales,
+// the row mu_bar W_bar added to every output row as a bias:
+//   Y[i, j] = g_dec(A) g_dec(B) * acc[i, j] + bias[j].
+//
+// Why pairs.  A 128 x 256 tile of one CTA needs 12 KB of operands (A 4 KB,
+// B 8 KB) per 64-deep k-block, 48 KB per 256-deep stage plus scales, and one
+// SM brings in about 70 bytes per clock from L2: longer than the 73 ns the
+// k-block's MMA takes, and with three stages in shared memory the load
+// latency (about 0.8 us per stage) is not covered either.  Two CTAs on two
+// SMs of a cluster share one 256 x 256 tile: each holds its 128 rows of A
+// and half (128 rows) of B, and the MMA issued by the first CTA
+// (tcgen05.mma.cta_group::2, M 256, N 256, K 64) reads A from each CTA's own
+// shared memory and B from both.  Each SM then loads 8 KB per k-block, a
+// stage is 38 KB with scales, and four stages fit.
+//
+// Roles (both CTAs have the same warps; CTA rank 0 of the pair leads):
+//   warp 0     : tensor-memory allocation (cta_group::2, in both CTAs); in
+//                the leading CTA one thread issues the pair's MMAs;
+//   warps 1..4 : TMA producers in both CTAs, one operand each (A rows, B
+//                rows, A's scale atoms, B's scale atoms for all 256 columns
+//                plus the resident ones).  Every copy completes on the
+//                leading CTA's barrier, whose producers expect the bytes of
+//                both CTAs;
+//   warp 5     : in the leading CTA, the scale copier (tcgen05.cp
+//                cta_group::2: each CTA's atoms into its own tensor memory);
+//   warps 6..13: epilogue in both CTAs, each over its own 128 x 256
+//                accumulator: the bias row staged in shared memory,
+//                tcgen05.ld, alpha * acc + bias, bf16, TMA store.
+// The leading CTA's MMA commits signal both CTAs' barriers (multicast
+// commit); the second CTA's epilogue hands the accumulator back through a
+// remote arrive on the leading CTA's barrier.  No TMA load is multicast.
+//
+// B's scales of the first full stages (up to kResMaxStages) stay resident in
+// tensor memory while a pair works on one column block, as in the one-CTA
+// kernel.
+#include <map>
+#include <mutex>
+
+#include "device.cuh"
+#include "internal.h"
+
+namespace avr {
+
+namespace {
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// the shared::cluster address of the same shared-memory location in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// arrive on an mbarrier given by its shared::cluster address (possibly another CTA's)
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// TMA 2-D load into this CTA's shared memory completing on the barrier at a
+// shared::cluster address in either CTA of the pair
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int32_t x,
+                                                 int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int32_t x,
+                                                 int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+               ::"r"(smem_u32(dst_smem)), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// arrive once on *bar (this CTA) when the pair operations this thread issued have completed
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               ::"r"(smem_u32(bar)) : "memory");
+}
+// ... on the barrier at the same offset in both CTAs of the pair
+__device__ __forceinline__ void tc_commit_pair_both(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+               ::"r"(smem_u32(bar)), "h"(static_cast<uint16_t>(3)) : "memory");
+}
+__device__ __forceinline__ void mma_nvf4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
+      "}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+__device__ __forceinline__ void tc_cp_32x128b_warpx4_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+}  // namespace
+
+struct Gemm2Cfg {
+  static constexpr int kBM = 128;                          // rows per CTA (256 per pair)
+  static constexpr int kBN = 256;                          // columns per tile
+  static constexpr int kBNHalf = kBN / 2;                  // B rows per CTA
+  static constexpr int kStageK = 256;
+  static constexpr int kRowBytes = kStageK / 2;
+  static constexpr int kStages = 4;
+  static constexpr int kKbPerStage = kStageK / 64;
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kFirstEpiWarp = 6;
+  static constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
+  static constexpr uint32_t kSbo = 8 * kRowBytes;
+  static constexpr int kABytes = kBM * kRowBytes;          // 16 KB
+  static constexpr int kBBytes = kBNHalf * kRowBytes;      // 16 KB
+  static constexpr int kSfaBytes = kKbPerStage * 512;      // 2 KB
+  static constexpr int kSfbBytes = 2 * kKbPerStage * 512;  // 4 KB: all 256 columns
+  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  static constexpr int kStageOutBytes = kBM * kBN * 2 / 2; // 32 KB: half the bf16 tile per round
+  // tensor memory (the same columns in both CTAs)
+  static constexpr int kAccCols = kBN;
+  static constexpr int kSfaCols = kKbPerStage * 4;
+  static constexpr int kSfbKbCols = kBN / 32;
+  static constexpr int kSfbCols = kKbPerStage * kSfbKbCols;
+  static constexpr int kSlots = 2;
+  static constexpr int kSlotCols = kSfaCols + kSfbCols;
+  static constexpr int kSlotCol = kAccCols;
+  static constexpr int kResCol = kSlotCol + kSlots * kSlotCols;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kResMaxStages = (kTmemCols - kResCol) / kSfbCols;   // 5
+  static constexpr int kResBytes = kResMaxStages * kSfbBytes;
+  // shared memory
+  static constexpr int kOutOffset = kStages * kStageBytes;
+  static constexpr int kResOffset = kOutOffset + kStageOutBytes;
+  static constexpr int kBiasOffset = kResOffset + kResBytes;
+  static constexpr int kBarOffset = kBiasOffset + kBN * 4;
+  static constexpr int kSmemBytes = kBarOffset + 256;
+  static_assert(kResMaxStages >= 1, "tensor memory budget");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+  // instruction descriptor: E2M1 A and B, UE4M3 scales, K-major, N >> 3 at
+  // bit 17, M >> 4 at bit 24 (M = 256 for the pair)
+  static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kBN >> 3) << 17) |
+                                     (static_cast<uint32_t>((2 * kBM) >> 4) << 24);
+};
+
+struct Gemm2Params {
+  int64_t M, N, K;
+  int tiles_m, num_tiles;   // pair tiles of 256 x 256, M fastest
+  int res_stages;
+  const float* gdec_a;
+  const float* gdec_b;
+  const float* bias;
+  uint32_t* status;
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 1)
+    gemm2_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                       const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
+                       const __grid_constant__ CUtensorMap map_sfb_res, const __grid_constant__ CUtensorMap map_y,
+                       const Gemm2Params p) {
+  using Cfg = Gemm2Cfg;
+  constexpr int kEpiThreads = 32 * Cfg::kEpiWarps;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // the swizzled tiles need 1024-byte alignment; a CTA without it still takes
+  // part in the pair's cluster barriers and allocation, but does no work
+  const bool aligned = (smem_u32(smem_raw) & 1023u) == 0;
+  uint8_t* smem = smem_raw;
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + Cfg::kStages * Cfg::kABytes;
+  uint8_t* sSfa = sB + Cfg::kStages * Cfg::kBBytes;
+  uint8_t* sSfb = sSfa + Cfg::kStages * Cfg::kSfaBytes;
+  uint8_t* sOut = smem + Cfg::kOutOffset;
+  uint8_t* sRes = smem + Cfg::kResOffset;      // [2 row groups][stage][4 atoms]
+  float* bias_s = reinterpret_cast<float*>(smem + Cfg::kBiasOffset);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOffset);  // [kStages] (used in the leading CTA)
+  uint64_t* empty = full + Cfg::kStages;        // [kStages] both CTAs
+  uint64_t* sf_full = empty + Cfg::kStages;     // [kSlots] leading CTA
+  uint64_t* sf_empty = sf_full + Cfg::kSlots;   // [kSlots] leading CTA
+  uint64_t* acc_full = sf_empty + Cfg::kSlots;  // both CTAs
+  uint64_t* acc_empty = acc_full + 1;           // leading CTA: both epilogues arrive
+  uint64_t* res_load = acc_empty + 1;           // leading CTA: resident scales landed in both CTAs
+  uint64_t* res_cp = res_load + 1;              // both CTAs: resident scales copied
+  uint64_t* res_free = res_cp + 1;              // leading CTA: the MMAs of a column block are done
+  uint64_t* drained = res_free + 1;             // [2] leading CTA: MMA and copy threads drained
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool lead = rank == 0;
+  const int n_kst = static_cast<int>((p.K + Cfg::kStageK - 1) / Cfg::kStageK);
+  const int n_full = static_cast<int>(p.K / Cfg::kStageK);
+  const int tail_kb = static_cast<int>((p.K % Cfg::kStageK) / 64);
+  const int res_st = p.res_stages;
+
+  if (threadIdx.x == 0) {
+    if (!aligned) raise_status(p.status, AVR_ERR_MISALIGNED);
+    prefetch_tensormap(&map_a);
+    prefetch_tensormap(&map_b);
+    prefetch_tensormap(&map_sfa);
+    prefetch_tensormap(&map_sfb);
+    prefetch_tensormap(&map_sfb_res);
+    prefetch_tensormap(&map_y);
+    for (int s = 0; s < Cfg::kStages; ++s) {
+      mbar_init(&full[s], 4);                   // the leading CTA's four producers
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < Cfg::kSlots; ++s) {
+      mbar_init(&sf_full[s], 1);
+      mbar_init(&sf_empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 2 * Cfg::kEpiWarps);   // every epilogue warp of both CTAs
+    mbar_init(res_load, 1);
+    mbar_init(res_cp, 1);
+    mbar_init(res_free, 1);
+    mbar_init(&drained[0], 1);
+    mbar_init(&drained[1], 1);
+    fence_mbarrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc_pair(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync_all();          // barriers initialised and tensor memory allocated in both CTAs
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait_prior_grid();
+  pdl_allow_next_grid();
+
+  // the pair's run of tiles: pair q of G / 2 takes tiles [first, first + count)
+  const int pairs = static_cast<int>(gridDim.x) / 2, pair = static_cast<int>(blockIdx.x) / 2;
+  int first = 0, count = 0;
+  {
+    const int q = p.num_tiles / pairs, r = p.num_tiles % pairs;
+    first = pair * q + (pair < r ? pair : r);
+    count = aligned ? q + (pair < r ? 1 : 0) : 0;
+  }
+  auto new_block = [&](int i) { return i == 0 || (first + i) / p.tiles_m != (first + i - 1) / p.tiles_m; };
+  auto last_of_block = [&](int i) { return i + 1 == count || (first + i + 1) / p.tiles_m != (first + i) / p.tiles_m; };
+  // barriers of the leading CTA, as shared::cluster addresses
+  const uint32_t full_lead = mapa_shared(smem_u32(full), 0);
+  const uint32_t res_load_lead = mapa_shared(smem_u32(res_load), 0);
+  const uint32_t acc_empty_lead = mapa_shared(smem_u32(acc_empty), 0);
+
+  if (warp >= 1 && warp <= 4) {
+    if (lane == 0) {
+      // ---------------- producers: warp 1 A, 2 B, 3 A's scales, 4 B's scales (+ resident) ----------------
+      const int role = warp - 1;
+      uint32_t st = 0, ph = 0;
+      int it = 0, res_uses = 0;
+      bool ok = true;
+      for (int i = 0; i < count && ok; ++i) {
+        const int tile = first + i;
+        const int32_t m0 = (tile % p.tiles_m) * (2 * Cfg::kBM) + static_cast<int32_t>(rank) * Cfg::kBM;
+        const int32_t n0 = (tile / p.tiles_m) * Cfg::kBN;
+        if (role == 3 && res_st > 0 && new_block(i)) {
+          // both CTAs' resident buffers are free once the previous block's copies ran
+          if (res_uses >= 1 && !mbar_wait(res_cp, static_cast<uint32_t>(res_uses - 1) & 1u, p.status)) break;
+          ++res_uses;
+          if (lead) mbar_arrive_expect_tx(res_load, static_cast<uint32_t>(2 * res_st * Cfg::kSfbBytes));
+          tma_load_3d_pair(sRes, &map_sfb_res, res_load_lead, 0, 0, n0 / 128);
+        }
+        for (int ks = 0; ks < n_kst; ++ks, ++it) {
+          if (it >= Cfg::kStages && !mbar_wait(&empty[st], ph ^ 1u, p.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t bar = full_lead + static_cast<uint32_t>(st * 8);
+          if (role == 0) {
+            if (lead) mbar_arrive_expect_tx(&full[st], 2 * Cfg::kABytes);
+            tma_load_2d_pair(sA + st * Cfg::kABytes, &map_a, bar, ks * Cfg::kRowBytes, m0);
+          } else if (role == 1) {
+            if (lead) mbar_arrive_expect_tx(&full[st], 2 * Cfg::kBBytes);
+            tma_load_2d_pair(sB + st * Cfg::kBBytes, &map_b, bar, ks * Cfg::kRowBytes,
+                             n0 + static_cast<int32_t>(rank) * Cfg::kBNHalf);
+          } else if (role == 2) {
+            if (lead) mbar_arrive_expect_tx(&full[st], 2 * Cfg::kSfaBytes);
+            tma_load_2d_pair(sSfa + st * Cfg::kSfaBytes, &map_sfa, bar, ks * 256, m0 / 128);
+          } else if (ks >= res_st) {
+            if (lead) mbar_arrive_expect_tx(&full[st], 2 * Cfg::kSfbBytes);
+            tma_load_2d_pair(sSfb + st * Cfg::kSfbBytes, &map_sfb, bar, ks * 256, n0 / 128);
+          } else if (lead) {
+            mbar_arrive(&full[st]);               // this stage's B scales are resident
+          }
+          if (++st == Cfg::kStages) {
+            st = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 5) {
+    if (lead && lane == 0) {
+      // ---------------- scale copier (leading CTA; each copy fills both CTAs) ----------------
+      uint32_t st = 0, ph = 0, sl = 0, sph = 0;
+      int it = 0, res_uses = 0;
+      bool ok = true;
+      const uint64_t res_d = smem_desc(smem_u32(sRes), 0, 128, kLayoutSwizzleNone);
+      for (int i = 0; i < count && ok; ++i) {
+        if (res_st > 0 && new_block(i)) {
+          if (res_uses >= 1 && !mbar_wait_poll(res_free, static_cast<uint32_t>(res_uses - 1) & 1u, p.status)) break;
+          if (!mbar_wait_poll(res_load, static_cast<uint32_t>(res_uses) & 1u, p.status)) break;
+          ++res_uses;
+          tc_fence_after();
+          for (int ks = 0; ks < res_st; ++ks)
+#pragma unroll
+            for (int kb = 0; kb < Cfg::kKbPerStage; ++kb)
+#pragma unroll
+              for (int g = 0; g < 2; ++g)
+                tc_cp_32x128b_warpx4_pair(tmem + Cfg::kResCol + Cfg::kSfbKbCols * (ks * Cfg::kKbPerStage + kb) + 4 * g,
+                                          res_d + static_cast<uint64_t>(32 * ((g * res_st + ks) * Cfg::kKbPerStage + kb)));
+          tc_commit_pair_both(res_cp);
+        }
+        for (int ks = 0; ks < n_kst; ++ks, ++it) {
+          if (!mbar_wait_poll(&full[st], ph, p.status)) {
+            ok = false;
+            break;
+          }
+          if (it >= Cfg::kSlots && !mbar_wait_poll(&sf_empty[sl], sph ^ 1u, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sfa_t = tmem + Cfg::kSlotCol + sl * Cfg::kSlotCols;
+          const uint32_t sfb_t = sfa_t + Cfg::kSfaCols;
+          const uint64_t sfa_d = smem_desc(smem_u32(sSfa + st * Cfg::kSfaBytes), 0, 128, kLayoutSwizzleNone);
+          const uint64_t sfb_d = smem_desc(smem_u32(sSfb + st * Cfg::kSfbBytes), 0, 128, kLayoutSwizzleNone);
+          const bool sfb = ks >= res_st;
+          const int nkb = ks < n_full ? Cfg::kKbPerStage : tail_kb;
+          for (int kb = 0; kb < nkb; ++kb) {
+            tc_cp_32x128b_warpx4_pair(sfa_t + 4 * kb, sfa_d + static_cast<uint64_t>(32 * kb));
+            if (sfb) {
+#pragma unroll
+              for (int g = 0; g < 2; ++g)
+                tc_cp_32x128b_warpx4_pair(sfb_t + Cfg::kSfbKbCols * kb + 4 * g,
+                                          sfb_d + static_cast<uint64_t>(32 * (g * Cfg::kKbPerStage + kb)));
+            }
+          }
+          tc_commit_pair(&sf_full[sl]);
+          if (++st == Cfg::kStages) {
+            st = 0;
+            ph ^= 1u;
+          }
+          if (++sl == Cfg::kSlots) {
+            sl = 0;
+            sph ^= 1u;
+          }
+        }
+      }
+      tc_commit_pair(&drained[1]);
+      mbar_wait(&drained[1], 0, p.status);
+    }
+  } else if (warp == 0) {
+    if (lead && lane == 0) {
+      // ---------------- MMA issuer (leading CTA) ----------------
+      uint32_t st = 0, ph = 0, sl = 0, sph = 0;
+      int res_uses = 0;
+      bool ok = true;
+      for (int i = 0; i < count && ok; ++i) {
+        if (res_st > 0 && new_block(i)) {
+          if (!mbar_wait_poll(res_cp, static_cast<uint32_t>(res_uses) & 1u, p.status)) break;
+          ++res_uses;
+        }
+        for (int ks = 0; ks < n_kst; ++ks) {
+          if (!mbar_wait_poll(&sf_full[sl], sph, p.status) || !mbar_wait_poll(&full[st], ph, p.status)) {
+            ok = false;
+            break;
+          }
+          if (ks == 0 && i >= 1 && !mbar_wait_poll(acc_empty, static_cast<uint32_t>(i - 1) & 1u, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sfa_t = tmem + Cfg::kSlotCol + sl * Cfg::kSlotCols;
+          const uint32_t sfb_t = ks < res_st ? tmem + Cfg::kResCol + Cfg::kSfbKbCols * (ks * Cfg::kKbPerStage)
+                                             : sfa_t + Cfg::kSfaCols;
+          const uint64_t a0 = smem_desc(smem_u32(sA + st * Cfg::kABytes), 16, Cfg::kSbo, kLayoutSwizzle128B);
+          const uint64_t b0 = smem_desc(smem_u32(sB + st * Cfg::kBBytes), 16, Cfg::kSbo, kLayoutSwizzle128B);
+          if (ks < n_full) {
+#pragma unroll
+            for (int kb = 0; kb < Cfg::kKbPerStage; ++kb)
+              mma_nvf4_pair(tmem, a0 + static_cast<uint64_t>(2 * kb), b0 + static_cast<uint64_t>(2 * kb), Cfg::kIdesc,
+                            sfa_t + 4 * kb, sfb_t + Cfg::kSfbKbCols * kb, (ks > 0 || kb > 0) ? 1u : 0u);
+          } else {
+            for (int kb = 0; kb < tail_kb; ++kb)
+              mma_nvf4_pair(tmem, a0 + static_cast<uint64_t>(2 * kb), b0 + static_cast<uint64_t>(2 * kb), Cfg::kIdesc,
+                            sfa_t + 4 * kb, sfb_t + Cfg::kSfbKbCols * kb, (ks > 0 || kb > 0) ? 1u : 0u);
+          }
+          tc_commit_pair_both(&empty[st]);        // both CTAs' producers may refill the stage
+          tc_commit_pair(&sf_empty[sl]);
+          if (++st == Cfg::kStages) {
+            st = 0;
+            ph ^= 1u;
+          }
+          if (++sl == Cfg::kSlots) {
+            sl = 0;
+            sph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_both(acc_full);
+        if (res_st > 0 && last_of_block(i)) tc_commit_pair(res_free);
+      }
+      tc_commit_pair(&drained[0]);
+      mbar_wait(&drained[0], 0, p.status);
+    }
+  } else {
+    // ---------------- epilogue (both CTAs, own rows) ----------------
+    const int ew = warp - Cfg::kFirstEpiWarp;
+    const int q = warp & 3;                    // lane quarter of tensor memory this warp may read
+    const int h = ew / 4;                      // which 128-column half
+    const int r = 32 * q + lane;               // row of this CTA's 128
+    const bool store_thr = (ew == 0 && lane == 0);
+    const float alpha = __ldg(p.gdec_a) * __ldg(p.gdec_b);
+    for (int i = 0; i < count; ++i) {
+      const int tile = first + i;
+      const int64_t m0 = static_cast<int64_t>(tile % p.tiles_m) * (2 * Cfg::kBM) + static_cast<int64_t>(rank) * Cfg::kBM;
+      const int64_t n0 = static_cast<int64_t>(tile / p.tiles_m) * Cfg::kBN;
+      if (store_thr) bulk_wait_group_read<0>();
+      named_barrier(1, kEpiThreads);
+      {
+        const int64_t col = n0 + ew * 32 + lane;
+        bias_s[ew * 32 + lane] = (p.bias != nullptr && col < p.N) ? __ldg(p.bias + col) : 0.0f;
+      }
+      uint32_t okw = 0;
+      if (lane == 0) okw = mbar_wait(acc_full, static_cast<uint32_t>(i) & 1u, p.status) ? 1u : 0u;
+      const bool ok = __shfl_sync(0xFFFFFFFFu, okw, 0) != 0;
+      if (named_barrier_or(1, kEpiThreads, !ok)) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem + (static_cast<uint32_t>(32 * q) << 16);
+      auto pack_bf16 = [&](int c, const uint32_t (&v)[32], uint32_t (&w)[16]) {
+        const float* b = bias_s + 32 * (4 * h + c);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const __nv_bfloat162 pr = __floats2bfloat162_rn(fmaf(alpha, __uint_as_float(v[2 * k]), b[2 * k]),
+                                                          fmaf(alpha, __uint_as_float(v[2 * k + 1]), b[2 * k + 1]));
+          w[k] = *reinterpret_cast<const uint32_t*>(&pr);
+        }
+      };
+      auto stage_bf16 = [&](int c, const uint32_t (&w)[16]) {
+        uint8_t* box = sOut + h * (Cfg::kBM * 128);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int piece = ((c & 1) * 4 + u) ^ (r & 7);
+          *reinterpret_cast<uint4*>(box + r * 128 + piece * 16) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        }
+      };
+      auto store_round = [&](int first_col) {
+        fence_proxy_async_smem();
+        named_barrier(1, kEpiThreads);
+        if (store_thr) {
+          if (m0 < p.M) {
+#pragma unroll
+            for (int bx = 0; bx < 2; ++bx) {
+              const int64_t col = n0 + first_col + bx * 128;
+              if (col < p.N)
+                tma_store_2d(&map_y, sOut + bx * (Cfg::kBM * 128), static_cast<int32_t>(col), static_cast<int32_t>(m0));
+            }
+          }
+          bulk_commit_group();
+        }
+      };
+      uint32_t v0[32], v1[32];
+      tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(32 * (4 * h + 0)), v0);
+      tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(32 * (4 * h + 1)), v1);
+      tmem_ld_wait();
+      {
+        uint32_t w[16];
+        pack_bf16(0, v0, w);
+        stage_bf16(0, w);
+        pack_bf16(1, v1, w);
+        stage_bf16(1, w);
+      }
+      tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(32 * (4 * h + 2)), v0);
+      tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(32 * (4 * h + 3)), v1);
+      tmem_ld_wait();
+      // the accumulator goes back to the leading CTA's MMA thread
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty_lead);
+      uint32_t w2[16], w3[16];
+      pack_bf16(2, v0, w2);
+      pack_bf16(3, v1, w3);
+      store_round(0);
+      if (store_thr) bulk_wait_group_read<0>();
+      named_barrier(1, kEpiThreads);
+      stage_bf16(2, w2);
+      stage_bf16(3, w3);
+      store_round(64);
+    }
+    if (store_thr) bulk_wait_group_all();
+  }
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync_all();          // no CTA leaves while its pair may still signal its barriers
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, Cfg::kTmemCols);
+  }
+}
+
+// Clusters of two CTAs of gemm2_nvfp4_kernel that can be resident at once on
+// the current device (cached per device).
+static int resident_pairs() {
+  static std::mutex mu;
+  static std::map<int, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  std::lock_guard<std::mutex> g(mu);
+  auto it = cache.find(dev);
+  if (it != cache.end()) return it->second;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * (sm_count() / 2)));
+  cfg.blockDim = dim3(Gemm2Cfg::kThreads);
+  cfg.dynamicSmemBytes = Gemm2Cfg::kSmemBytes;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(gemm2_nvfp4_kernel), &cfg) != cudaSuccess || n < 1)
+    n = sm_count() / 2;
+  cache[dev] = n;
+  return n;
+}
+
+// The pair kernel serves dense bf16 outputs; its tiles are 256 rows x 256 columns.
+bool gemm_pair_applies(const GemmArgs& a) {
+  return a.yt == AVR_BF16 && a.block_expert == nullptr && a.row_scale == nullptr && a.groups == 1;
+}
+
+cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s, bool pdl) {
+  using Cfg = Gemm2Cfg;
+  constexpr CUtensorMapSwizzle kOpSwizzle = CU_TENSOR_MAP_SWIZZLE_128B;
+  CUtensorMap ma, mb, msa, msb, my;
+  if (!make_tensor_map_2d(&ma, a.a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(a.M),
+                          static_cast<uint64_t>(a.K / 2), Cfg::kBM, Cfg::kRowBytes, kOpSwizzle))
+    return cudaErrorInvalidValue;
+  if (!make_tensor_map_2d(&mb, a.b_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(a.N),
+                          static_cast<uint64_t>(a.K / 2), Cfg::kBNHalf, Cfg::kRowBytes, kOpSwizzle))
+    return cudaErrorInvalidValue;
+  const uint64_t sf_cols = static_cast<uint64_t>(a.K / 64) * 64;
+  if (!make_tensor_map_2d(&msa, a.a_scales, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, static_cast<uint64_t>((a.M + 127) / 128),
+                          sf_cols, 1, 256, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  const uint64_t b_groups = static_cast<uint64_t>((a.N + 127) / 128);
+  if (!make_tensor_map_2d(&msb, a.b_scales, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, b_groups, sf_cols, 2, 256,
+                          CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  const int64_t n_full = a.K / Cfg::kStageK;
+  const int res_stages = static_cast<int>(min64(n_full, Cfg::kResMaxStages));
+  CUtensorMap msr = msb;
+  if (res_stages > 0) {
+    const uint64_t dims[3] = {256, static_cast<uint64_t>(n_full), b_groups};
+    const uint64_t strides[2] = {2048, sf_cols * 8};
+    const uint32_t box[3] = {256, static_cast<uint32_t>(res_stages), 2};
+    if (!make_tensor_map_3d(&msr, a.b_scales, CU_TENSOR_MAP_DATA_TYPE_UINT64, dims, strides, box))
+      return cudaErrorInvalidValue;
+  }
+  if (!make_tensor_map_2d(&my, a.Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, static_cast<uint64_t>(a.M),
+                          static_cast<uint64_t>(a.N), Cfg::kBM, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  Gemm2Params p;
+  p.M = a.M;
+  p.N = a.N;
+  p.K = a.K;
+  p.tiles_m = static_cast<int>((a.M + 2 * Cfg::kBM - 1) / (2 * Cfg::kBM));
+  p.num_tiles = p.tiles_m * static_cast<int>((a.N + Cfg::kBN - 1) / Cfg::kBN);
+  p.res_stages = res_stages;
+  p.gdec_a = a.a_gdec;
+  p.gdec_b = a.b_gdec;
+  p.bias = a.bias;
+  p.status = a.status;
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm2_nvfp4_kernel), Cfg::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  // one pair per two SMs that can hold pairs at once: the run of tiles is
+  // split statically, so a pair that had to wait for another would double the time
+  const int max_pairs = resident_pairs();
+  const int pairs = p.num_tiles < max_pairs ? p.num_tiles : max_pairs;
+  return launch_ex(gemm2_nvfp4_kernel, dim3(2 * pairs), dim3(Cfg::kThreads), Cfg::kSmemBytes, s, pdl, ma, mb, msa,
+                   msb, msr, my, p);
+}
+
+}  // namespace avr

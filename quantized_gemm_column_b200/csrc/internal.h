@@ -19,6 +19,12 @@ constexpr int kStripCols = 512;      // columns per warp in the quantizer (16 pe
 // per-column-tile tickets sit at fixed offsets whatever the sizes, so a
 // workspace can be reused across shapes; everything after them is scratch
 // that each call writes before it reads.
+// The first 256 bytes of a workspace are its status block: the status word
+// at 0, the one-kernel split's barrier counter and generation at 64 and 128,
+// and at kWaitLimitOffset the bound (uint64 ns, 0 = the default 2 s) of the
+// waits on other CTAs.
+constexpr size_t kWaitLimitOffset = 192;
+
 struct WsLayout {
   size_t status = 0;
   size_t tickets = 256;
@@ -221,6 +227,50 @@ struct GemmArgs {
   uint32_t* status;
 };
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, bool pdl);
+// the 2-CTA kernel (gemm2.cu): dense bf16 outputs, 256 x 256 tiles on CTA pairs
+bool gemm_pair_applies(const GemmArgs& a);
+cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s, bool pdl);
+
+// ---------------- host-side validation and the split chain (api.cu) ----------------
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool dtype_ok(avr_dtype t) { return t == AVR_F32 || t == AVR_BF16; }
+inline bool round_ok(avr_round r) { return r == AVR_RNE || r == AVR_SR; }
+constexpr int64_t kMaxDim = (int64_t{1} << 31) - 1;
+inline bool k_ok(int64_t K) { return K > 0 && K % 64 == 0 && K <= int64_t{kColTile} * kMaxColTiles; }
+inline bool l_ok(int64_t l) { return l >= 0 && l <= kMaxDim; }
+inline bool n_ok(int64_t N) { return N > 0 && N % 64 == 0 && N <= kMaxDim; }
+inline avr_status cuda_status(cudaError_t e) { return e == cudaSuccess ? AVR_OK : AVR_ERR_CUDA; }
+
+#define AVR_TRY(expr)                  \
+  do {                                 \
+    avr_status st_ = (expr);           \
+    if (st_ != AVR_OK) return st_;     \
+  } while (0)
+
+// AVR_OK when the current device is an sm_100 part, else AVR_ERR_NO_DEVICE
+avr_status device_ok();
+// an NVFP4 descriptor of `rows` x K: non-null parts, matching shape, codes and
+// scales 16-byte aligned, g_dec 4-byte aligned
+avr_status check_nvfp4(const avr_nvfp4* t, int64_t rows, int64_t K);
+
+// a workspace (or any scratch laid out like one) and its regions
+struct Ws {
+  char* base;
+  WsLayout lay;
+  uint32_t* status() const { return reinterpret_cast<uint32_t*>(base + lay.status); }
+  float* slot_xr() const { return reinterpret_cast<float*>(base + lay.slots); }
+  float* slot_mu() const { return slot_xr() + kMaxColTiles; }
+  template <typename T>
+  T* at(size_t off) const { return reinterpret_cast<T*>(base + off); }
+};
+
+// K1 + K2 on `ws` (+ mean quantizer and rank-one row when mu_q / w are
+// given); fused: the one-kernel split; pdl: chain the launches with
+// programmatic dependent launch
+avr_status split_chain(const void* X, avr_dtype xt, int64_t l, int64_t K, int split, avr_round rm,
+                       uint64_t seed, uint64_t offset, uint32_t tag, uint32_t tag_mu, float* mu_buf,
+                       const avr_nvfp4* mu_q, const avr_nvfp4* xr_q, float* xr_debug, const avr_nvfp4* w,
+                       float* bias, const Ws& ws, cudaStream_t s, bool fused = false, bool pdl = true);
 
 // ---------------- diagnostics ----------------
 cudaError_t launch_probe_convert(const float* in, uint8_t* e4m3, uint8_t* e2m1, int64_t n,
@@ -235,6 +285,11 @@ cudaError_t launch_probe_philox(uint64_t seed, uint64_t offset, uint32_t tag, in
 bool make_tensor_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
                         int elem_bytes, uint64_t rows, uint64_t cols, uint32_t box_rows,
                         uint32_t box_cols, CUtensorMapSwizzle swizzle);
+
+// 3-D tensor of elem-sized elements: dims[0] contiguous, byte strides of
+// dims 1 and 2; no swizzle.
+bool make_tensor_map_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, const uint64_t dims[3],
+                        const uint64_t strides[2], const uint32_t box[3]);
 
 // cudaFuncAttributeMaxDynamicSharedMemorySize for the current device (set
 // once per device and function).

@@ -14,8 +14,13 @@
 // library holds it (kNoAllocScratchBytes) until the process exits, and every
 // call shares it, so two calls that overlap on the GPU (for example on two
 // streams) race and must not be issued.  Host code cannot use the array's
-// name as a device address; the first call on each device looks the address
-// up with cudaGetSymbolAddress (with that device current) and reuses it.
+// name as a device address; the address is looked up with
+// cudaGetSymbolAddress (with the device current) on the first call in each
+// device context and reused while that context lives.  A cudaDeviceReset
+// ends the context and its module, so the next call looks the address up
+// again instead of writing through a stale one.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "internal.h"
@@ -26,19 +31,50 @@ constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;   // 4 MiB per device
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
+// The unique ID of the calling thread's current context (false if none is
+// current yet, or the driver lacks the call).
+static bool current_context_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 static avr_status noalloc_scratch(void** out) {
+  struct Entry {
+    unsigned long long ctx;
+    void* ptr;
+  };
   static std::mutex mu;
-  static void* ptr[256] = {};
+  static Entry cache[256] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return AVR_ERR_NO_DEVICE;
   if (dev < 0 || dev >= 256) return AVR_ERR_NO_DEVICE;
   std::lock_guard<std::mutex> g(mu);
-  if (ptr[dev] == nullptr) {
+  unsigned long long ctx = 0;
+  if (cache[dev].ptr == nullptr || !current_context_id(&ctx) || ctx != cache[dev].ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return AVR_ERR_CUDA;
-    ptr[dev] = p;
+    // the lookup made the device's context current, so its ID exists now
+    if (!current_context_id(&ctx)) return AVR_ERR_CUDA;
+    cache[dev].ctx = ctx;
+    cache[dev].ptr = p;
   }
-  *out = ptr[dev];
+  *out = cache[dev].ptr;
   return AVR_OK;
 }
 
@@ -57,75 +93,37 @@ extern "C" avr_status averis_split_quant_noalloc(const void* X, avr_dtype xt, in
                                                  int grad, float* mu, const avr_nvfp4* mu_q,
                                                  const avr_nvfp4* xr_q, float* xr_debug,
                                                  uint32_t* device_status, avr_stream stream) {
-  if (!(xt == AVR_F32 || xt == AVR_BF16) || !(rm == AVR_RNE || rm == AVR_SR)) return AVR_ERR_INVALID_ARG;
-  if (K <= 0 || K % 64 != 0 || K > int64_t{kColTile} * kMaxColTiles || l < 0 || l > INT32_MAX)
-    return AVR_ERR_UNSUPPORTED_SHAPE;
-  if (l == 0) return AVR_OK;
-  if (!X || !xr_q || !xr_q->codes || !xr_q->scales || !xr_q->g_dec) return AVR_ERR_INVALID_ARG;
-  if (xr_q->rows != l || xr_q->K != K) return AVR_ERR_INVALID_ARG;
-  if (mu_q && (!mu_q->codes || !mu_q->scales || !mu_q->g_dec || mu_q->rows != 1 || mu_q->K != K))
-    return AVR_ERR_INVALID_ARG;
-  auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-  if (!a16(X) || !a16(mu) || !a16(xr_debug) || !a16(xr_q->codes) || !a16(xr_q->scales) ||
-      (mu_q && (!a16(mu_q->codes) || !a16(mu_q->scales))) ||
+  // the same checks, in the same order, as averis_split_quant
+  if (!dtype_ok(xt) || !round_ok(rm)) return AVR_ERR_INVALID_ARG;
+  if (!k_ok(K) || !l_ok(l)) return AVR_ERR_UNSUPPORTED_SHAPE;
+  if (l == 0) return AVR_OK;   // no tokens: nothing is read or written
+  if (!X) return AVR_ERR_INVALID_ARG;
+  AVR_TRY(check_nvfp4(xr_q, l, K));
+  if (mu_q) AVR_TRY(check_nvfp4(mu_q, 1, K));
+  if (!aligned16(X) || !aligned16(mu) || !aligned16(xr_debug) ||
       (reinterpret_cast<uintptr_t>(device_status) & 3u))
     return AVR_ERR_MISALIGNED;
 
   // The reduce needs the status word, tickets, amax slots, chunk partials and
   // the mean: everything in the workspace layout before the mean's codes.
-  const WsLayout lay = ws_layout(l, K, 0);
-  if (lay.mu_codes > kNoAllocScratchBytes) return AVR_ERR_WORKSPACE_TOO_SMALL;
+  Ws w;
+  w.lay = ws_layout(l, K, 0);
+  if (w.lay.mu_codes > kNoAllocScratchBytes) return AVR_ERR_WORKSPACE_TOO_SMALL;
+  AVR_TRY(device_ok());
   void* scratch = nullptr;
-  avr_status st = noalloc_scratch(&scratch);
-  if (st != AVR_OK) return st;
-  char* base = static_cast<char*>(scratch);
+  AVR_TRY(noalloc_scratch(&scratch));
+  w.base = static_cast<char*>(scratch);
   cudaStream_t s = stream;
 
   // The array keeps the previous call's contents: the status word and the
   // tickets must start at zero (slots, partials and mean are written before
   // they are read).
-  if (cudaMemsetAsync(base, 0, lay.slots, s) != cudaSuccess) return AVR_ERR_CUDA;
-
-  float* mu_buf = mu ? mu : reinterpret_cast<float*>(base + lay.mu);
-  ColReduceArgs ca;
-  ca.X = X;
-  ca.xt = xt;
-  ca.l = l;
-  ca.K = K;
-  ca.split = 1;
-  ca.mu_out = mu_buf;
-  ca.energy = 0;
-  ca.ws = base;
-  ca.lay = &lay;
-  if (launch_colreduce(ca, s, false) != cudaSuccess) return AVR_ERR_CUDA;
-
-  QuantArgs qa = {};
-  qa.X = X;
-  qa.xt = xt;
-  qa.rows = l;
-  qa.K = K;
-  qa.mu = mu_buf;
-  qa.n_tiles = static_cast<int>((K + kColTile - 1) / kColTile);
-  qa.slot_xr = reinterpret_cast<float*>(base + lay.slots);
-  qa.codes = xr_q->codes;
-  qa.scales = xr_q->scales;
-  qa.g_dec = xr_q->g_dec;
-  qa.xr_debug = xr_debug;
-  qa.seed = seed;
-  qa.offset = offset;
-  qa.tag = grad ? 3u : 1u;
-  qa.sr = rm == AVR_SR;
-  qa.status = reinterpret_cast<uint32_t*>(base + lay.status);
-  qa.slot_mu = qa.slot_xr + kMaxColTiles;
-  qa.tag_mu = grad ? 4u : 2u;
-  if (mu_q) {
-    qa.mu_codes = mu_q->codes;
-    qa.mu_scales = mu_q->scales;
-    qa.mu_gdec = mu_q->g_dec;
-  }
-  if (launch_quant(qa, s, false) != cudaSuccess) return AVR_ERR_CUDA;
+  if (cudaMemsetAsync(w.base, 0, w.lay.slots, s) != cudaSuccess) return AVR_ERR_CUDA;
+  float* mu_buf = mu ? mu : w.at<float>(w.lay.mu);
+  AVR_TRY(split_chain(X, xt, l, K, 1, rm, seed, offset, grad ? 3u : 1u, grad ? 4u : 2u, mu_buf, mu_q, xr_q,
+                      xr_debug, nullptr, nullptr, w, s, false, false));
   if (device_status) {
-    forward_status<<<1, 1, 0, s>>>(reinterpret_cast<const uint32_t*>(base + lay.status), device_status);
+    forward_status<<<1, 1, 0, s>>>(w.status(), device_status);
     if (cudaGetLastError() != cudaSuccess) return AVR_ERR_CUDA;
   }
   return AVR_OK;

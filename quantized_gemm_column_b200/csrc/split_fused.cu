@@ -40,6 +40,7 @@ struct FusedParams {
   float* slot_mu;           // [G] per-CTA max |mu|
   uint32_t* bar_count;
   uint32_t* bar_gen;
+  const uint64_t* wait_limit;   // ns for the grid barriers' waits (0: the default bound)
   uint8_t* codes;
   uint8_t* scales;
   float* g_dec;
@@ -114,6 +115,7 @@ __global__ void __launch_bounds__(kFuThreads, kBf16 ? 2 : 1) split_fused_kernel(
   __syncthreads();
   pdl_wait_prior_grid();
   pdl_allow_next_grid();
+  const uint64_t wait_limit = __ldcg(p.wait_limit);
 
   // ---------------- phase 1: chunk partials, units kept resident ----------------
   const int n_res = min(kRing, n_mine);        // units that stay in shared memory
@@ -165,7 +167,7 @@ __global__ void __launch_bounds__(kFuThreads, kBf16 ? 2 : 1) split_fused_kernel(
     }
   }
 
-  if (!grid_barrier(p.bar_count, p.bar_gen, static_cast<uint32_t>(G), p.status)) {
+  if (!grid_barrier(p.bar_count, p.bar_gen, static_cast<uint32_t>(G), p.status, wait_limit)) {
     drain();
     return;
   }
@@ -226,7 +228,7 @@ __global__ void __launch_bounds__(kFuThreads, kBf16 ? 2 : 1) split_fused_kernel(
     }
   }
 
-  if (!grid_barrier(p.bar_count, p.bar_gen, static_cast<uint32_t>(G), p.status)) {
+  if (!grid_barrier(p.bar_count, p.bar_gen, static_cast<uint32_t>(G), p.status, wait_limit)) {
     drain();
     return;
   }
@@ -331,8 +333,21 @@ static cudaError_t launch_split_fused_t(const CUtensorMap& map, const FusedParam
   cudaError_t e = set_max_dynamic_smem(fn, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   if (blocks_per_sm(fn, kFuThreads, Cfg::kSmemBytes) < 1) return cudaErrorInvalidConfiguration;
-  return launch_ex(split_fused_kernel<kBf16, kSR>, dim3(static_cast<unsigned>(grid)), dim3(kFuThreads),
-                   Cfg::kSmemBytes, s, pdl, map, p);
+  // A cooperative launch: the runtime refuses a grid whose CTAs cannot all be
+  // resident at once, instead of leaving the grid barriers to time out.  It
+  // is not combined with programmatic dependent launch.
+  (void)pdl;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kFuThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, split_fused_kernel<kBf16, kSR>, map, p);
 }
 
 cudaError_t launch_split_fused(const ColReduceArgs& ca, const QuantArgs& qa, cudaStream_t s, bool pdl) {
@@ -357,6 +372,7 @@ cudaError_t launch_split_fused(const ColReduceArgs& ca, const QuantArgs& qa, cud
   p.status = reinterpret_cast<uint32_t*>(ca.ws + ca.lay->status);
   p.bar_count = p.status + 16;      // 64 and 128 bytes into the status block
   p.bar_gen = p.status + 32;
+  p.wait_limit = reinterpret_cast<const uint64_t*>(ca.ws + ca.lay->status + kWaitLimitOffset);
   p.codes = qa.codes;
   p.scales = qa.scales;
   p.g_dec = qa.g_dec;

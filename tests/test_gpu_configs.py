@@ -1,8 +1,9 @@
 """Parity at the full sizes of the larger workloads (the FFN projections, the
 mean-strength sweep, the 32768-token layer shapes), in the launch
-configuration the benchmark uses: the mean bit-exact over every column, the
-quantized residual bit-exact on sampled rows, outputs within the R19 bound on
-the same rows.
+configuration the benchmark uses: the fp32 mean bit-exact over every column,
+the quantized mean (codes, every scale byte and its decode scale) bit-exact,
+the residual's decode scale bit-exact, the quantized residual bit-exact on
+sampled rows, outputs within the R19 bound on the same rows.
 
 The oracle quantizes only the sampled rows.  Row r of an [l, K] tensor is the
 1 x K tensor at stream offset offset + r K / 16 with the full tensor's amax:
@@ -16,7 +17,7 @@ import torch
 import oracle
 from oracle import nvfp4 as F
 from quantized_gemm_column_b200 import inputs
-from nvfp4_io import check_bf16_output, gemm_tolerance, to_oracle
+from nvfp4_io import assert_nvfp4_equal, check_bf16_output, gemm_tolerance, to_oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -44,11 +45,16 @@ def _rows_of(q, rows):
     return codes, lin
 
 
-def _check_split_rows(xq, muq, x, rows, rm, seed, offset, grad):
-    """The split of x checked on `rows`: X_bar_R rows, mu_bar, decode scales."""
+def _check_split_rows(xq, muq, mu_dev, x, rows, rm, seed, offset, grad):
+    """The split of x: the fp32 mean over every column, the whole of mu_bar
+    (codes, scale bytes, decode scale), X_bar_R's decode scale, and X_bar_R's
+    codes and scales on `rows`."""
     t_r, t_mu = (oracle.TAGS["d_r"], oracle.TAGS["mu_d"]) if grad else (oracle.TAGS["x_r"], oracle.TAGS["mu_x"])
     mu, XR, A = oracle.column_mean_and_residual_amax(x)
     K = x.shape[1]
+    got = mu_dev.cpu().numpy()
+    bad = np.flatnonzero(got.view(np.uint32) != mu.astype(np.float32).view(np.uint32))
+    assert bad.size == 0, f"{bad.size} of {K} mean columns differ, first {bad[:5].tolist()}"
     g_enc, g_dec = F.tensor_scales(A)
     assert np.float32(xq.g_dec.item()).view(np.uint32) == np.float32(g_dec).view(np.uint32)
     codes, lin = _rows_of(xq, rows)
@@ -56,9 +62,7 @@ def _check_split_rows(xq, muq, x, rows, rm, seed, offset, grad):
         ref = oracle.nvfp4_quantize(XR[r:r + 1], rm, seed, offset + (int(r) * K) // 16, t_r, amax=A)
         assert np.array_equal(codes[i], ref.codes[0]), f"codes of row {r}"
         assert np.array_equal(lin[i], ref.scales[0]), f"scales of row {r}"
-    if muq is not None:
-        rmu = oracle.nvfp4_quantize(mu[None, :], rm, seed, offset, t_mu)
-        assert np.array_equal(muq.codes.cpu().numpy(), rmu.codes)
+    assert_nvfp4_equal(muq, oracle.nvfp4_quantize(mu[None, :], rm, seed, offset, t_mu), "mu_bar")
     return mu
 
 
@@ -72,16 +76,24 @@ def _linear_rows(api, X, W, D, rm, seed, n_rows=48):
     xr, muq = api.NVFP4Tensor(l, m), api.NVFP4Tensor(1, m)
     Y = torch.empty((l, n), dtype=torch.bfloat16, device="cuda")
     api.averis_linear_fwd(X.cuda(), w_fwd, rm, seed, 0, Y, ws, save_xr=xr, save_mu=muq)
+    # the same split once more with the fp32 mean requested: it must repeat
+    # the forward's saved operands byte for byte
+    mu_x = torch.empty(m, dtype=torch.float32, device="cuda")
+    xr2, muq2 = api.NVFP4Tensor(l, m), api.NVFP4Tensor(1, m)
+    api.averis_split_quant(X.cuda(), rm, seed, 0, False, mu_x, muq2, xr2, None, ws)
     dr, dmu = api.NVFP4Tensor(l, n), api.NVFP4Tensor(1, n)
-    api.averis_split_quant(D.cuda(), rm, seed + 1, 0, True, None, dmu, dr, None, ws)
+    mu_d = torch.empty(n, dtype=torch.float32, device="cuda")
+    api.averis_split_quant(D.cuda(), rm, seed + 1, 0, True, mu_d, dmu, dr, None, ws)
     dX = torch.empty((l, m), dtype=torch.bfloat16, device="cuda")
     api.averis_linear_dgrad(D.cuda(), w_dgrad, rm, seed + 1, 0, dX, ws)
     assert api.averis_check_status(ws) == 0
+    for a, b in ((xr, xr2), (muq, muq2)):
+        assert torch.equal(a.codes, b.codes) and torch.equal(a.scales, b.scales) and torch.equal(a.g_dec, b.g_dec)
     rows = np.sort(np.random.default_rng(seed).choice(l, n_rows, replace=False))
     x, d = inputs.bf16_as_f32(X), inputs.bf16_as_f32(D)
-    for q, mq, src, w_q, out, K, s, grad in ((xr, muq, x, wf, Y, m, seed, False),
-                                            (dr, dmu, d, wd, dX, n, seed + 1, True)):
-        _check_split_rows(q, mq, src, rows, rm, s, 0, grad)
+    for q, mq, mu_dev, src, w_q, out, K, s, grad in ((xr, muq, mu_x, x, wf, Y, m, seed, False),
+                                                    (dr, dmu, mu_d, d, wd, dX, n, seed + 1, True)):
+        _check_split_rows(q, mq, mu_dev, src, rows, rm, s, 0, grad)
         a_rows = to_oracle(q)
         a_rows = oracle.NVFP4(a_rows.codes[rows], a_rows.scales[rows], a_rows.g_dec, len(rows), K)
         b = oracle.bias_row(to_oracle(mq), w_q)

@@ -142,3 +142,43 @@ def test_quantized_operands_from_oracle(api):
     Y = _gemm(api, a, b)
     ref = oracle.gemm_reference(a, b)
     assert np.linalg.norm(Y - ref) / np.linalg.norm(ref) <= 1e-5
+
+
+def _gemm_sampled(api, a_q, b_q, cols, bias=None, out=torch.float32):
+    """Run the GEMM and return its output and the oracle's product on the
+    columns `cols` (rows of B) only."""
+    Y = _gemm(api, a_q, b_q, bias, out=out)
+    b_sub = oracle.NVFP4(b_q.codes[cols], b_q.scales[cols], b_q.g_dec, len(cols), b_q.K)
+    ref = oracle.gemm_reference(a_q, b_sub, None if bias is None else np.asarray(bias)[cols])
+    return Y[:, cols], ref, b_sub
+
+
+@pytest.mark.parametrize("K", [256, 1280, 1536, 2112])
+def test_resident_b_scales_across_column_blocks_bf16(api, K):
+    """Many more tiles than CTAs with two row blocks, so a CTA's run of tiles
+    changes column block (B's resident scales are reloaded) and shares it
+    between tiles.  K = 256 and 1280 keep every stage's B scales resident,
+    1536 five of six, 2112 five of nine with a partial last stage."""
+    rng = np.random.default_rng(K)
+    M, N = 256, 256 * 160
+    a = _rand_q(rng, M, K, g_dec=0.01)
+    b = _rand_q(rng, N, K, g_dec=0.003)
+    bias = rng.standard_normal(N) * 0.1
+    cols = np.sort(rng.choice(N, 640, replace=False))
+    Y, ref, b_sub = _gemm_sampled(api, a, b, cols, bias, out=torch.bfloat16)
+    check_bf16_output(Y, ref, gemm_tolerance(a, b_sub, np.asarray(bias)[cols], K))
+
+
+@pytest.mark.parametrize("K", [3072, 3264])
+def test_resident_b_scales_across_column_blocks_fp32(api, K):
+    """The fp32-output tiles (128 columns) keep up to twelve stages of B's
+    scales resident: K = 3072 is all resident, 3264 leaves a partial
+    thirteenth stage streamed."""
+    rng = np.random.default_rng(K + 1)
+    M, N = 256, 128 * 320
+    a = _rand_q(rng, M, K, g_dec=0.013)
+    b = _rand_q(rng, N, K, g_dec=0.002)
+    cols = np.sort(rng.choice(N, 512, replace=False))
+    Y, ref, _ = _gemm_sampled(api, a, b, cols)
+    rel = np.linalg.norm(Y - ref) / np.linalg.norm(ref)
+    assert rel <= 1e-5, rel

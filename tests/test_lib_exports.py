@@ -234,3 +234,73 @@ def test_valid_call_without_a_device_fails_loudly(lib):
     st = lib.averis_linear_fwd(ctypes.c_void_p(16), 1, 256, 128, 192, ctypes.byref(wf), 1, 0, 0,
                                ctypes.c_void_p(32), 1, None, None, ctypes.c_void_p(256), 1 << 40, None)
     assert st == api.AVR_ERR_NO_DEVICE
+
+
+def test_noalloc_validation_matches_the_workspace_entry_point(lib):
+    """averis_split_quant_noalloc rejects what averis_split_quant rejects, with
+    the same codes, before it touches a device: null and mis-shaped
+    descriptors, misaligned codes, scales and decode scales, a misaligned
+    status word, sizes beyond its fixed scratch."""
+    from quantized_gemm_column_b200 import api
+    f = lib.averis_split_quant_noalloc
+    X = ctypes.c_void_p(16)
+
+    def call(xr, muq=None, x=X, l=256, K=128, status=None, xt=1, rm=0):
+        return f(x, xt, l, K, rm, 0, 0, 0, None, None if muq is None else ctypes.byref(muq),
+                 None if xr is None else ctypes.byref(xr), None, status, None)
+
+    good = api.avr_nvfp4(16, 16, 16, 256, 128)
+    assert call(None) == api.AVR_ERR_INVALID_ARG                                   # no X_bar_R descriptor
+    assert call(good, x=None) == api.AVR_ERR_INVALID_ARG                           # no input
+    assert call(api.avr_nvfp4(0, 16, 16, 256, 128)) == api.AVR_ERR_INVALID_ARG     # null codes
+    assert call(api.avr_nvfp4(16, 0, 16, 256, 128)) == api.AVR_ERR_INVALID_ARG     # null scales
+    assert call(api.avr_nvfp4(16, 16, 0, 256, 128)) == api.AVR_ERR_INVALID_ARG     # null g_dec
+    assert call(api.avr_nvfp4(16, 16, 16, 255, 128)) == api.AVR_ERR_INVALID_ARG   # rows != l
+    assert call(api.avr_nvfp4(16, 16, 16, 256, 192)) == api.AVR_ERR_INVALID_ARG   # K disagrees
+    assert call(good, api.avr_nvfp4(16, 16, 16, 2, 128)) == api.AVR_ERR_INVALID_ARG   # mu_bar rows != 1
+    assert call(good, api.avr_nvfp4(0, 16, 16, 1, 128)) == api.AVR_ERR_INVALID_ARG    # mu_bar null codes
+    assert call(api.avr_nvfp4(24, 16, 16, 256, 128)) == api.AVR_ERR_MISALIGNED    # codes
+    assert call(api.avr_nvfp4(16, 24, 16, 256, 128)) == api.AVR_ERR_MISALIGNED    # scales
+    assert call(api.avr_nvfp4(16, 16, 18, 256, 128)) == api.AVR_ERR_MISALIGNED    # g_dec
+    assert call(good, api.avr_nvfp4(16, 16, 18, 1, 128)) == api.AVR_ERR_MISALIGNED   # mu_bar g_dec
+    assert call(good, x=ctypes.c_void_p(24)) == api.AVR_ERR_MISALIGNED           # input
+    assert call(good, status=ctypes.c_void_p(18)) == api.AVR_ERR_MISALIGNED      # status word
+    assert call(good, K=100) == api.AVR_ERR_UNSUPPORTED_SHAPE
+    assert call(good, xt=5) == api.AVR_ERR_INVALID_ARG
+    assert call(good, rm=3) == api.AVR_ERR_INVALID_ARG
+    assert call(api.avr_nvfp4(16, 16, 16, 0, 128), l=0) == api.AVR_OK             # no tokens: no-op
+    # beyond the fixed scratch: 3 ceil(l/256) K 4 bytes of partials alone exceed 4 MiB
+    big = api.avr_nvfp4(16, 16, 16, 32768, 4096)
+    assert call(big, l=32768, K=4096) == api.AVR_ERR_WORKSPACE_TOO_SMALL
+    # the workspace entry point gives the same codes for the same arguments
+    ws = ctypes.c_void_p(256)
+    for xr, muq in ((api.avr_nvfp4(16, 16, 18, 256, 128), None), (api.avr_nvfp4(16, 16, 16, 255, 128), None),
+                    (good, api.avr_nvfp4(16, 16, 16, 2, 128))):
+        ws_code = lib.averis_split_quant(X, 1, 256, 128, 0, 0, 0, 0, None,
+                                         None if muq is None else ctypes.byref(muq), ctypes.byref(xr), None,
+                                         ws, 1 << 40, None)
+        assert call(xr, muq) == ws_code
+
+
+def test_noalloc_without_a_device_fails_loudly(lib):
+    """A valid no-alloc call returns AVR_ERR_NO_DEVICE on a host without an
+    sm_100 device (skipped where a GPU is visible)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is visible; this check is for a host without one")
+    from quantized_gemm_column_b200 import api
+    xr = api.avr_nvfp4(16, 16, 16, 256, 128)
+    st = lib.averis_split_quant_noalloc(ctypes.c_void_p(16), 1, 256, 128, 1, 0, 0, 0, None, None,
+                                        ctypes.byref(xr), None, None, None)
+    assert st == api.AVR_ERR_NO_DEVICE
+
+
+def test_set_wait_limit_validation_on_the_host(lib):
+    from quantized_gemm_column_b200 import api
+    f = lib.averis_set_wait_limit
+    assert f(None, 1 << 20, 5, None) == api.AVR_ERR_INVALID_ARG
+    assert f(ctypes.c_void_p(272), 1 << 20, 5, None) == api.AVR_ERR_MISALIGNED
+    assert f(ctypes.c_void_p(256), 128, 5, None) == api.AVR_ERR_WORKSPACE_TOO_SMALL
+    import torch
+    if not torch.cuda.is_available():
+        assert f(ctypes.c_void_p(256), 1 << 20, 5, None) == api.AVR_ERR_NO_DEVICE
