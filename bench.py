@@ -142,18 +142,21 @@ class ClockSampler:
 STACK_SHAPES = (("qkv", 1024, 4096), ("o_proj", 2048, 1024), ("gate_up", 1024, 6144), ("down", 3072, 1024))
 
 
-def stack_timing(dev, stream, layers=28, tokens=32768, steps=2):
+def stack_timing(dev, stream, layers=28, tokens=32768, steps=3):
     """Forward + dgrad through the 4 linears of each of `layers` layers at
-    `tokens` tokens, Averis and vanilla NVFP4, CUDA-graph replay of one layer.
-    Inputs are drawn on the device (seeded): activations = per-column mean
-    N(0, 0.5) with 1% of channels x20 + N(0, 1) (the down projection's input:
-    silu(a) b with a, b ~ N(0.2, 1)); output gradients 1e-3 (N(0, 1) + per-column
-    N(0, 0.3)); weights N(0, 1/sqrt(m)), one per shape for all layers."""
+    `tokens` tokens, Averis and vanilla NVFP4, one CUDA graph of the whole
+    stack per mode, replayed `steps` times.  Every layer has its own weights
+    (N(0, 1/sqrt(m)), quantized once); the activations and output gradients
+    of a shape are shared by the layers (drawn on the device, seeded):
+    activations = per-column mean N(0, 0.5) with 1% of channels x20 + N(0, 1)
+    (the down projection's input: silu(a) b with a, b ~ N(0.2, 1)); output
+    gradients 1e-3 (N(0, 1) + per-column N(0, 0.3)).  SM clocks are sampled
+    over the timed replays (tens of ms, so several samples fall inside)."""
     import torch
     from quantized_gemm_column_b200 import api
     g = torch.Generator(device=dev)
     g.manual_seed(20)
-    bufs = []
+    acts, weights = [], []
     for name, m, n in STACK_SHAPES:
         if name == "down":
             a = torch.randn(tokens, m, generator=g, device=dev) + 0.2
@@ -167,52 +170,69 @@ def stack_timing(dev, stream, layers=28, tokens=32768, steps=2):
             X = (torch.randn(tokens, m, generator=g, device=dev) + mu).to(torch.bfloat16)
         D = ((torch.randn(tokens, n, generator=g, device=dev) + torch.randn(n, generator=g, device=dev) * 0.3)
              * 1e-3).to(torch.bfloat16)
-        W = (torch.randn(m, n, generator=g, device=dev) / m ** 0.5).to(torch.bfloat16)
-        w_fwd, w_dgrad = api.NVFP4Tensor(n, m, dev), api.NVFP4Tensor(m, n, dev)
         ws = api.workspace(tokens, max(m, n), max(m, n), dev)
-        torch.cuda.synchronize(dev)            # drawn on the default stream, consumed on `stream`
-        api.averis_quant_weight(W, w_fwd, w_dgrad, ws, stream)
         Y = torch.empty((tokens, n), dtype=torch.bfloat16, device=dev)
         dX = torch.empty((tokens, m), dtype=torch.bfloat16, device=dev)
-        bufs.append((X, D, w_fwd, w_dgrad, ws, Y, dX))
+        acts.append((X, D, ws, Y, dX))
+    torch.cuda.synchronize(dev)                # drawn on the default stream, consumed on `stream`
+    for _ in range(layers):
+        per_layer = []
+        for name, m, n in STACK_SHAPES:
+            W = (torch.randn(m, n, generator=g, device=dev) / m ** 0.5).to(torch.bfloat16)
+            w_fwd, w_dgrad = api.NVFP4Tensor(n, m, dev), api.NVFP4Tensor(m, n, dev)
+            wq_ws = api.workspace(m, n, n, dev)
+            torch.cuda.synchronize(dev)
+            api.averis_quant_weight(W, w_fwd, w_dgrad, wq_ws, stream)
+            torch.cuda.synchronize(dev)
+            if api.averis_check_status(wq_ws, stream):
+                raise RuntimeError("device status set by the stack's weight quantization")
+            del W, wq_ws
+            per_layer.append((w_fwd, w_dgrad))
+        weights.append(per_layer)
 
-    def layer(vanilla):
-        for X, D, w_fwd, w_dgrad, ws, Y, dX in bufs:
-            if vanilla:
-                api.nvfp4_linear_fwd(X, w_fwd, "sr", 1, 0, Y, ws, stream=stream)
-                api.nvfp4_linear_dgrad(D, w_dgrad, "sr", 2, 0, dX, ws, stream=stream)
-            else:
-                api.averis_linear_fwd(X, w_fwd, "sr", 1, 0, Y, ws, stream=stream)
-                api.averis_linear_dgrad(D, w_dgrad, "sr", 2, 0, dX, ws, stream=stream)
+    def stack(vanilla):
+        for per_layer in weights:
+            for (X, D, ws, Y, dX), (w_fwd, w_dgrad) in zip(acts, per_layer):
+                if vanilla:
+                    api.nvfp4_linear_fwd(X, w_fwd, "sr", 1, 0, Y, ws, stream=stream)
+                    api.nvfp4_linear_dgrad(D, w_dgrad, "sr", 2, 0, dX, ws, stream=stream)
+                else:
+                    api.averis_linear_fwd(X, w_fwd, "sr", 1, 0, Y, ws, stream=stream)
+                    api.averis_linear_dgrad(D, w_dgrad, "sr", 2, 0, dX, ws, stream=stream)
 
     torch.cuda.synchronize(dev)
-    out = {}
+    out, clocks = {}, {}
     for vanilla in (False, True):
         with torch.cuda.stream(stream):
-            layer(vanilla)
+            stack(vanilla)
             torch.cuda.synchronize(dev)
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr, stream=stream):
-                layer(vanilla)
-            for _ in range(layers):
-                gr.replay()
+                stack(vanilla)
+            gr.replay()
             torch.cuda.synchronize(dev)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(steps * layers):
-                gr.replay()
-            b.record(stream)
-            torch.cuda.synchronize(dev)
+            with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+                t0 = time.monotonic()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for _ in range(steps):
+                    gr.replay()
+                b.record(stream)
+                torch.cuda.synchronize(dev)
+                clk.region(t0, time.monotonic())
+            clocks["vanilla" if vanilla else "averis"] = clk.summary()
         out["vanilla_ms" if vanilla else "averis_ms"] = a.elapsed_time(b) / steps
         del gr
-    for _, _, _, _, ws, _, _ in bufs:
+    for _, _, ws, _, _ in acts:
         if api.averis_check_status(ws, stream):
             raise RuntimeError("device status set by the stack timing")
     flops = sum(2.0 * tokens * m * n * 2 for _, m, n in STACK_SHAPES) * layers
     return {"layers": layers, "tokens": tokens, "shapes": {s[0]: [s[1], s[2]] for s in STACK_SHAPES},
+            "weights": "distinct per layer", "launch": "one CUDA graph of the whole stack per mode",
             "averis_ms_per_step": out["averis_ms"], "vanilla_ms_per_step": out["vanilla_ms"],
             "averis_overhead_vs_vanilla": out["averis_ms"] / out["vanilla_ms"] - 1.0,
             "tflops": flops / (out["averis_ms"] * 1e-3) / 1e12,
+            "clocks": clocks,
             "data": "synthetic, drawn on the device (seeded)"}
 
 
@@ -247,6 +267,181 @@ def moe_timing(dev, stream, avg_us):
     return {"experts": E, "tokens_routed": tokens, "rows_padded": l_cap, "m": m, "n": n,
             "fwd_us": fwd, "dgrad_us": dgr, "tflops": 2 * flops / ((fwd + dgr) * 1e-6) / 1e12,
             "launches_per_pass": 5}
+
+
+# ---------------------------------------------------------------------------
+# the measured FP4 ceiling
+# ---------------------------------------------------------------------------
+def fp4_ceiling(dev, stream):
+    """The dense block-scaled FP4 rate of this device, measured two ways: this
+    library's MMA-only tcgen05 loop on every SM (the tensor pipe alone, no
+    loads), and cuBLASLt's NVFP4 GEMM at 8192^3 through torch._scaled_mm (a
+    library GEMM, loads included).  Each is the best of 3 timed runs."""
+    import torch
+    from quantized_gemm_column_b200 import api
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    ns = torch.zeros(sms, dtype=torch.int64, device=dev)
+    ws = api.workspace(0, 64, 0, dev)
+    iters = 20000
+    best = None
+    with torch.cuda.stream(stream):
+        api.averis_probe_mma_rate(2000, ns, ws, stream)
+        for _ in range(3):
+            api.averis_probe_mma_rate(iters, ns, ws, stream)
+            torch.cuda.synchronize(dev)
+            t = 2.0 * 128 * 256 * 256 * iters * sms / (int(ns.max().item()) * 1e-9) / 1e12
+            best = t if best is None else max(best, t)
+    if api.averis_check_status(ws, stream):
+        raise RuntimeError("device status set by the MMA-rate loop")
+    out = {"mma_loop_tflops": best, "mma_loop": f"{sms} CTAs x {iters} stages of 4 MMAs (M128 N256 K64), constant operands"}
+    try:
+        n = 8192
+        a = torch.randint(0, 256, (n, n // 2), dtype=torch.uint8, device=dev).view(torch.float4_e2m1fn_x2)
+        b = torch.randint(0, 256, (n, n // 2), dtype=torch.uint8, device=dev).view(torch.float4_e2m1fn_x2)
+        sa = (torch.rand(n * n // 16, device=dev) + 0.5).to(torch.float8_e4m3fn)
+        sb = (torch.rand(n * n // 16, device=dev) + 0.5).to(torch.float8_e4m3fn)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                torch._scaled_mm(a, b.t(), sa, sb, out_dtype=torch.bfloat16)
+            best = None
+            for _ in range(3):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(10):
+                    torch._scaled_mm(a, b.t(), sa, sb, out_dtype=torch.bfloat16)
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                t = 2.0 * n ** 3 / (e0.elapsed_time(e1) * 1e-3 / 10) / 1e12
+                best = t if best is None else max(best, t)
+        out["cublaslt_nvfp4_8192_tflops"] = best
+        del a, b, sa, sb
+    except Exception as exc:          # a torch without the NVFP4 path
+        out["cublaslt_nvfp4_8192_tflops"] = None
+        out["cublaslt_error"] = f"{type(exc).__name__}: {str(exc)[:120]}"
+    return out
+
+
+# ---------------------------------------------------------------------------
+# one linear at full size: Averis vs vanilla, the split and the GEMMs
+# ---------------------------------------------------------------------------
+def linear_timing(dev, stream, avg_us, X, W, D, fp4_peak):
+    """Forward + dgrad of one linear (X [l, m], W [m, n], dY [l, n]), stochastic
+    rounding: Averis and vanilla step times, the two splits and the two GEMMs
+    on their own, TFLOP/s, the Averis overhead and the GEMMs' fraction of the
+    measured FP4 peak."""
+    import torch
+    from quantized_gemm_column_b200 import api
+    l, m = X.shape
+    n = W.shape[1]
+    Xd, Wd, Dd = X.to(dev), W.to(dev), D.to(dev)
+    w_fwd, w_dgrad = api.NVFP4Tensor(n, m, dev), api.NVFP4Tensor(m, n, dev)
+    ws = api.workspace(l, max(m, n), max(m, n), dev)
+    torch.cuda.synchronize(dev)
+    api.averis_quant_weight(Wd, w_fwd, w_dgrad, ws, stream)
+    Y = torch.empty((l, n), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((l, m), dtype=torch.bfloat16, device=dev)
+    xr, dr = api.NVFP4Tensor(l, m, dev), api.NVFP4Tensor(l, n, dev)
+    muq, dmuq = api.NVFP4Tensor(1, m, dev), api.NVFP4Tensor(1, n, dev)
+
+    def averis(i):
+        api.averis_linear_fwd(Xd, w_fwd, "sr", 1 + i, 0, Y, ws, stream=stream)
+        api.averis_linear_dgrad(Dd, w_dgrad, "sr", 1 + i, 0, dX, ws, stream=stream)
+
+    def vanilla(i):
+        api.nvfp4_linear_fwd(Xd, w_fwd, "sr", 1 + i, 0, Y, ws, stream=stream)
+        api.nvfp4_linear_dgrad(Dd, w_dgrad, "sr", 1 + i, 0, dX, ws, stream=stream)
+
+    t_a = avg_us(averis)
+    t_v = avg_us(vanilla)
+    sq_x = avg_us(lambda i: api.averis_split_quant(Xd, "sr", 1, 0, False, None, muq, xr, None, ws, stream))
+    sq_d = avg_us(lambda i: api.averis_split_quant(Dd, "sr", 1, 0, True, None, dmuq, dr, None, ws, stream))
+    g_f = avg_us(lambda i: api.nvfp4_gemm(xr, w_fwd, None, Y, ws, stream))
+    g_d = avg_us(lambda i: api.nvfp4_gemm(dr, w_dgrad, None, dX, ws, stream))
+    if api.averis_check_status(ws, stream):
+        raise RuntimeError("device status set by the linear timing")
+    flops = 2.0 * 2 * l * m * n
+    gemm_tf = flops / ((g_f + g_d) * 1e-6) / 1e12
+    del Xd, Wd, Dd, Y, dX, xr, dr
+    return {"l": l, "m": m, "n": n, "averis_us": t_a, "vanilla_us": t_v,
+            "averis_overhead_vs_vanilla": t_a / t_v - 1.0, "tflops": flops / (t_a * 1e-6) / 1e12,
+            "split_quant_us": {"X": sq_x, "dY": sq_d}, "gemm_us": {"fwd": g_f, "dgrad": g_d},
+            "gemm_tflops": gemm_tf, "gemm_frac_fp4_peak": gemm_tf / fp4_peak}
+
+
+# ---------------------------------------------------------------------------
+# the mean-strength sweep: the pages' effect measured on this library's output
+# ---------------------------------------------------------------------------
+E2M1_VALUES = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0]
+
+
+def dequantize(q, dev):
+    """value(code) * value(scale) * g_dec of a device NVFP4 tensor, fp32 on the
+    device (codes two per byte, element 2k low; scales in the 128 x 4 atom
+    layout).  A reporting aid of this script."""
+    import torch
+    R, K = q.rows, q.K
+    lut = torch.tensor(E2M1_VALUES, dtype=torch.float32, device=dev)
+    c = q.codes.to(torch.int64)
+    vals = torch.stack([lut[c & 15], lut[c >> 4]], dim=-1).reshape(R, K)
+    r = torch.arange(R, device=dev)[:, None]
+    cb = torch.arange(K // 16, device=dev)[None, :]
+    off = ((r // 128) * (K // 64) + cb // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + cb % 4
+    sc = q.scales[off].view(torch.float8_e4m3fn).to(torch.float32)
+    return vals * sc.repeat_interleave(16, dim=1) * q.g_dec.float()
+
+
+def sweep_metrics(dev, stream, avg_us, rows_checked=256):
+    """The mean-strength sweep (X [16384, 2048] = c 1 mu^T + rank-4 spike +
+    N(0, 1), W [2048, 2048]) at c in {0, 0.5, 2, 8, 32}, stochastic rounding.
+    Per c: entries over t = 3 and 4 (sigma of the Gaussian tail = 1) in X and
+    in the residual X - 1 mu; the FP4 reconstruction error ||deq - X||_F /
+    ||X||_F of vanilla Q4(X) and of Averis 1 deq(mu_bar) + deq(X_bar_R); the
+    forward output's error against the fp64 product X W on sampled rows; and
+    the Averis and vanilla forward times (split + GEMM)."""
+    import torch
+    from quantized_gemm_column_b200 import api, inputs
+    out = []
+    for c in inputs.WORKLOADS[3]["mean_scales"]:
+        X, W = inputs.workload3(c)
+        l, m = X.shape
+        n = W.shape[1]
+        Xd, Wd = X.to(dev), W.to(dev)
+        w_fwd, w_dgrad = api.NVFP4Tensor(n, m, dev), api.NVFP4Tensor(m, n, dev)
+        ws = api.workspace(l, max(m, n), max(m, n), dev)
+        torch.cuda.synchronize(dev)
+        api.averis_quant_weight(Wd, w_fwd, w_dgrad, ws, stream)
+        mu = torch.empty(m, dtype=torch.float32, device=dev)
+        xr, muq, xv = api.NVFP4Tensor(l, m, dev), api.NVFP4Tensor(1, m, dev), api.NVFP4Tensor(l, m, dev)
+        api.averis_split_quant(Xd, "sr", 7, 0, False, mu, muq, xr, None, ws, stream)
+        api.nvfp4_quant(Xd, "sr", 7, 0, False, xv, ws, stream)
+        Ya = torch.empty((l, n), dtype=torch.bfloat16, device=dev)
+        Yv = torch.empty((l, n), dtype=torch.bfloat16, device=dev)
+        t_a = avg_us(lambda i: api.averis_linear_fwd(Xd, w_fwd, "sr", 7, 0, Ya, ws, stream=stream))
+        t_v = avg_us(lambda i: api.nvfp4_linear_fwd(Xd, w_fwd, "sr", 7, 0, Yv, ws, stream=stream))
+        if api.averis_check_status(ws, stream):
+            raise RuntimeError("device status set by the sweep")
+        with torch.cuda.stream(stream):
+            x = Xd.float()
+            xres = x - mu[None, :]
+            over = {f"t{t}": {"X": int((x.abs() > t).sum().item()), "X_R": int((xres.abs() > t).sum().item())}
+                    for t in (3, 4)}
+            nx = torch.linalg.vector_norm(x).item()
+            err_v = torch.linalg.vector_norm(dequantize(xv, dev) - x).item() / nx
+            rec_a = dequantize(xr, dev) + dequantize(muq, dev)
+            err_a = torch.linalg.vector_norm(rec_a - x).item() / nx
+            del rec_a, xres
+            rows = torch.randperm(l, generator=torch.Generator().manual_seed(5))[:rows_checked].to(dev)
+            ref = Xd[rows].double() @ Wd.double()
+            nref = torch.linalg.vector_norm(ref).item()
+            gerr_a = torch.linalg.vector_norm(Ya[rows].double() - ref).item() / nref
+            gerr_v = torch.linalg.vector_norm(Yv[rows].double() - ref).item() / nref
+            torch.cuda.synchronize(dev)
+        out.append({"c": c, "over_threshold": over, "elements": l * m,
+                    "fp4_recon_rel_err": {"vanilla": err_v, "averis": err_a},
+                    "gemm_rel_err_vs_fp64_xw": {"vanilla": gerr_v, "averis": gerr_a, "rows": rows_checked},
+                    "fwd_us": {"averis": t_a, "vanilla": t_v}})
+        del Xd, Wd, x, Ya, Yv, xr, xv
+    return {"l": 16384, "m": 2048, "n": 2048, "rounding": "philox-sr", "per_c": out}
 
 
 # ---------------------------------------------------------------------------
@@ -332,8 +527,9 @@ def run_reference(args, rank, world):
 # ---------------------------------------------------------------------------
 # measured DRAM traffic (ncu), valid only for the kernel sources it was taken on
 # ---------------------------------------------------------------------------
-KERNEL_SOURCES = ["colreduce.cu", "quant.cu", "quant_common.cuh", "split_fused.cu", "gemm.cu", "device.cuh", "internal.h"]
-TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "traffic_qkv_step.md")
+KERNEL_SOURCES = ["colreduce.cu", "quant.cu", "quant_common.cuh", "split_fused.cu", "gemm.cu", "gemm2.cu",
+                  "device.cuh", "internal.h"]
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "traffic_qkv_step.json")
 
 
 def kernel_digest():
@@ -346,19 +542,16 @@ def kernel_digest():
 
 
 def measured_traffic(key):
-    """DRAM bytes per step of a kernel group from the committed ncu summary,
-    or None if the summary is missing or was taken on other kernel sources."""
+    """DRAM bytes per step of a kernel group ("split-quant" or "gemm") from the
+    committed ncu capture (profiles/traffic_qkv_step.json), or None if it is
+    missing or was taken on other kernel sources."""
     try:
-        fields = {}
-        for line in open(TRAFFIC_PROFILE):
-            line = line.strip()
-            if line.startswith("traffic-") and ":" in line:
-                k, v = line.split(":", 1)
-                fields[k.strip()] = v.strip()
-        if fields.get("traffic-digest") != kernel_digest():
+        with open(TRAFFIC_PROFILE) as fh:
+            rec = json.load(fh)
+        if rec.get("digest") != kernel_digest():
             return None
-        return int(fields[f"traffic-{key}-bytes-per-step"])
-    except (OSError, KeyError, ValueError):
+        return int(rec["bytes_per_step"][key])
+    except (OSError, KeyError, ValueError, TypeError):
         return None
 
 
@@ -540,6 +733,28 @@ def run_gpu(args, rank, world, local_rank):
              "gemm_tflops": 2 * L * M * N / (g_w * 1e-6) / 1e12}
 
     moe = moe_timing(dev, stream, avg_us)
+    fp4 = fp4_ceiling(dev, stream)
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        pass
+    bf16_peak = peaks.get("bf16_tflops", 1590.0)
+    fp4_nominal = 4.0 * bf16_peak          # nominal dense FP4 : BF16 ratio 9 : 2.25
+    fp4_peak = fp4["mma_loop_tflops"] or fp4_nominal
+    fp4["bf16x4_nominal_tflops"] = fp4_nominal
+    # the FFN projections of the Qwen3-0.6B layer at 16384 tokens, one linear at a time
+    from quantized_gemm_column_b200 import inputs
+    gX = inputs.to_bf16(inputs.spiked_activations(inputs.rng_for(2, 1), 16384, 1024, rank=4,
+                                                  s=(16.0, 8.0, 6.0, 4.0), n_hot=10))
+    gW = inputs.to_bf16(inputs.weight(inputs.rng_for(2, 2), 1024, 6144))
+    gD = inputs.to_bf16(inputs.output_gradient(inputs.rng_for(2, 3), 16384, 6144))
+    ffn = {"gate_up": linear_timing(dev, stream, avg_us, gX, gW, gD, fp4_peak)}
+    del gX, gW, gD
+    dXin, dWin, dDin = inputs.workload2_down()
+    ffn["down"] = linear_timing(dev, stream, avg_us, dXin, dWin, dDin, fp4_peak)
+    del dXin, dWin, dDin
+    sweep = sweep_metrics(dev, stream, avg_us)
     stack = stack_timing(dev, stream)
 
     # split-quant algorithmic bytes: read the input twice (reduce, quantize),
@@ -548,24 +763,18 @@ def run_gpu(args, rank, world, local_rank):
         return rows * K * (2 * 2 + 0.5 + 1.0 / 16)
     sq_gbs = (sq_bytes(L, M) + sq_bytes(L, N)) / ((sq_x + sq_d) * 1e-6) / 1e9
 
-    peaks = {}
-    try:
-        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
-    except Exception:
-        pass
-    bf16_peak = peaks.get("bf16_tflops", 1590.0)
-    fp4_peak = 4.0 * bf16_peak             # nominal dense FP4 : BF16 ratio 9 : 2.25
     hbm_peak = peaks.get("hbm_gbs", 6650.0)
     peak_src = "measured" if peaks else "fallback"
 
     # dominant kernel group by time share of the step
     gemm_share = (g_f + g_d) / (step_ms * 1e3)
     if gemm_share >= 0.5:
-        roof = {"bound": "tensor", "kernel": "gemm_nvfp4_kernel (fwd + dgrad)",
+        roof = {"bound": "tensor", "kernel": "gemm2_nvfp4_kernel (fwd + dgrad)",
                 "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                 "frac": gemm_tflops / fp4_peak, "traffic": measured_traffic("gemm"),
                 "traffic_unit": "DRAM bytes per step (fwd + dgrad launches)",
-                "peak_source": f"{peak_src} bf16 x 4 (nominal FP4:BF16 ratio)"}
+                "peak_source": "measured: this device's MMA-only tcgen05 FP4 loop",
+                "peak_bf16x4_nominal": fp4_nominal}
     else:
         roof = {"bound": "hbm", "kernel": "colreduce_kernel + fold_kernel + quant_kernel (split-quant, X and dY)",
                 "achieved": sq_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": sq_gbs / hbm_peak,
@@ -652,6 +861,9 @@ def run_gpu(args, rank, world, local_rank):
         "moe": moe,
         "stack": stack,
         "gemm_frac_fp4_peak": gemm_tflops / fp4_peak,
+        "fp4_ceiling": fp4,
+        "ffn": ffn,
+        "sweep": sweep,
         "vanilla_ms_per_step": ms_van / args.steps,
         "averis_overhead_vs_vanilla": (ms / ms_van) - 1.0,
         "weight_quant_us": wq_us,

@@ -406,6 +406,16 @@ avr_status averis_probe_convert(const float* in, uint8_t* e4m3, uint8_t* e2m1, i
 avr_status averis_probe_convert_sr(const float* in, const uint32_t* rbits, uint16_t* out, int64_t n,
                                    avr_stream stream);
 
+/* The tensor pipe's block-scaled FP4 rate, measured (for the roofline; not
+ * part of the method): `grid` CTAs, one per SM at most, each issue `iters`
+ * stages of four tcgen05.mma.kind::mxf4nvf4.block_scale.block16 of M 128 x
+ * N 256 x K 64 from constant shared-memory operands, no loads or copies in
+ * the loop.  ns [grid] (device, 8-byte aligned) receives each CTA's elapsed
+ * nanoseconds; the rate is 2*128*256*256*iters*grid / max(ns) flop/ns.  ws:
+ * a workspace for the status word (timeouts).  Errors: AVR_ERR_INVALID_ARG
+ * (iters or grid < 1, null ns), AVR_ERR_MISALIGNED, AVR_ERR_NO_DEVICE. */
+avr_status averis_probe_mma_rate(int iters, int grid, uint64_t* ns, void* ws, size_t ws_bytes, avr_stream stream);
+
 /* out[4*i .. 4*i+3] = Philox4x32-10 words of counter (lo32(offset+i),
  * hi32(offset+i), tag, 0) under key (lo32(seed), hi32(seed)), i < n. */
 avr_status averis_probe_philox(uint64_t seed, uint64_t offset, uint32_t tag, int64_t n,

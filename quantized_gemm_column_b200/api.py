@@ -56,6 +56,7 @@ _SIGS = {
     "averis_workspace_init": (_c_int, [_c_ptr, _c_size, _c_ptr]),
     "averis_check_status": (_c_int, [_c_ptr, _c_ptr]),
     "averis_set_wait_limit": (_c_int, [_c_ptr, _c_size, _c_u64, _c_ptr]),
+    "averis_probe_mma_rate": (_c_int, [_c_int, _c_int, _c_ptr, _c_ptr, _c_size, _c_ptr]),
     "averis_status_string": (ctypes.c_char_p, [_c_int]),
     "averis_split_quant": (_c_int, [_c_ptr, _c_int, _c_i64, _c_i64, _c_int, _c_u64, _c_u64, _c_int,
                                     _c_ptr, ctypes.POINTER(avr_nvfp4), ctypes.POINTER(avr_nvfp4),
@@ -215,6 +216,13 @@ def averis_workspace_init(ws, stream=None):
 def averis_check_status(ws, stream=None):
     """Synchronize and return the latched device status (0 = ok)."""
     return int(load().averis_check_status(_ptr(ws), _stream(stream)))
+
+
+def averis_probe_mma_rate(iters, ns, ws, stream=None):
+    """MMA-only tcgen05 FP4 loop on ns.numel() CTAs; ns (int64, device) gets
+    each CTA's elapsed nanoseconds."""
+    _check(load().averis_probe_mma_rate(int(iters), ns.numel(), _ptr(ns), _ptr(ws), ws.numel(), _stream(stream)),
+           "averis_probe_mma_rate")
 
 
 def averis_set_wait_limit(ws, limit_ns, stream=None):

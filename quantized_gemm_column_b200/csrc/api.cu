@@ -93,7 +93,7 @@ bool make_tensor_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType 
 }
 
 bool make_tensor_map_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, const uint64_t dims[3],
-                        const uint64_t strides[2], const uint32_t box[3]) {
+                        const uint64_t strides[2], const uint32_t box[3], CUtensorMapSwizzle swizzle) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
@@ -101,7 +101,7 @@ bool make_tensor_map_3d(CUtensorMap* map, const void* base, CUtensorMapDataType 
   cuuint32_t b[3] = {box[0], box[1], box[2]};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, dtype, 3, const_cast<void*>(base), d, st, b, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -922,6 +922,15 @@ avr_status averis_probe_convert_sr(const float* in, const uint32_t* rbits, uint1
   if (n == 0) return AVR_OK;
   AVR_TRY(device_ok());
   return cuda_status(launch_probe_convert_sr(in, rbits, out, n, stream));
+}
+
+avr_status averis_probe_mma_rate(int iters, int grid, uint64_t* ns, void* ws, size_t ws_bytes, avr_stream stream) {
+  if (iters < 1 || grid < 1 || !ns) return AVR_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ns) & 7u) return AVR_ERR_MISALIGNED;
+  Ws w;
+  AVR_TRY(make_ws(ws, ws_bytes, 0, 64, 0, &w));
+  AVR_TRY(device_ok());
+  return cuda_status(launch_mma_rate(iters, grid, ns, w.status(), stream));
 }
 
 avr_status averis_probe_philox(uint64_t seed, uint64_t offset, uint32_t tag, int64_t n,

@@ -612,6 +612,86 @@ static cudaError_t launch_gemm_t(const GemmArgs& a, cudaStream_t s, bool pdl) {
   return launch_ex(kern, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmemBytes, s, pdl, ma, mb, msa, msb, msr, my, p);
 }
 
+// MMA-only loop: the tensor pipe's block-scaled FP4 rate on this device.
+// Each CTA (one per SM) fills shared memory with constant E2M1 codes and
+// E4M3 scales, copies the scales into tensor memory once, then issues `iters`
+// stages of four M 128 x N 256 x K 64 MMAs into one accumulator, waiting on
+// a commit every 16 stages; ns[b] = the CTA's elapsed time.  A measurement
+// aid for the roofline, not part of the method.
+__global__ void __launch_bounds__(128, 1) mma_rate_kernel(int iters, uint64_t* ns, uint32_t* status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) raise_status(status, AVR_ERR_MISALIGNED);
+    return;
+  }
+  uint8_t* sA = smem_raw;                 // 128 rows x 128 B
+  uint8_t* sB = sA + 16384;               // 256 rows x 128 B
+  uint8_t* sSF = sB + 32768;              // SFA 4 atoms, SFB 8 atoms
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sSF + 6144);
+  uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 1);
+  for (int i = threadIdx.x; i < (16384 + 32768) / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(sA)[i] = 0x22222222u;
+  for (int i = threadIdx.x; i < 6144 / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(sSF)[i] = 0x38383838u;
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbarrier_init();
+  }
+  fence_proxy_async_smem();
+  if (threadIdx.x < 32) {
+    tmem_alloc(slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *slot;
+  if (threadIdx.x == 0) {
+    constexpr uint32_t idesc = GemmCfg<256, true>::kIdesc;
+    const uint32_t sfa = tmem + 256, sfb = tmem + 272;
+    for (int kb = 0; kb < 4; ++kb) {
+      tc_cp_32x128b_warpx4(sfa + 4 * kb, smem_desc(smem_u32(sSF + kb * 512), 0, 128, kLayoutSwizzleNone));
+      for (int g = 0; g < 2; ++g)
+        tc_cp_32x128b_warpx4(sfb + 8 * kb + 4 * g,
+                             smem_desc(smem_u32(sSF + 2048 + (g * 4 + kb) * 512), 0, 128, kLayoutSwizzleNone));
+    }
+    tc_commit(bar);
+    uint32_t phase = 0;
+    bool ok = mbar_wait(bar, phase, status);
+    phase ^= 1u;
+    const uint64_t t0 = globaltimer_ns();
+    const uint64_t a0 = smem_desc(smem_u32(sA), 16, 1024, kLayoutSwizzle128B);
+    const uint64_t b0 = smem_desc(smem_u32(sB), 16, 1024, kLayoutSwizzle128B);
+    for (int it = 0; it < iters && ok; ++it) {
+#pragma unroll
+      for (int kb = 0; kb < 4; ++kb)
+        mma_nvf4(tmem, a0 + static_cast<uint64_t>(2 * kb), b0 + static_cast<uint64_t>(2 * kb), idesc, sfa + 4 * kb,
+                 sfb + 8 * kb, (it | kb) ? 1u : 0u);
+      if ((it & 15) == 15) {
+        tc_commit(bar);
+        ok = mbar_wait(bar, phase, status);
+        phase ^= 1u;
+      }
+    }
+    tc_commit(bar);
+    if (ok) mbar_wait(bar, phase, status);
+    ns[blockIdx.x] = globaltimer_ns() - t0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+cudaError_t launch_mma_rate(int iters, int grid, uint64_t* ns, uint32_t* status, cudaStream_t s) {
+  // more than half of the SM's shared memory, so one CTA per SM
+  constexpr int kSmem = 16384 + 32768 + 6144 + 64 + 64 * 1024;
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(mma_rate_kernel), kSmem);
+  if (e != cudaSuccess) return e;
+  mma_rate_kernel<<<grid, 128, kSmem, s>>>(iters, ns, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, bool pdl) {
   if (gemm_pair_applies(a)) return launch_gemm_pair(a, s, pdl);
   if (a.row_scale != nullptr) {

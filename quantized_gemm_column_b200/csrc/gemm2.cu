@@ -21,14 +21,14 @@
 // Roles (both CTAs have the same warps; CTA rank 0 of the pair leads):
 //   warp 0     : tensor-memory allocation (cta_group::2, in both CTAs); in
 //                the leading CTA one thread issues the pair's MMAs;
-//   warps 1..4 : TMA producers in both CTAs, one operand each (A rows, B
-//                rows, A's scale atoms, B's scale atoms for all 256 columns
-//                plus the resident ones).  Every copy completes on the
-//                leading CTA's barrier, whose producers expect the bytes of
-//                both CTAs;
-//   warp 5     : in the leading CTA, the scale copier (tcgen05.cp
+//   warps 1..8 : TMA producers in both CTAs, two per operand taking
+//                alternate stages (A rows, B rows, A's scale atoms, B's
+//                scale atoms for all 256 columns plus the resident ones).
+//                Every copy completes on the leading CTA's barrier, whose
+//                producers expect the bytes of both CTAs;
+//   warp 9     : in the leading CTA, the scale copier (tcgen05.cp
 //                cta_group::2: each CTA's atoms into its own tensor memory);
-//   warps 6..13: epilogue in both CTAs, each over its own 128 x 256
+//   warps 10..17: epilogue in both CTAs, each over its own 128 x 256
 //                accumulator: the bias row staged in shared memory,
 //                tcgen05.ld, alpha * acc + bias, bf16, TMA store.
 // The leading CTA's MMA commits signal both CTAs' barriers (multicast
@@ -64,18 +64,10 @@ __device__ __forceinline__ void cluster_sync_all() {
 }
 // arrive on an mbarrier given by its shared::cluster address (possibly another CTA's)
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
-// TMA 2-D load into this CTA's shared memory completing on the barrier at a
+// TMA 3-D load into this CTA's shared memory completing on the barrier at a
 // shared::cluster address in either CTA of the pair
-__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int32_t x,
-                                                 int32_t y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];"
-      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
-      : "memory");
-}
 __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int32_t x,
                                                  int32_t y, int32_t z) {
   asm volatile(
@@ -124,39 +116,45 @@ struct Gemm2Cfg {
   static constexpr int kBM = 128;                          // rows per CTA (256 per pair)
   static constexpr int kBN = 256;                          // columns per tile
   static constexpr int kBNHalf = kBN / 2;                  // B rows per CTA
-  static constexpr int kStageK = 256;
-  static constexpr int kRowBytes = kStageK / 2;
-  static constexpr int kStages = 4;
-  static constexpr int kKbPerStage = kStageK / 64;
+  static constexpr int kChunkK = 256;                      // K per 128-byte swizzled row chunk
+  static constexpr int kChunks = 1;                        // chunks per stage
+  static constexpr int kStageK = kChunkK * kChunks;        // 256
+  static constexpr int kStages = 5;
+  static constexpr int kKbPerStage = kStageK / 64;         // 4 MMAs per stage
   static constexpr int kEpiWarps = 8;
-  static constexpr int kFirstEpiWarp = 6;
+  static constexpr int kProducers = 8;                     // two per operand, alternate stages
+  static constexpr int kCopyWarp = 1 + kProducers;
+  static constexpr int kFirstEpiWarp = kCopyWarp + 1;
   static constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
-  static constexpr uint32_t kSbo = 8 * kRowBytes;
-  static constexpr int kABytes = kBM * kRowBytes;          // 16 KB
-  static constexpr int kBBytes = kBNHalf * kRowBytes;      // 16 KB
-  static constexpr int kSfaBytes = kKbPerStage * 512;      // 2 KB
-  static constexpr int kSfbBytes = 2 * kKbPerStage * 512;  // 4 KB: all 256 columns
+  static constexpr uint32_t kSbo = 8 * 128;                // 8-row swizzle atom of 128-byte rows
+  static constexpr int kAChunkBytes = kBM * 128;           // 16 KB
+  static constexpr int kABytes = kChunks * kAChunkBytes;   // 16 KB
+  static constexpr int kBChunkBytes = kBNHalf * 128;       // 16 KB
+  static constexpr int kBBytes = kChunks * kBChunkBytes;   // 16 KB
+  static constexpr int kSfaBytes = kKbPerStage * 512;      // 2 KB: 4 atoms
+  static constexpr int kSfbBytes = 2 * kKbPerStage * 512;  // 4 KB: [row group][4 atoms]
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
   static constexpr int kStageOutBytes = kBM * kBN * 2 / 2; // 32 KB: half the bf16 tile per round
-  // tensor memory (the same columns in both CTAs)
+  // tensor memory (the same columns in both CTAs): accumulator, A's scale
+  // slots (one per stage), then B's scales: all of K resident (K <= 1280,
+  // as many k-blocks as the streamed slots hold) or one slot per stage
   static constexpr int kAccCols = kBN;
-  static constexpr int kSfaCols = kKbPerStage * 4;
-  static constexpr int kSfbKbCols = kBN / 32;
-  static constexpr int kSfbCols = kKbPerStage * kSfbKbCols;
-  static constexpr int kSlots = 2;
-  static constexpr int kSlotCols = kSfaCols + kSfbCols;
-  static constexpr int kSlotCol = kAccCols;
-  static constexpr int kResCol = kSlotCol + kSlots * kSlotCols;
+  static constexpr int kSfaSlotCols = kKbPerStage * 4;     // 16
+  static constexpr int kSfaCol = kAccCols;
+  static constexpr int kSfbKbCols = kBN / 32;              // 8
+  static constexpr int kSfbStageCols = kKbPerStage * kSfbKbCols;   // 32
+  static constexpr int kSfbCol = kSfaCol + kStages * kSfaSlotCols; // 336
   static constexpr int kTmemCols = 512;
-  static constexpr int kResMaxStages = (kTmemCols - kResCol) / kSfbCols;   // 5
-  static constexpr int kResBytes = kResMaxStages * kSfbBytes;
-  // shared memory
+  static constexpr int kResAllStages = kStages;                    // resident: the slots' columns, K <= 1280
+  static constexpr int kStreamSlotCol = kSfbCol;
+  static_assert(kSfbCol + kStages * kSfbStageCols <= kTmemCols, "tensor memory budget");
+  // shared memory; the resident B scales reuse the per-stage B-scale buffers
+  // (contiguous, kStages * kSfbBytes), which resident mode does not stream into
   static constexpr int kOutOffset = kStages * kStageBytes;
   static constexpr int kResOffset = kOutOffset + kStageOutBytes;
-  static constexpr int kBiasOffset = kResOffset + kResBytes;
+  static constexpr int kBiasOffset = kResOffset;
   static constexpr int kBarOffset = kBiasOffset + kBN * 4;
   static constexpr int kSmemBytes = kBarOffset + 256;
-  static_assert(kResMaxStages >= 1, "tensor memory budget");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   // instruction descriptor: E2M1 A and B, UE4M3 scales, K-major, N >> 3 at
   // bit 17, M >> 4 at bit 24 (M = 256 for the pair)
@@ -167,7 +165,7 @@ struct Gemm2Cfg {
 struct Gemm2Params {
   int64_t M, N, K;
   int tiles_m, num_tiles;   // pair tiles of 256 x 256, M fastest
-  int res_stages;
+  int res_stages;           // stages whose B scales stay resident per column block (all of K, or 1)
   const float* gdec_a;
   const float* gdec_b;
   const float* bias;
@@ -177,8 +175,7 @@ struct Gemm2Params {
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 1)
     gemm2_nvfp4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                        const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
-                       const __grid_constant__ CUtensorMap map_sfb_res, const __grid_constant__ CUtensorMap map_y,
-                       const Gemm2Params p) {
+                       const __grid_constant__ CUtensorMap map_y, const Gemm2Params p) {
   using Cfg = Gemm2Cfg;
   constexpr int kEpiThreads = 32 * Cfg::kEpiWarps;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -191,13 +188,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
   uint8_t* sSfa = sB + Cfg::kStages * Cfg::kBBytes;
   uint8_t* sSfb = sSfa + Cfg::kStages * Cfg::kSfaBytes;
   uint8_t* sOut = smem + Cfg::kOutOffset;
-  uint8_t* sRes = smem + Cfg::kResOffset;      // [2 row groups][stage][4 atoms]
+  uint8_t* sRes = sSfb;                        // resident mode: [2 row groups][chunk][4 atoms]
   float* bias_s = reinterpret_cast<float*>(smem + Cfg::kBiasOffset);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOffset);  // [kStages] (used in the leading CTA)
-  uint64_t* empty = full + Cfg::kStages;        // [kStages] both CTAs
-  uint64_t* sf_full = empty + Cfg::kStages;     // [kSlots] leading CTA
-  uint64_t* sf_empty = sf_full + Cfg::kSlots;   // [kSlots] leading CTA
-  uint64_t* acc_full = sf_empty + Cfg::kSlots;  // both CTAs
+  uint64_t* full_ab = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOffset);  // [kStages] leading CTA: A, B landed
+  uint64_t* full_sf = full_ab + Cfg::kStages;   // [kStages] leading CTA: scale atoms landed
+  uint64_t* empty = full_sf + Cfg::kStages;     // [kStages] both CTAs
+  uint64_t* sf_full = empty + Cfg::kStages;     // [kStages] leading CTA: the stage's scales are in tensor memory
+  uint64_t* acc_full = sf_full + Cfg::kStages;  // both CTAs
   uint64_t* acc_empty = acc_full + 1;           // leading CTA: both epilogues arrive
   uint64_t* res_load = acc_empty + 1;           // leading CTA: resident scales landed in both CTAs
   uint64_t* res_cp = res_load + 1;              // both CTAs: resident scales copied
@@ -209,9 +206,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
   const uint32_t rank = cluster_ctarank();
   const bool lead = rank == 0;
   const int n_kst = static_cast<int>((p.K + Cfg::kStageK - 1) / Cfg::kStageK);
-  const int n_full = static_cast<int>(p.K / Cfg::kStageK);
-  const int tail_kb = static_cast<int>((p.K % Cfg::kStageK) / 64);
+  const int n_kb = static_cast<int>(p.K / 64);
   const int res_st = p.res_stages;
+  // B's scales of stage ks in tensor memory: resident, or a streamed slot
+  auto sfb_tmem_of = [&](uint32_t tmem, int ks, int st) -> uint32_t {
+    return ks < res_st ? tmem + Cfg::kSfbCol + Cfg::kSfbStageCols * ks
+                       : tmem + Cfg::kStreamSlotCol + Cfg::kSfbStageCols * st;
+  };
 
   if (threadIdx.x == 0) {
     if (!aligned) raise_status(p.status, AVR_ERR_MISALIGNED);
@@ -219,15 +220,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
     prefetch_tensormap(&map_b);
     prefetch_tensormap(&map_sfa);
     prefetch_tensormap(&map_sfb);
-    prefetch_tensormap(&map_sfb_res);
     prefetch_tensormap(&map_y);
     for (int s = 0; s < Cfg::kStages; ++s) {
-      mbar_init(&full[s], 4);                   // the leading CTA's four producers
+      mbar_init(&full_ab[s], 2);                // the leading CTA's A and B producers
+      mbar_init(&full_sf[s], 2);                // ... and its two scale producers
       mbar_init(&empty[s], 1);
-    }
-    for (int s = 0; s < Cfg::kSlots; ++s) {
       mbar_init(&sf_full[s], 1);
-      mbar_init(&sf_empty[s], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * Cfg::kEpiWarps);   // every epilogue warp of both CTAs
@@ -261,62 +259,68 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
   auto new_block = [&](int i) { return i == 0 || (first + i) / p.tiles_m != (first + i - 1) / p.tiles_m; };
   auto last_of_block = [&](int i) { return i + 1 == count || (first + i + 1) / p.tiles_m != (first + i) / p.tiles_m; };
   // barriers of the leading CTA, as shared::cluster addresses
-  const uint32_t full_lead = mapa_shared(smem_u32(full), 0);
+  const uint32_t full_ab_lead = mapa_shared(smem_u32(full_ab), 0);
+  const uint32_t full_sf_lead = mapa_shared(smem_u32(full_sf), 0);
   const uint32_t res_load_lead = mapa_shared(smem_u32(res_load), 0);
   const uint32_t acc_empty_lead = mapa_shared(smem_u32(acc_empty), 0);
 
-  if (warp >= 1 && warp <= 4) {
+  if (warp >= 1 && warp <= Cfg::kProducers) {
     if (lane == 0) {
-      // ---------------- producers: warp 1 A, 2 B, 3 A's scales, 4 B's scales (+ resident) ----------------
-      const int role = warp - 1;
-      uint32_t st = 0, ph = 0;
+      // ---------------- producers: A, B, A's scales, B's scales (+ resident) ----------------
+      // One copy per operand and stage.  A thread's copies complete one after
+      // another, so each operand has two threads, taking the even and the odd
+      // stages of the sequence.
+      const int role = (warp - 1) >> 1, parity = (warp - 1) & 1;
       int it = 0, res_uses = 0;
       bool ok = true;
       for (int i = 0; i < count && ok; ++i) {
         const int tile = first + i;
         const int32_t m0 = (tile % p.tiles_m) * (2 * Cfg::kBM) + static_cast<int32_t>(rank) * Cfg::kBM;
         const int32_t n0 = (tile / p.tiles_m) * Cfg::kBN;
-        if (role == 3 && res_st > 0 && new_block(i)) {
+        if (role == 3 && parity == 0 && res_st > 0 && new_block(i)) {
           // both CTAs' resident buffers are free once the previous block's copies ran
-          if (res_uses >= 1 && !mbar_wait(res_cp, static_cast<uint32_t>(res_uses - 1) & 1u, p.status)) break;
+          if (res_uses >= 1 && !mbar_wait_poll(res_cp, static_cast<uint32_t>(res_uses - 1) & 1u, p.status)) break;
           ++res_uses;
           if (lead) mbar_arrive_expect_tx(res_load, static_cast<uint32_t>(2 * res_st * Cfg::kSfbBytes));
-          tma_load_3d_pair(sRes, &map_sfb_res, res_load_lead, 0, 0, n0 / 128);
+          // box of res_st * 2 chunks: this launch's B-scale map is sized for it (see the launch)
+          tma_load_3d_pair(sRes, &map_sfb, res_load_lead, 0, 0, n0 / 128);
         }
         for (int ks = 0; ks < n_kst; ++ks, ++it) {
-          if (it >= Cfg::kStages && !mbar_wait(&empty[st], ph ^ 1u, p.status)) {
+          if ((it & 1) != parity) continue;
+          const uint32_t st = static_cast<uint32_t>(it % Cfg::kStages);
+          const uint32_t ph = static_cast<uint32_t>(it / Cfg::kStages) & 1u;
+          if (it >= Cfg::kStages && !mbar_wait_poll(&empty[st], ph ^ 1u, p.status)) {
             ok = false;
             break;
           }
-          const uint32_t bar = full_lead + static_cast<uint32_t>(st * 8);
+          const uint32_t bar_ab = full_ab_lead + static_cast<uint32_t>(st * 8);
+          const uint32_t bar_sf = full_sf_lead + static_cast<uint32_t>(st * 8);
           if (role == 0) {
-            if (lead) mbar_arrive_expect_tx(&full[st], 2 * Cfg::kABytes);
-            tma_load_2d_pair(sA + st * Cfg::kABytes, &map_a, bar, ks * Cfg::kRowBytes, m0);
+            if (lead) mbar_arrive_expect_tx(&full_ab[st], 2 * Cfg::kABytes);
+            tma_load_3d_pair(sA + st * Cfg::kABytes, &map_a, bar_ab, 0, m0, Cfg::kChunks * ks);
           } else if (role == 1) {
-            if (lead) mbar_arrive_expect_tx(&full[st], 2 * Cfg::kBBytes);
-            tma_load_2d_pair(sB + st * Cfg::kBBytes, &map_b, bar, ks * Cfg::kRowBytes,
-                             n0 + static_cast<int32_t>(rank) * Cfg::kBNHalf);
+            if (lead) mbar_arrive_expect_tx(&full_ab[st], 2 * Cfg::kBBytes);
+            tma_load_3d_pair(sB + st * Cfg::kBBytes, &map_b, bar_ab, 0, n0 + static_cast<int32_t>(rank) * Cfg::kBNHalf,
+                             Cfg::kChunks * ks);
           } else if (role == 2) {
-            if (lead) mbar_arrive_expect_tx(&full[st], 2 * Cfg::kSfaBytes);
-            tma_load_2d_pair(sSfa + st * Cfg::kSfaBytes, &map_sfa, bar, ks * 256, m0 / 128);
+            if (lead) mbar_arrive_expect_tx(&full_sf[st], 2 * Cfg::kSfaBytes);
+            tma_load_3d_pair(sSfa + st * Cfg::kSfaBytes, &map_sfa, bar_sf, 0, Cfg::kChunks * ks, m0 / 128);
           } else if (ks >= res_st) {
-            if (lead) mbar_arrive_expect_tx(&full[st], 2 * Cfg::kSfbBytes);
-            tma_load_2d_pair(sSfb + st * Cfg::kSfbBytes, &map_sfb, bar, ks * 256, n0 / 128);
+            if (lead) mbar_arrive_expect_tx(&full_sf[st], 2 * Cfg::kSfbBytes);
+            tma_load_3d_pair(sSfb + st * Cfg::kSfbBytes, &map_sfb, bar_sf, 0, Cfg::kChunks * ks, n0 / 128);
           } else if (lead) {
-            mbar_arrive(&full[st]);               // this stage's B scales are resident
-          }
-          if (++st == Cfg::kStages) {
-            st = 0;
-            ph ^= 1u;
+            mbar_arrive(&full_sf[st]);            // this stage's B scales are resident
           }
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == Cfg::kCopyWarp) {
     if (lead && lane == 0) {
       // ---------------- scale copier (leading CTA; each copy fills both CTAs) ----------------
-      uint32_t st = 0, ph = 0, sl = 0, sph = 0;
-      int it = 0, res_uses = 0;
+      // Stage ks's copies go to the slots of its stage buffer st: the slot's
+      // previous MMAs completed before the stage was refilled.
+      uint32_t st = 0, ph = 0;
+      int res_uses = 0;
       bool ok = true;
       const uint64_t res_d = smem_desc(smem_u32(sRes), 0, 128, kLayoutSwizzleNone);
       for (int i = 0; i < count && ok; ++i) {
@@ -325,48 +329,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
           if (!mbar_wait_poll(res_load, static_cast<uint32_t>(res_uses) & 1u, p.status)) break;
           ++res_uses;
           tc_fence_after();
-          for (int ks = 0; ks < res_st; ++ks)
+          // sRes: [group g][k-block kb of the resident stages], 512 bytes each
+          const int res_kb = min(res_st * Cfg::kKbPerStage, n_kb);
+          for (int kb = 0; kb < res_kb; ++kb)
 #pragma unroll
-            for (int kb = 0; kb < Cfg::kKbPerStage; ++kb)
-#pragma unroll
-              for (int g = 0; g < 2; ++g)
-                tc_cp_32x128b_warpx4_pair(tmem + Cfg::kResCol + Cfg::kSfbKbCols * (ks * Cfg::kKbPerStage + kb) + 4 * g,
-                                          res_d + static_cast<uint64_t>(32 * ((g * res_st + ks) * Cfg::kKbPerStage + kb)));
+            for (int g = 0; g < 2; ++g)
+              tc_cp_32x128b_warpx4_pair(tmem + Cfg::kSfbCol + Cfg::kSfbKbCols * kb + 4 * g,
+                                        res_d + static_cast<uint64_t>(32 * (g * res_st * Cfg::kKbPerStage + kb)));
           tc_commit_pair_both(res_cp);
         }
-        for (int ks = 0; ks < n_kst; ++ks, ++it) {
-          if (!mbar_wait_poll(&full[st], ph, p.status)) {
-            ok = false;
-            break;
-          }
-          if (it >= Cfg::kSlots && !mbar_wait_poll(&sf_empty[sl], sph ^ 1u, p.status)) {
+        for (int ks = 0; ks < n_kst; ++ks) {
+          if (!mbar_wait_poll(&full_sf[st], ph, p.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sfa_t = tmem + Cfg::kSlotCol + sl * Cfg::kSlotCols;
-          const uint32_t sfb_t = sfa_t + Cfg::kSfaCols;
+          const uint32_t sfa_t = tmem + Cfg::kSfaCol + Cfg::kSfaSlotCols * st;
           const uint64_t sfa_d = smem_desc(smem_u32(sSfa + st * Cfg::kSfaBytes), 0, 128, kLayoutSwizzleNone);
           const uint64_t sfb_d = smem_desc(smem_u32(sSfb + st * Cfg::kSfbBytes), 0, 128, kLayoutSwizzleNone);
-          const bool sfb = ks >= res_st;
-          const int nkb = ks < n_full ? Cfg::kKbPerStage : tail_kb;
-          for (int kb = 0; kb < nkb; ++kb) {
-            tc_cp_32x128b_warpx4_pair(sfa_t + 4 * kb, sfa_d + static_cast<uint64_t>(32 * kb));
-            if (sfb) {
+          const int nkb = min(Cfg::kKbPerStage, n_kb - ks * Cfg::kKbPerStage);
+          for (int kb = 0; kb < nkb; ++kb) tc_cp_32x128b_warpx4_pair(sfa_t + 4 * kb, sfa_d + static_cast<uint64_t>(32 * kb));
+          if (ks >= res_st) {
+            const uint32_t sfb_t = sfb_tmem_of(tmem, ks, static_cast<int>(st));
+            for (int kb = 0; kb < nkb; ++kb)
 #pragma unroll
               for (int g = 0; g < 2; ++g)
                 tc_cp_32x128b_warpx4_pair(sfb_t + Cfg::kSfbKbCols * kb + 4 * g,
                                           sfb_d + static_cast<uint64_t>(32 * (g * Cfg::kKbPerStage + kb)));
-            }
           }
-          tc_commit_pair(&sf_full[sl]);
+          tc_commit_pair(&sf_full[st]);
           if (++st == Cfg::kStages) {
             st = 0;
             ph ^= 1u;
-          }
-          if (++sl == Cfg::kSlots) {
-            sl = 0;
-            sph ^= 1u;
           }
         }
       }
@@ -376,7 +370,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
   } else if (warp == 0) {
     if (lead && lane == 0) {
       // ---------------- MMA issuer (leading CTA) ----------------
-      uint32_t st = 0, ph = 0, sl = 0, sph = 0;
+      uint32_t st = 0, ph = 0;
       int res_uses = 0;
       bool ok = true;
       for (int i = 0; i < count && ok; ++i) {
@@ -385,7 +379,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
           ++res_uses;
         }
         for (int ks = 0; ks < n_kst; ++ks) {
-          if (!mbar_wait_poll(&sf_full[sl], sph, p.status) || !mbar_wait_poll(&full[st], ph, p.status)) {
+          if (!mbar_wait_poll(&sf_full[st], ph, p.status) || !mbar_wait_poll(&full_ab[st], ph, p.status)) {
             ok = false;
             break;
           }
@@ -394,30 +388,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
             break;
           }
           tc_fence_after();
-          const uint32_t sfa_t = tmem + Cfg::kSlotCol + sl * Cfg::kSlotCols;
-          const uint32_t sfb_t = ks < res_st ? tmem + Cfg::kResCol + Cfg::kSfbKbCols * (ks * Cfg::kKbPerStage)
-                                             : sfa_t + Cfg::kSfaCols;
+          const uint32_t sfa_t = tmem + Cfg::kSfaCol + Cfg::kSfaSlotCols * st;
+          const uint32_t sfb_t = sfb_tmem_of(tmem, ks, static_cast<int>(st));
+          // k-block kb: chunk kb / 4 (16 KB tiles), 32-byte step kb % 4 inside it
           const uint64_t a0 = smem_desc(smem_u32(sA + st * Cfg::kABytes), 16, Cfg::kSbo, kLayoutSwizzle128B);
           const uint64_t b0 = smem_desc(smem_u32(sB + st * Cfg::kBBytes), 16, Cfg::kSbo, kLayoutSwizzle128B);
-          if (ks < n_full) {
+          const int nkb = min(Cfg::kKbPerStage, n_kb - ks * Cfg::kKbPerStage);
+          if (nkb == Cfg::kKbPerStage) {
 #pragma unroll
-            for (int kb = 0; kb < Cfg::kKbPerStage; ++kb)
-              mma_nvf4_pair(tmem, a0 + static_cast<uint64_t>(2 * kb), b0 + static_cast<uint64_t>(2 * kb), Cfg::kIdesc,
-                            sfa_t + 4 * kb, sfb_t + Cfg::kSfbKbCols * kb, (ks > 0 || kb > 0) ? 1u : 0u);
+            for (int kb = 0; kb < Cfg::kKbPerStage; ++kb) {
+              const uint64_t step = static_cast<uint64_t>((kb >> 2) * (Cfg::kAChunkBytes >> 4) + 2 * (kb & 3));
+              const uint64_t stepb = static_cast<uint64_t>((kb >> 2) * (Cfg::kBChunkBytes >> 4) + 2 * (kb & 3));
+              mma_nvf4_pair(tmem, a0 + step, b0 + stepb, Cfg::kIdesc, sfa_t + 4 * kb, sfb_t + Cfg::kSfbKbCols * kb,
+                            (ks > 0 || kb > 0) ? 1u : 0u);
+            }
           } else {
-            for (int kb = 0; kb < tail_kb; ++kb)
-              mma_nvf4_pair(tmem, a0 + static_cast<uint64_t>(2 * kb), b0 + static_cast<uint64_t>(2 * kb), Cfg::kIdesc,
-                            sfa_t + 4 * kb, sfb_t + Cfg::kSfbKbCols * kb, (ks > 0 || kb > 0) ? 1u : 0u);
+            for (int kb = 0; kb < nkb; ++kb) {
+              const uint64_t step = static_cast<uint64_t>((kb >> 2) * (Cfg::kAChunkBytes >> 4) + 2 * (kb & 3));
+              const uint64_t stepb = static_cast<uint64_t>((kb >> 2) * (Cfg::kBChunkBytes >> 4) + 2 * (kb & 3));
+              mma_nvf4_pair(tmem, a0 + step, b0 + stepb, Cfg::kIdesc, sfa_t + 4 * kb, sfb_t + Cfg::kSfbKbCols * kb,
+                            (ks > 0 || kb > 0) ? 1u : 0u);
+            }
           }
           tc_commit_pair_both(&empty[st]);        // both CTAs' producers may refill the stage
-          tc_commit_pair(&sf_empty[sl]);
           if (++st == Cfg::kStages) {
             st = 0;
             ph ^= 1u;
-          }
-          if (++sl == Cfg::kSlots) {
-            sl = 0;
-            sph ^= 1u;
           }
         }
         if (!ok) break;
@@ -429,6 +425,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
     }
   } else {
     // ---------------- epilogue (both CTAs, own rows) ----------------
+    // The whole 128-column slice of a warp is taken out of tensor memory and
+    // packed to bf16 in registers, chunk by chunk, before the accumulator is
+    // handed back; only then is it staged and stored.
     const int ew = warp - Cfg::kFirstEpiWarp;
     const int q = warp & 3;                    // lane quarter of tensor memory this warp may read
     const int h = ew / 4;                      // which 128-column half
@@ -451,15 +450,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
       if (named_barrier_or(1, kEpiThreads, !ok)) break;
       tc_fence_after();
       const uint32_t t_row = tmem + (static_cast<uint32_t>(32 * q) << 16);
-      auto pack_bf16 = [&](int c, const uint32_t (&v)[32], uint32_t (&w)[16]) {
+      // chunk c of this warp's four: alpha * acc + bias as 16 bf16 pairs
+      auto load_pack = [&](int c, uint32_t (&w)[16]) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(32 * (4 * h + c)), v);
+        tmem_ld_wait();
         const float* b = bias_s + 32 * (4 * h + c);
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          const __nv_bfloat162 pr = __floats2bfloat162_rn(fmaf(alpha, __uint_as_float(v[2 * k]), b[2 * k]),
-                                                          fmaf(alpha, __uint_as_float(v[2 * k + 1]), b[2 * k + 1]));
+          const float2 bb = *reinterpret_cast<const float2*>(b + 2 * k);
+          const __nv_bfloat162 pr = __floats2bfloat162_rn(fmaf(alpha, __uint_as_float(v[2 * k]), bb.x),
+                                                          fmaf(alpha, __uint_as_float(v[2 * k + 1]), bb.y));
           w[k] = *reinterpret_cast<const uint32_t*>(&pr);
         }
       };
+      // 16 bf16 pairs of chunk c = 64 bytes = four 16-byte pieces of row r in
+      // box h of the staging buffer (a box is 128 rows x 64 columns)
       auto stage_bf16 = [&](int c, const uint32_t (&w)[16]) {
         uint8_t* box = sOut + h * (Cfg::kBM * 128);
 #pragma unroll
@@ -483,27 +489,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
           bulk_commit_group();
         }
       };
-      uint32_t v0[32], v1[32];
-      tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(32 * (4 * h + 0)), v0);
-      tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(32 * (4 * h + 1)), v1);
-      tmem_ld_wait();
+      // round 0's chunks go straight to the (free) staging buffer; round 1's
+      // stay in registers; the accumulator goes back to the leading CTA's MMA
+      // thread as soon as the last chunk is out of tensor memory
       {
         uint32_t w[16];
-        pack_bf16(0, v0, w);
+        load_pack(0, w);
         stage_bf16(0, w);
-        pack_bf16(1, v1, w);
+        load_pack(1, w);
         stage_bf16(1, w);
       }
-      tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(32 * (4 * h + 2)), v0);
-      tmem_ld_32x32b_x32(t_row + static_cast<uint32_t>(32 * (4 * h + 3)), v1);
-      tmem_ld_wait();
-      // the accumulator goes back to the leading CTA's MMA thread
+      uint32_t w2[16], w3[16];
+      load_pack(2, w2);
+      load_pack(3, w3);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty_lead);
-      uint32_t w2[16], w3[16];
-      pack_bf16(2, v0, w2);
-      pack_bf16(3, v1, w3);
       store_round(0);
       if (store_thr) bulk_wait_group_read<0>();
       named_barrier(1, kEpiThreads);
@@ -543,39 +544,44 @@ static int resident_pairs() {
   return n;
 }
 
-// The pair kernel serves dense bf16 outputs; its tiles are 256 rows x 256 columns.
+// The pair kernel serves dense bf16 outputs with K a multiple of 256 (its
+// operand copies take whole 256-deep chunks); its tiles are 256 x 256.
 bool gemm_pair_applies(const GemmArgs& a) {
-  return a.yt == AVR_BF16 && a.block_expert == nullptr && a.row_scale == nullptr && a.groups == 1;
+  return a.yt == AVR_BF16 && a.block_expert == nullptr && a.row_scale == nullptr && a.groups == 1 && a.K % 256 == 0;
+}
+
+// [rows, K/2 bytes] codes as a 3-D tensor (128 bytes, rows, K/256 chunks):
+// a box of (128, box_rows, 2) brings two 128-byte-swizzled chunk tiles
+static bool codes_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, uint32_t box_rows) {
+  const uint64_t dims[3] = {128, static_cast<uint64_t>(rows), static_cast<uint64_t>(K / 256)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(K / 2), 128};
+  const uint32_t box[3] = {128, box_rows, static_cast<uint32_t>(Gemm2Cfg::kChunks)};
+  return make_tensor_map_3d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+// scale atoms as a 3-D tensor of 8-byte elements (256 = one chunk's 4
+// atoms, K/256 chunks, row groups of 128)
+static bool scales_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, uint32_t box_chunks,
+                       uint32_t box_groups) {
+  const uint64_t dims[3] = {256, static_cast<uint64_t>(K / 256), static_cast<uint64_t>((rows + 127) / 128)};
+  const uint64_t strides[2] = {2048, static_cast<uint64_t>(K / 64) * 512};
+  const uint32_t box[3] = {256, box_chunks, box_groups};
+  return make_tensor_map_3d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT64, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s, bool pdl) {
   using Cfg = Gemm2Cfg;
-  constexpr CUtensorMapSwizzle kOpSwizzle = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!gemm_pair_applies(a)) return cudaErrorInvalidValue;
+  const int n_kst = static_cast<int>((a.K + Cfg::kStageK - 1) / Cfg::kStageK);
+  // B's scales: all of K resident when they fit, else streamed per stage
+  const int res_stages = n_kst <= Cfg::kResAllStages ? n_kst : 0;
   CUtensorMap ma, mb, msa, msb, my;
-  if (!make_tensor_map_2d(&ma, a.a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(a.M),
-                          static_cast<uint64_t>(a.K / 2), Cfg::kBM, Cfg::kRowBytes, kOpSwizzle))
+  if (!codes_map(&ma, a.a_codes, a.M, a.K, Cfg::kBM) || !codes_map(&mb, a.b_codes, a.N, a.K, Cfg::kBNHalf) ||
+      !scales_map(&msa, a.a_scales, a.M, a.K, Cfg::kChunks, 1))
     return cudaErrorInvalidValue;
-  if (!make_tensor_map_2d(&mb, a.b_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(a.N),
-                          static_cast<uint64_t>(a.K / 2), Cfg::kBNHalf, Cfg::kRowBytes, kOpSwizzle))
+  // one map for B's scales: its box is the resident block (res_stages stages
+  // of both row groups) when every stage is resident, else one stage
+  if (!scales_map(&msb, a.b_scales, a.N, a.K, static_cast<uint32_t>(Cfg::kChunks * (res_stages > 0 ? res_stages : 1)), 2))
     return cudaErrorInvalidValue;
-  const uint64_t sf_cols = static_cast<uint64_t>(a.K / 64) * 64;
-  if (!make_tensor_map_2d(&msa, a.a_scales, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, static_cast<uint64_t>((a.M + 127) / 128),
-                          sf_cols, 1, 256, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return cudaErrorInvalidValue;
-  const uint64_t b_groups = static_cast<uint64_t>((a.N + 127) / 128);
-  if (!make_tensor_map_2d(&msb, a.b_scales, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, b_groups, sf_cols, 2, 256,
-                          CU_TENSOR_MAP_SWIZZLE_NONE))
-    return cudaErrorInvalidValue;
-  const int64_t n_full = a.K / Cfg::kStageK;
-  const int res_stages = static_cast<int>(min64(n_full, Cfg::kResMaxStages));
-  CUtensorMap msr = msb;
-  if (res_stages > 0) {
-    const uint64_t dims[3] = {256, static_cast<uint64_t>(n_full), b_groups};
-    const uint64_t strides[2] = {2048, sf_cols * 8};
-    const uint32_t box[3] = {256, static_cast<uint32_t>(res_stages), 2};
-    if (!make_tensor_map_3d(&msr, a.b_scales, CU_TENSOR_MAP_DATA_TYPE_UINT64, dims, strides, box))
-      return cudaErrorInvalidValue;
-  }
   if (!make_tensor_map_2d(&my, a.Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, static_cast<uint64_t>(a.M),
                           static_cast<uint64_t>(a.N), Cfg::kBM, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
@@ -597,7 +603,7 @@ cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s, bool pdl) {
   const int max_pairs = resident_pairs();
   const int pairs = p.num_tiles < max_pairs ? p.num_tiles : max_pairs;
   return launch_ex(gemm2_nvfp4_kernel, dim3(2 * pairs), dim3(Cfg::kThreads), Cfg::kSmemBytes, s, pdl, ma, mb, msa,
-                   msb, msr, my, p);
+                   msb, my, p);
 }
 
 }  // namespace avr

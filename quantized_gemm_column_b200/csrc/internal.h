@@ -277,6 +277,7 @@ cudaError_t launch_probe_convert(const float* in, uint8_t* e4m3, uint8_t* e2m1, 
                                  cudaStream_t s);
 cudaError_t launch_probe_convert_sr(const float* in, const uint32_t* rbits, uint16_t* out, int64_t n,
                                     cudaStream_t s);
+cudaError_t launch_mma_rate(int iters, int grid, uint64_t* ns, uint32_t* status, cudaStream_t s);
 cudaError_t launch_probe_philox(uint64_t seed, uint64_t offset, uint32_t tag, int64_t n,
                                 uint32_t* out, cudaStream_t s);
 
@@ -287,9 +288,10 @@ bool make_tensor_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType 
                         uint32_t box_cols, CUtensorMapSwizzle swizzle);
 
 // 3-D tensor of elem-sized elements: dims[0] contiguous, byte strides of
-// dims 1 and 2; no swizzle.
+// dims 1 and 2.
 bool make_tensor_map_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, const uint64_t dims[3],
-                        const uint64_t strides[2], const uint32_t box[3]);
+                        const uint64_t strides[2], const uint32_t box[3],
+                        CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE);
 
 // cudaFuncAttributeMaxDynamicSharedMemorySize for the current device (set
 // once per device and function).

@@ -34,48 +34,55 @@ def _gemm(api, a_q, b_q, bias=None, out=torch.float32):
     return Y.float().cpu().numpy().astype(np.float64)
 
 
-@pytest.mark.parametrize("out", [torch.float32, torch.bfloat16])
-def test_scale_layout_probe_A(api, out):
+# bf16 outputs with K a multiple of 256 run on the CTA-pair kernel, the
+# others on the one-CTA kernel: the probes run at K = 64 and 256 to cover both.
+KERNELS = [(torch.float32, 64), (torch.bfloat16, 64), (torch.bfloat16, 256)]
+
+
+@pytest.mark.parametrize("out,K", KERNELS)
+def test_scale_layout_probe_A(api, out, K):
     """A has every code 1.0 and random E4M3 scales; row j of B is 1.0 on the
-    16-block (j mod 4) of a 64-wide K and 0 elsewhere, with scale 1.  Then
-    Y[r, j] = 16 * scale_A[r, j mod 4] exactly: each output names one scale
+    16-block (j mod K/16) of K and 0 elsewhere, with scale 1.  Then
+    Y[r, j] = 16 * scale_A[r, j mod K/16] exactly: each output names one scale
     of A, so a wrong tensor-memory scale layout cannot pass."""
     rng = np.random.default_rng(0)
-    M, K, N = 256, 64, 64
+    M, N = 256, 64
+    nb = K // 16
     a = F.NVFP4(F.pack_codes(np.full((M, K), 2, np.uint8)),
                 rng.integers(0x20, 0x58, (M, K // 16)).astype(np.uint8), np.float32(1.0), M, K)
     bc = np.zeros((N, K), np.uint8)
     for j in range(N):
-        bc[j, 16 * (j % 4):16 * (j % 4) + 16] = 2
+        bc[j, 16 * (j % nb):16 * (j % nb) + 16] = 2
     b = F.NVFP4(F.pack_codes(bc), np.full((N, K // 16), 0x38, np.uint8), np.float32(1.0), N, K)
     Y = _gemm(api, a, b, out=out)
-    want = 16.0 * oracle.e4m3_value(a.scales).astype(np.float64)[:, np.arange(N) % 4]
+    want = 16.0 * oracle.e4m3_value(a.scales).astype(np.float64)[:, np.arange(N) % nb]
     assert np.array_equal(Y, want)
 
 
-@pytest.mark.parametrize("out", [torch.float32, torch.bfloat16])
-def test_scale_layout_probe_B(api, out):
-    """The same with the roles swapped: Y[i, j] = 16 * scale_B[j, i mod 4]
+@pytest.mark.parametrize("out,K", KERNELS)
+def test_scale_layout_probe_B(api, out, K):
+    """The same with the roles swapped: Y[i, j] = 16 * scale_B[j, i mod K/16]
     for N = 256 (two 128-row scale atoms of B)."""
     rng = np.random.default_rng(1)
-    M, K, N = 128, 64, 256
+    M, N = 256, 256
+    nb = K // 16
     ac = np.zeros((M, K), np.uint8)
     for i in range(M):
-        ac[i, 16 * (i % 4):16 * (i % 4) + 16] = 2
+        ac[i, 16 * (i % nb):16 * (i % nb) + 16] = 2
     a = F.NVFP4(F.pack_codes(ac), np.full((M, K // 16), 0x38, np.uint8), np.float32(1.0), M, K)
     b = F.NVFP4(F.pack_codes(np.full((N, K), 2, np.uint8)),
                 rng.integers(0x20, 0x58, (N, K // 16)).astype(np.uint8), np.float32(1.0), N, K)
     Y = _gemm(api, a, b, out=out)
-    want = 16.0 * oracle.e4m3_value(b.scales).astype(np.float64)[:, np.arange(M) % 4].T
+    want = 16.0 * oracle.e4m3_value(b.scales).astype(np.float64)[:, np.arange(M) % nb].T
     assert np.array_equal(Y, want)
 
 
-@pytest.mark.parametrize("out", [torch.float32, torch.bfloat16])
-def test_nibble_order_probe(api, out):
+@pytest.mark.parametrize("out,K", KERNELS)
+def test_nibble_order_probe(api, out, K):
     """Row j of B is one-hot at element j: Y[r, j] = value of A's element
     (r, j), so a swapped nibble order shows at every odd j."""
     rng = np.random.default_rng(2)
-    M, K = 128, 64
+    M = 256
     ac = rng.integers(0, 16, (M, K)).astype(np.uint8)
     a = F.NVFP4(F.pack_codes(ac), np.full((M, K // 16), 0x38, np.uint8), np.float32(1.0), M, K)
     bc = np.zeros((K, K), np.uint8)
@@ -85,14 +92,17 @@ def test_nibble_order_probe(api, out):
     assert np.array_equal(Y, oracle.e2m1_value(ac).astype(np.float64))
 
 
-@pytest.mark.parametrize("out", [torch.float32, torch.bfloat16])
-def test_k_stage_and_kblock_order(api, out):
+@pytest.mark.parametrize("out,K", [(torch.float32, 640), (torch.bfloat16, 640), (torch.bfloat16, 1280),
+                                   (torch.bfloat16, 2304)])
+def test_k_stage_and_kblock_order(api, out, K):
     """Each 64-element k-block of A holds one constant per row and row j of B
-    selects k-block j mod 10, so Y[:, j] = 64 * that constant: a wrong k
-    advance inside a stage or across stages (K = 640 leaves a partial last
-    stage) changes the products.  All values are exact in fp32 and bf16."""
+    selects k-block j mod K/64, so Y[:, j] = 64 * that constant: a wrong k
+    advance inside a stage or across stages changes the products.  K = 640
+    leaves the one-CTA kernel a partial last stage; 1280 gives the pair kernel
+    a last stage of one 256-deep chunk with all of B's scales resident, 2304
+    the same with B's scales streamed.  All values are exact in fp32 and bf16."""
     rng = np.random.default_rng(3)
-    M, K = 128, 640
+    M = 256
     nkb = K // 64
     ac = np.zeros((M, K), np.uint8)
     for kb in range(nkb):
@@ -101,7 +111,7 @@ def test_k_stage_and_kblock_order(api, out):
     N = 64
     bc = np.zeros((N, K), np.uint8)
     for j in range(N):
-        kb = j % nkb
+        kb = (j * 7) % nkb
         bc[j, 64 * kb:64 * kb + 64] = 2
     b = F.NVFP4(F.pack_codes(bc), np.full((N, K // 16), 0x38, np.uint8), np.float32(1.0), N, K)
     Y = _gemm(api, a, b, out=out)
@@ -153,14 +163,17 @@ def _gemm_sampled(api, a_q, b_q, cols, bias=None, out=torch.float32):
     return Y[:, cols], ref, b_sub
 
 
-@pytest.mark.parametrize("K", [256, 1280, 1536, 2112])
+@pytest.mark.parametrize("K", [256, 1280, 1536, 2112, 2048, 2304])
 def test_resident_b_scales_across_column_blocks_bf16(api, K):
-    """Many more tiles than CTAs with two row blocks, so a CTA's run of tiles
-    changes column block (B's resident scales are reloaded) and shares it
-    between tiles.  K = 256 and 1280 keep every stage's B scales resident,
-    1536 five of six, 2112 five of nine with a partial last stage."""
+    """Many more tiles than CTAs (or CTA pairs), so a run of tiles changes
+    column block (B's resident scales are reloaded) and shares it between
+    tiles.  The pair kernel (K a multiple of 256) keeps all of B's scales
+    resident up to K = 1536 (256, 1280: a last stage of one chunk) and
+    streams them past one resident stage beyond (2048, 2304: a last stage of
+    one chunk); K = 2112 runs the one-CTA kernel (five of nine stages
+    resident, a partial last stage)."""
     rng = np.random.default_rng(K)
-    M, N = 256, 256 * 160
+    M, N = 512, 256 * 160
     a = _rand_q(rng, M, K, g_dec=0.01)
     b = _rand_q(rng, N, K, g_dec=0.003)
     bias = rng.standard_normal(N) * 0.1

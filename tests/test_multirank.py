@@ -86,16 +86,18 @@ def test_reference_arm_under_torchrun(tmp_path):
 
 
 def test_measured_traffic_follows_kernel_sources(tmp_path, monkeypatch):
-    """The roofline's DRAM traffic comes from the committed ncu summary only
-    while the kernel sources hash to the digest it records."""
+    """The roofline's DRAM traffic comes from the committed ncu capture
+    (a JSON record) only while the kernel sources hash to the digest it
+    records."""
     import bench
-    prof = tmp_path / "traffic.md"
-    prof.write_text(f"    traffic-digest: {bench.kernel_digest()}\n"
-                    "    traffic-split-quant-bytes-per-step: 123\n")
+    prof = tmp_path / "traffic.json"
+    prof.write_text(json.dumps({"digest": bench.kernel_digest(), "bytes_per_step": {"split-quant": 123}}))
     monkeypatch.setattr(bench, "TRAFFIC_PROFILE", str(prof))
     assert bench.measured_traffic("split-quant") == 123
     assert bench.measured_traffic("gemm") is None
-    prof.write_text("    traffic-digest: 0000000000000000\n    traffic-split-quant-bytes-per-step: 123\n")
+    prof.write_text(json.dumps({"digest": "0000000000000000", "bytes_per_step": {"split-quant": 123}}))
+    assert bench.measured_traffic("split-quant") is None
+    prof.write_text("not json")
     assert bench.measured_traffic("split-quant") is None
 
 
