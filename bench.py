@@ -50,6 +50,9 @@ def parse():
     p.add_argument("--cpu-sample-rows", type=int, default=8192)
     p.add_argument("--cpu-sample-steps", type=int, default=2)
     p.add_argument("--copies", type=int, default=4, help="input copies rotated between steps")
+    p.add_argument("--case", choices=["qkv"], default=None,
+                   help="profiling case: the QKV step's kernels alone (weight quantization, then --steps Averis "
+                        "and --steps vanilla fwd + dgrad steps, eager launches), no timing and no JSON line")
     return p.parse_args()
 
 
@@ -578,6 +581,38 @@ def job_value(flops_per_step, world, step_ms):
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
+def run_case(args):
+    """The QKV step's launches alone, for ncu captures: the weight
+    quantization once, then args.warmup + args.steps Averis steps and as many
+    vanilla steps (eager launches on one stream, inputs rotating over
+    args.copies copies); the device status is checked at the end."""
+    import torch
+    from quantized_gemm_column_b200 import api, inputs
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    api.load()
+    X0, W0, D0 = inputs.workload1()
+    copies = max(1, args.copies)
+    Xs = [X0.to(dev) for _ in range(copies)]
+    Ds = [D0.to(dev) for _ in range(copies)]
+    Wd = W0.to(dev)
+    w_fwd, w_dgrad = api.NVFP4Tensor(N, M, dev), api.NVFP4Tensor(M, N, dev)
+    ws = api.workspace(L, N, N, dev)
+    Y = torch.empty((L, N), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((L, M), dtype=torch.bfloat16, device=dev)
+    torch.cuda.synchronize(dev)
+    api.averis_quant_weight(Wd, w_fwd, w_dgrad, ws)
+    for i in range(args.warmup + args.steps):
+        api.averis_linear_fwd(Xs[i % copies], w_fwd, "sr", 1 + i, 0, Y, ws)
+        api.averis_linear_dgrad(Ds[i % copies], w_dgrad, "sr", 1 + i, 0, dX, ws)
+    for i in range(args.warmup + args.steps):
+        api.nvfp4_linear_fwd(Xs[i % copies], w_fwd, "sr", 1 + i, 0, Y, ws)
+        api.nvfp4_linear_dgrad(Ds[i % copies], w_dgrad, "sr", 1 + i, 0, dX, ws)
+    st = api.averis_check_status(ws)
+    if st:
+        raise RuntimeError(f"device status {st} in the profiling case")
+
+
 def run_gpu(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -890,6 +925,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.case is not None:
+        run_case(args)
         return
     import torch
     import torch.distributed as dist
