@@ -24,11 +24,19 @@
 //   warps 1..8 : TMA producers in both CTAs, two per operand taking
 //                alternate stages (A rows, B rows, A's scale atoms, B's
 //                scale atoms for all 256 columns plus the resident ones).
-//                Every copy completes on the leading CTA's barrier, whose
-//                producers expect the bytes of both CTAs;
-//   warp 9     : in the leading CTA, the scale copier (tcgen05.cp
-//                cta_group::2: each CTA's atoms into its own tensor memory);
-//   warps 10..17: epilogue in both CTAs, each over its own 128 x 256
+//                The copies of A, B and B's scales complete on the leading
+//                CTA's barrier, whose producers expect the bytes of both
+//                CTAs; A's scale atoms are each CTA's own and complete on
+//                its own barrier;
+//   warp 9     : in the leading CTA, B's scale copier (tcgen05.cp
+//                cta_group::2: each CTA's atoms into its own tensor
+//                memory);
+//   warps 10..13: A's scales into tensor memory, one warp per lane quarter
+//                in each CTA, by tcgen05.st from registers (the image a
+//                32x128b.warpx4 copy makes).  Tensor memory takes writes at
+//                a limited rate while the MMAs run: splitting them between
+//                the copy engine (B) and the stores (A) spreads the load;
+//   warps 14..21: epilogue in both CTAs, each over its own 128 x 256
 //                accumulator: the bias row staged in shared memory,
 //                tcgen05.ld, alpha * acc + bias, bf16, TMA store.
 // The leading CTA's MMA commits signal both CTAs' barriers (multicast
@@ -109,6 +117,19 @@ __device__ __forceinline__ void mma_nvf4_pair(uint32_t d_tmem, uint64_t a_desc, 
 __device__ __forceinline__ void tc_cp_32x128b_warpx4_pair(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
+// 32 lanes x 16 consecutive 32-bit columns from registers: thread t of the
+// warp writes lane (32 * (warp % 4) + t)
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
 
 }  // namespace
 
@@ -123,8 +144,10 @@ struct Gemm2Cfg {
   static constexpr int kKbPerStage = kStageK / 64;         // 4 MMAs per stage
   static constexpr int kEpiWarps = 8;
   static constexpr int kProducers = 8;                     // two per operand, alternate stages
+  static constexpr int kSfWarps = 4;                       // one per lane quarter
   static constexpr int kCopyWarp = 1 + kProducers;
-  static constexpr int kFirstEpiWarp = kCopyWarp + 1;
+  static constexpr int kFirstSfWarp = kCopyWarp + 1;
+  static constexpr int kFirstEpiWarp = kFirstSfWarp + kSfWarps;
   static constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
   static constexpr uint32_t kSbo = 8 * 128;                // 8-row swizzle atom of 128-byte rows
   static constexpr int kAChunkBytes = kBM * 128;           // 16 KB
@@ -154,7 +177,7 @@ struct Gemm2Cfg {
   static constexpr int kResOffset = kOutOffset + kStageOutBytes;
   static constexpr int kBiasOffset = kResOffset;
   static constexpr int kBarOffset = kBiasOffset + kBN * 4;
-  static constexpr int kSmemBytes = kBarOffset + 256;
+  static constexpr int kSmemBytes = kBarOffset + 512;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   // instruction descriptor: E2M1 A and B, UE4M3 scales, K-major, N >> 3 at
   // bit 17, M >> 4 at bit 24 (M = 256 for the pair)
@@ -191,8 +214,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
   uint8_t* sRes = sSfb;                        // resident mode: [2 row groups][chunk][4 atoms]
   float* bias_s = reinterpret_cast<float*>(smem + Cfg::kBiasOffset);
   uint64_t* full_ab = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOffset);  // [kStages] leading CTA: A, B landed
-  uint64_t* full_sf = full_ab + Cfg::kStages;   // [kStages] leading CTA: scale atoms landed
-  uint64_t* empty = full_sf + Cfg::kStages;     // [kStages] both CTAs
+  uint64_t* full_sfb = full_ab + Cfg::kStages;  // [kStages] leading CTA: B's scale atoms landed in both CTAs
+  uint64_t* full_sfa = full_sfb + Cfg::kStages; // [kStages] both CTAs: this CTA's A scale atoms landed
+  uint64_t* empty = full_sfa + Cfg::kStages;    // [kStages] both CTAs
   uint64_t* sf_full = empty + Cfg::kStages;     // [kStages] leading CTA: the stage's scales are in tensor memory
   uint64_t* acc_full = sf_full + Cfg::kStages;  // both CTAs
   uint64_t* acc_empty = acc_full + 1;           // leading CTA: both epilogues arrive
@@ -223,9 +247,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
     prefetch_tensormap(&map_y);
     for (int s = 0; s < Cfg::kStages; ++s) {
       mbar_init(&full_ab[s], 2);                // the leading CTA's A and B producers
-      mbar_init(&full_sf[s], 2);                // ... and its two scale producers
+      mbar_init(&full_sfb[s], 1);               // ... and its B-scale producer
+      mbar_init(&full_sfa[s], 1);               // this CTA's A-scale producer
       mbar_init(&empty[s], 1);
-      mbar_init(&sf_full[s], 1);
+      mbar_init(&sf_full[s], 2 * Cfg::kSfWarps + 1);   // the A-scale warps of both CTAs, the B-scale copies
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * Cfg::kEpiWarps);   // every epilogue warp of both CTAs
@@ -260,7 +285,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
   auto last_of_block = [&](int i) { return i + 1 == count || (first + i + 1) / p.tiles_m != (first + i) / p.tiles_m; };
   // barriers of the leading CTA, as shared::cluster addresses
   const uint32_t full_ab_lead = mapa_shared(smem_u32(full_ab), 0);
-  const uint32_t full_sf_lead = mapa_shared(smem_u32(full_sf), 0);
+  const uint32_t full_sfb_lead = mapa_shared(smem_u32(full_sfb), 0);
+  const uint32_t sf_full_lead = mapa_shared(smem_u32(sf_full), 0);
   const uint32_t res_load_lead = mapa_shared(smem_u32(res_load), 0);
   const uint32_t acc_empty_lead = mapa_shared(smem_u32(acc_empty), 0);
 
@@ -294,7 +320,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
             break;
           }
           const uint32_t bar_ab = full_ab_lead + static_cast<uint32_t>(st * 8);
-          const uint32_t bar_sf = full_sf_lead + static_cast<uint32_t>(st * 8);
+          const uint32_t bar_sfb = full_sfb_lead + static_cast<uint32_t>(st * 8);
           if (role == 0) {
             if (lead) mbar_arrive_expect_tx(&full_ab[st], 2 * Cfg::kABytes);
             tma_load_3d_pair(sA + st * Cfg::kABytes, &map_a, bar_ab, 0, m0, Cfg::kChunks * ks);
@@ -303,20 +329,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
             tma_load_3d_pair(sB + st * Cfg::kBBytes, &map_b, bar_ab, 0, n0 + static_cast<int32_t>(rank) * Cfg::kBNHalf,
                              Cfg::kChunks * ks);
           } else if (role == 2) {
-            if (lead) mbar_arrive_expect_tx(&full_sf[st], 2 * Cfg::kSfaBytes);
-            tma_load_3d_pair(sSfa + st * Cfg::kSfaBytes, &map_sfa, bar_sf, 0, Cfg::kChunks * ks, m0 / 128);
+            mbar_arrive_expect_tx(&full_sfa[st], Cfg::kSfaBytes);
+            tma_load_3d(sSfa + st * Cfg::kSfaBytes, &map_sfa, &full_sfa[st], 0, Cfg::kChunks * ks, m0 / 128);
           } else if (ks >= res_st) {
-            if (lead) mbar_arrive_expect_tx(&full_sf[st], 2 * Cfg::kSfbBytes);
-            tma_load_3d_pair(sSfb + st * Cfg::kSfbBytes, &map_sfb, bar_sf, 0, Cfg::kChunks * ks, n0 / 128);
+            if (lead) mbar_arrive_expect_tx(&full_sfb[st], 2 * Cfg::kSfbBytes);
+            tma_load_3d_pair(sSfb + st * Cfg::kSfbBytes, &map_sfb, bar_sfb, 0, Cfg::kChunks * ks, n0 / 128);
           } else if (lead) {
-            mbar_arrive(&full_sf[st]);            // this stage's B scales are resident
+            mbar_arrive(&full_sfb[st]);           // this stage's B scales are resident
           }
         }
       }
     }
   } else if (warp == Cfg::kCopyWarp) {
     if (lead && lane == 0) {
-      // ---------------- scale copier (leading CTA; each copy fills both CTAs) ----------------
+      // ---------------- B's scale copier (leading CTA; each copy fills both CTAs) ----------------
       // Stage ks's copies go to the slots of its stage buffer st: the slot's
       // previous MMAs completed before the stage was refilled.
       uint32_t st = 0, ph = 0;
@@ -339,18 +365,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
           tc_commit_pair_both(res_cp);
         }
         for (int ks = 0; ks < n_kst; ++ks) {
-          if (!mbar_wait_poll(&full_sf[st], ph, p.status)) {
+          if (!mbar_wait_poll(&full_sfb[st], ph, p.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sfa_t = tmem + Cfg::kSfaCol + Cfg::kSfaSlotCols * st;
-          const uint64_t sfa_d = smem_desc(smem_u32(sSfa + st * Cfg::kSfaBytes), 0, 128, kLayoutSwizzleNone);
-          const uint64_t sfb_d = smem_desc(smem_u32(sSfb + st * Cfg::kSfbBytes), 0, 128, kLayoutSwizzleNone);
-          const int nkb = min(Cfg::kKbPerStage, n_kb - ks * Cfg::kKbPerStage);
-          for (int kb = 0; kb < nkb; ++kb) tc_cp_32x128b_warpx4_pair(sfa_t + 4 * kb, sfa_d + static_cast<uint64_t>(32 * kb));
           if (ks >= res_st) {
             const uint32_t sfb_t = sfb_tmem_of(tmem, ks, static_cast<int>(st));
+            const uint64_t sfb_d = smem_desc(smem_u32(sSfb + st * Cfg::kSfbBytes), 0, 128, kLayoutSwizzleNone);
+            const int nkb = min(Cfg::kKbPerStage, n_kb - ks * Cfg::kKbPerStage);
             for (int kb = 0; kb < nkb; ++kb)
 #pragma unroll
               for (int g = 0; g < 2; ++g)
@@ -366,6 +389,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
       }
       tc_commit_pair(&drained[1]);
       mbar_wait(&drained[1], 0, p.status);
+    }
+  } else if (warp >= Cfg::kFirstSfWarp && warp < Cfg::kFirstEpiWarp) {
+    // ---------------- A's scales into tensor memory (both CTAs) ----------------
+    // Each warp stores A's atoms of every stage (its CTA's rows) into the
+    // stage's slot in its own lane quarter.  A slot's previous MMAs completed
+    // before its stage was refilled, so the slot is free once the stage's
+    // atoms have landed.
+    const uint32_t t_quarter = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+    uint32_t st = 0, ph = 0;
+    for (int it = 0; it < count * n_kst; ++it) {
+      uint32_t okw = 1u;
+      if (lane == 0) okw = mbar_wait_poll(&full_sfa[st], ph, p.status) ? 1u : 0u;
+      if (__shfl_sync(0xFFFFFFFFu, okw, 0) == 0u) break;
+      tc_fence_after();
+      // lane l's 16 bytes of atom kb are columns 4 kb .. 4 kb + 3 of its lane
+      const uint8_t* src = sSfa + st * Cfg::kSfaBytes + 16 * lane;
+      uint32_t w[16];
+#pragma unroll
+      for (int kb = 0; kb < Cfg::kKbPerStage; ++kb) {
+        const uint4 v = *reinterpret_cast<const uint4*>(src + kb * 512);
+        w[4 * kb] = v.x;
+        w[4 * kb + 1] = v.y;
+        w[4 * kb + 2] = v.z;
+        w[4 * kb + 3] = v.w;
+      }
+      tmem_st_32x32b_x16(t_quarter + Cfg::kSfaCol + Cfg::kSfaSlotCols * st, w);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(sf_full_lead + static_cast<uint32_t>(st * 8));
+      if (++st == Cfg::kStages) {
+        st = 0;
+        ph ^= 1u;
+      }
     }
   } else if (warp == 0) {
     if (lead && lane == 0) {
