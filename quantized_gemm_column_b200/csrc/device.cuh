@@ -166,6 +166,22 @@ __device__ __forceinline__ bool mbar_wait_poll(uint64_t* bar, uint32_t parity, u
   return true;
 }
 
+// Polling with a short sleep between polls, for waiters off the critical
+// path: a warp spinning on test_wait keeps the shared-memory pipe busy, and
+// the MMA issuer's own barrier and tcgen05 operations queue behind it.
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, uint32_t* status) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_test(bar, parity)) {
+    __nanosleep(64);
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      raise_status(status, AVR_ERR_DEVICE_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------------------
 // TMA (tensor) loads and bulk copies, global -> shared, completing on an
 // mbarrier.  No cluster multicast anywhere in this library.

@@ -439,7 +439,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, kBf16Out>::kThreads, 1)
       float u_r = 1.0f;
       if (kRank1) u_r = (m0 + r < p.M) ? __ldg(p.row_scale + m0 + r) : 0.0f;
       uint32_t okw = 0;
-      if (lane == 0) okw = mbar_wait(&acc_full[ab], static_cast<uint32_t>(i / Cfg::kAccBufs) & 1u, p.status) ? 1u : 0u;
+      if (lane == 0) okw = mbar_wait_poll(&acc_full[ab], static_cast<uint32_t>(i / Cfg::kAccBufs) & 1u, p.status) ? 1u : 0u;
       const bool ok = __shfl_sync(0xFFFFFFFFu, okw, 0) != 0;
       // all epilogue threads agree, so the .sync.aligned loads below run in
       // every lane of every warp or in none; the barrier also publishes the
@@ -693,6 +693,7 @@ cudaError_t launch_mma_rate(int iters, int grid, uint64_t* ns, uint32_t* status,
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, bool pdl) {
+  if (gemm_pair_short_applies(a)) return launch_gemm_pair_short(a, s, pdl);
   if (gemm_pair_applies(a)) return launch_gemm_pair(a, s, pdl);
   if (a.row_scale != nullptr) {
     if (a.bias == nullptr || a.block_expert != nullptr) return cudaErrorInvalidValue;

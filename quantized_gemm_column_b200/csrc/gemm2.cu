@@ -51,87 +51,11 @@
 
 #include "device.cuh"
 #include "internal.h"
+#include "pair.cuh"
 
 namespace avr {
 
-namespace {
-
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// the shared::cluster address of the same shared-memory location in CTA `rank` of the cluster
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// arrive on an mbarrier given by its shared::cluster address (possibly another CTA's)
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-// TMA 3-D load into this CTA's shared memory completing on the barrier at a
-// shared::cluster address in either CTA of the pair
-__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int32_t x,
-                                                 int32_t y, int32_t z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];"
-      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
-               ::"r"(smem_u32(dst_smem)), "r"(ncols) : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-// arrive once on *bar (this CTA) when the pair operations this thread issued have completed
-__device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-               ::"r"(smem_u32(bar)) : "memory");
-}
-// ... on the barrier at the same offset in both CTAs of the pair
-__device__ __forceinline__ void tc_commit_pair_both(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
-               ::"r"(smem_u32(bar)), "h"(static_cast<uint16_t>(3)) : "memory");
-}
-__device__ __forceinline__ void mma_nvf4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
-      "}"
-      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-      : "memory");
-}
-__device__ __forceinline__ void tc_cp_32x128b_warpx4_pair(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-// 32 lanes x 16 consecutive 32-bit columns from registers: thread t of the
-// warp writes lane (32 * (warp % 4) + t)
-__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
-      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-}  // namespace
+using namespace pair;
 
 struct Gemm2Cfg {
   static constexpr int kBM = 128;                          // rows per CTA (256 per pair)
@@ -305,7 +229,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
         const int32_t n0 = (tile / p.tiles_m) * Cfg::kBN;
         if (role == 3 && parity == 0 && res_st > 0 && new_block(i)) {
           // both CTAs' resident buffers are free once the previous block's copies ran
-          if (res_uses >= 1 && !mbar_wait_poll(res_cp, static_cast<uint32_t>(res_uses - 1) & 1u, p.status)) break;
+          if (res_uses >= 1 && !mbar_wait_backoff(res_cp, static_cast<uint32_t>(res_uses - 1) & 1u, p.status)) break;
           ++res_uses;
           if (lead) mbar_arrive_expect_tx(res_load, static_cast<uint32_t>(2 * res_st * Cfg::kSfbBytes));
           // box of res_st * 2 chunks: this launch's B-scale map is sized for it (see the launch)
@@ -315,7 +239,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
           if ((it & 1) != parity) continue;
           const uint32_t st = static_cast<uint32_t>(it % Cfg::kStages);
           const uint32_t ph = static_cast<uint32_t>(it / Cfg::kStages) & 1u;
-          if (it >= Cfg::kStages && !mbar_wait_poll(&empty[st], ph ^ 1u, p.status)) {
+          if (it >= Cfg::kStages && !mbar_wait_backoff(&empty[st], ph ^ 1u, p.status)) {
             ok = false;
             break;
           }
@@ -400,7 +324,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
     uint32_t st = 0, ph = 0;
     for (int it = 0; it < count * n_kst; ++it) {
       uint32_t okw = 1u;
-      if (lane == 0) okw = mbar_wait_poll(&full_sfa[st], ph, p.status) ? 1u : 0u;
+      if (lane == 0) okw = mbar_wait_backoff(&full_sfa[st], ph, p.status) ? 1u : 0u;
       if (__shfl_sync(0xFFFFFFFFu, okw, 0) == 0u) break;
       tc_fence_after();
       // lane l's 16 bytes of atom kb are columns 4 kb .. 4 kb + 3 of its lane
@@ -502,7 +426,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
         bias_s[ew * 32 + lane] = (p.bias != nullptr && col < p.N) ? __ldg(p.bias + col) : 0.0f;
       }
       uint32_t okw = 0;
-      if (lane == 0) okw = mbar_wait(acc_full, static_cast<uint32_t>(i) & 1u, p.status) ? 1u : 0u;
+      if (lane == 0) okw = mbar_wait_backoff(acc_full, static_cast<uint32_t>(i) & 1u, p.status) ? 1u : 0u;
       const bool ok = __shfl_sync(0xFFFFFFFFu, okw, 0) != 0;
       if (named_barrier_or(1, kEpiThreads, !ok)) break;
       tc_fence_after();
@@ -608,17 +532,18 @@ bool gemm_pair_applies(const GemmArgs& a) {
 }
 
 // [rows, K/2 bytes] codes as a 3-D tensor (128 bytes, rows, K/256 chunks):
-// a box of (128, box_rows, 2) brings two 128-byte-swizzled chunk tiles
-static bool codes_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, uint32_t box_rows) {
+// a box of (128, box_rows, box_chunks) brings box_chunks 128-byte-swizzled
+// chunk tiles of box_rows rows, one after the other
+bool pair_codes_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, uint32_t box_rows, uint32_t box_chunks) {
   const uint64_t dims[3] = {128, static_cast<uint64_t>(rows), static_cast<uint64_t>(K / 256)};
   const uint64_t strides[2] = {static_cast<uint64_t>(K / 2), 128};
-  const uint32_t box[3] = {128, box_rows, static_cast<uint32_t>(Gemm2Cfg::kChunks)};
+  const uint32_t box[3] = {128, box_rows, box_chunks};
   return make_tensor_map_3d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT8, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 // scale atoms as a 3-D tensor of 8-byte elements (256 = one chunk's 4
 // atoms, K/256 chunks, row groups of 128)
-static bool scales_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, uint32_t box_chunks,
-                       uint32_t box_groups) {
+bool pair_scales_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, uint32_t box_chunks,
+                     uint32_t box_groups) {
   const uint64_t dims[3] = {256, static_cast<uint64_t>(K / 256), static_cast<uint64_t>((rows + 127) / 128)};
   const uint64_t strides[2] = {2048, static_cast<uint64_t>(K / 64) * 512};
   const uint32_t box[3] = {256, box_chunks, box_groups};
@@ -632,12 +557,13 @@ cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s, bool pdl) {
   // B's scales: all of K resident when they fit, else streamed per stage
   const int res_stages = n_kst <= Cfg::kResAllStages ? n_kst : 0;
   CUtensorMap ma, mb, msa, msb, my;
-  if (!codes_map(&ma, a.a_codes, a.M, a.K, Cfg::kBM) || !codes_map(&mb, a.b_codes, a.N, a.K, Cfg::kBNHalf) ||
-      !scales_map(&msa, a.a_scales, a.M, a.K, Cfg::kChunks, 1))
+  if (!pair_codes_map(&ma, a.a_codes, a.M, a.K, Cfg::kBM, Cfg::kChunks) ||
+      !pair_codes_map(&mb, a.b_codes, a.N, a.K, Cfg::kBNHalf, Cfg::kChunks) ||
+      !pair_scales_map(&msa, a.a_scales, a.M, a.K, Cfg::kChunks, 1))
     return cudaErrorInvalidValue;
   // one map for B's scales: its box is the resident block (res_stages stages
   // of both row groups) when every stage is resident, else one stage
-  if (!scales_map(&msb, a.b_scales, a.N, a.K, static_cast<uint32_t>(Cfg::kChunks * (res_stages > 0 ? res_stages : 1)), 2))
+  if (!pair_scales_map(&msb, a.b_scales, a.N, a.K, static_cast<uint32_t>(Cfg::kChunks * (res_stages > 0 ? res_stages : 1)), 2))
     return cudaErrorInvalidValue;
   if (!make_tensor_map_2d(&my, a.Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, static_cast<uint64_t>(a.M),
                           static_cast<uint64_t>(a.N), Cfg::kBM, 64, CU_TENSOR_MAP_SWIZZLE_128B))

@@ -230,6 +230,14 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s, bool pdl);
 // the 2-CTA kernel (gemm2.cu): dense bf16 outputs, 256 x 256 tiles on CTA pairs
 bool gemm_pair_applies(const GemmArgs& a);
 cudaError_t launch_gemm_pair(const GemmArgs& a, cudaStream_t s, bool pdl);
+// the short-contraction pair kernel (K <= 1024; B's column block resident)
+bool gemm_pair_short_applies(const GemmArgs& a);
+cudaError_t launch_gemm_pair_short(const GemmArgs& a, cudaStream_t s, bool pdl);
+// tensor maps of the pair kernels: codes as (128 bytes, rows, K/256 chunks),
+// scale atoms as (256 x 8 bytes, K/256 chunks, row groups of 128)
+bool pair_codes_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, uint32_t box_rows, uint32_t box_chunks);
+bool pair_scales_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, uint32_t box_chunks,
+                     uint32_t box_groups);
 
 // ---------------- host-side validation and the split chain (api.cu) ----------------
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
