@@ -156,7 +156,7 @@ __device__ __forceinline__ uint32_t gather_scale_word(uint32_t S) {
 // in [2^-10, 2688]), and so is every E2M1 value, so the per-element product
 // is taken exactly with the mixed f16 x f16 + f32 FMA and summed in fp32.
 // ---------------------------------------------------------------------------
-constexpr int kRowGroup = 32;   // output rows of one group (one per lane)
+constexpr int kRowGroup = 32;   // output rows per aux CTA when the aux CTAs are counted
 
 // two packed E2M1 codes (one byte, element 2i in the low nibble) -> f16x2
 __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
@@ -175,81 +175,76 @@ __device__ __forceinline__ float fma2_f16_f32(uint32_t a, uint32_t b, float c) {
   return d;
 }
 
-// Partial dot product of row j of w with the f16 values s_mu16[k - k_lo]
-// over k in [k0, k1) (multiples of 64 inside one window): one lane, 64
-// elements (two 16-byte code loads, one scale word) per step, four steps'
-// loads issued before any is used.  The E4M3 block scale is applied to each
-// 16-element partial.
-static __device__ float bias_dot(const uint16_t* s_mu16, int64_t k_lo, int64_t k0, int64_t k1, int64_t j,
-                          int64_t K, const uint8_t* w_codes, const uint8_t* w_scales) {
-  constexpr int kSteps = 4;
+// The rows of w over the window [k_lo, k_hi) of the f16 values
+// s_mu16[k - k_lo]: warp w of CTA `cta` takes the rows cta * 8 + w + t R,
+// R = 8 n_ctas, four at a time.  Lane l takes the 16-element blocks l,
+// l + 32, ... of the window (8 bytes of codes each: a warp reads 256
+// contiguous bytes of a row per block step); the loads of four rows x two
+// block steps are issued before any is used, and each mu_bar block read from
+// shared memory serves the four rows.  The block's E4M3 scale is applied to
+// its 16-element partial, and the lanes' sums are added by a fixed
+// butterfly.  The first window stores into out[j], later windows add to it,
+// and the last one scales by g_dec_prod.  (s_part is not used.)
+static __device__ void bias_window(const uint16_t* s_mu16, float* s_part, int64_t k_lo, int64_t k_hi, int64_t K,
+                                   const uint8_t* w_codes, const uint8_t* w_scales, float g_dec_prod,
+                                   int64_t n_out, int cta, int n_ctas, float* out) {
+  (void)s_part;
+  constexpr int kRows = 4, kSteps = 2;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t n_kb64 = static_cast<uint32_t>(K / 64);
-  const uint8_t* row = w_codes + j * (K / 2);
-  float acc = 0.0f;
-  for (int64_t kb = k0; kb < k1; kb += 64 * kSteps) {
-    uint4 c[kSteps][2];
-    uint32_t sw[kSteps];
+  const int64_t row_step = static_cast<int64_t>(n_ctas) * kQuantWarps;
+  for (int64_t j0 = static_cast<int64_t>(cta) * kQuantWarps + warp; j0 < n_out; j0 += kRows * row_step) {
+    float acc[kRows];
 #pragma unroll
-    for (int u = 0; u < kSteps; ++u) {
-      const int64_t k = kb + 64 * u;
-      if (k < k1) {
-        const uint4* q = reinterpret_cast<const uint4*>(row + k / 2);
-        c[u][0] = __ldg(q);
-        c[u][1] = __ldg(q + 1);
-        sw[u] = __ldg(reinterpret_cast<const uint32_t*>(
-            w_scales + scale_offset(static_cast<uint64_t>(j), static_cast<uint32_t>(k / 16), n_kb64)));
+    for (int t = 0; t < kRows; ++t) acc[t] = 0.0f;
+    for (int64_t kb = k_lo + 16 * lane; kb < k_hi; kb += 16 * 32 * kSteps) {
+      uint2 c[kSteps][kRows];
+      uint32_t sb[kSteps][kRows];
+#pragma unroll
+      for (int u = 0; u < kSteps; ++u) {
+        const int64_t k = kb + 16 * 32 * u;
+#pragma unroll
+        for (int t = 0; t < kRows; ++t) {
+          const int64_t j = j0 + t * row_step;
+          if (k < k_hi && j < n_out) {
+            c[u][t] = __ldg(reinterpret_cast<const uint2*>(w_codes + j * (K / 2) + k / 2));
+            sb[u][t] = __ldg(w_scales + scale_offset(static_cast<uint64_t>(j), static_cast<uint32_t>(k / 16), n_kb64));
+          } else {
+            c[u][t] = make_uint2(0u, 0u);
+            sb[u][t] = 0u;
+          }
+        }
       }
-    }
 #pragma unroll
-    for (int u = 0; u < kSteps; ++u) {
-      const int64_t k = kb + 64 * u;
-      if (k < k1) {
-        const uint4* m = reinterpret_cast<const uint4*>(s_mu16 + (k - k_lo));   // 64 f16 = 8 x 16 B
-        const uint32_t words[8] = {c[u][0].x, c[u][0].y, c[u][0].z, c[u][0].w,
-                                   c[u][1].x, c[u][1].y, c[u][1].z, c[u][1].w};
+      for (int u = 0; u < kSteps; ++u) {
+        const int64_t k = kb + 16 * 32 * u;
+        if (k >= k_hi) break;
+        const uint4* m = reinterpret_cast<const uint4*>(s_mu16 + (k - k_lo));   // 16 f16 = 2 x 16 B
+        const uint4 m0 = m[0], m1 = m[1];
+        const uint32_t mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {           // 16-element block b: code words 2b, 2b+1
-          const uint4 m0 = m[2 * b], m1 = m[2 * b + 1];
-          const uint32_t mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+        for (int t = 0; t < kRows; ++t) {
           float part = 0.0f;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            const uint32_t byte = (words[2 * b + q / 4] >> (8 * (q % 4))) & 0xFFu;
+            const uint32_t byte = ((q < 4 ? c[u][t].x : c[u][t].y) >> (8 * (q % 4))) & 0xFFu;
             part = fma2_f16_f32(e2m1x2_to_f16x2(byte), mv[q], part);
           }
-          acc = fmaf(part, e4m3_value((sw[u] >> (8 * b)) & 0xFFu), acc);
+          acc[t] = fmaf(part, e4m3_value(sb[u][t]), acc[t]);
         }
       }
     }
-  }
-  return acc;
-}
-
-// The rows of w in groups of kRowGroup, group g handled by CTA g mod
-// n_ctas: lane l takes row 32g + l and warp w the w-th of eight 64-aligned
-// segments of the window [k_lo, k_hi); warp 0 adds the eight partials in
-// warp order.  The first window stores into out[j], later windows add to it,
-// and the last one scales by g_dec_prod.  s_part: kQuantWarps * kRowGroup floats.
-static __device__ void bias_window(const uint16_t* s_mu16, float* s_part, int64_t k_lo, int64_t k_hi, int64_t K,
-                            const uint8_t* w_codes, const uint8_t* w_scales, float g_dec_prod,
-                            int64_t n_out, int cta, int n_ctas, float* out) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t seg = ((k_hi - k_lo + kQuantWarps * 64 - 1) / (kQuantWarps * 64)) * 64;
-  const int64_t k0 = min64(k_hi, k_lo + warp * seg), k1 = min64(k_hi, k0 + seg);
-  const int64_t n_groups = (n_out + kRowGroup - 1) / kRowGroup;
-  for (int64_t g = cta; g < n_groups; g += n_ctas) {
-    const int64_t j = g * kRowGroup + lane;
-    const float part = j < n_out ? bias_dot(s_mu16, k_lo, k0, k1, j, K, w_codes, w_scales) : 0.0f;
-    s_part[warp * kRowGroup + lane] = part;
-    __syncthreads();
-    if (warp == 0 && j < n_out) {
-      float acc = s_part[lane];
 #pragma unroll
-      for (int w = 1; w < kQuantWarps; ++w) acc += s_part[w * kRowGroup + lane];
-      if (k_lo != 0) acc += out[j];
-      out[j] = k_hi == K ? acc * g_dec_prod : acc;
+    for (int t = 0; t < kRows; ++t) {
+      float v = acc[t];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+      const int64_t j = j0 + t * row_step;
+      if (lane == 0 && j < n_out) {
+        if (k_lo != 0) v += out[j];
+        out[j] = k_hi == K ? v * g_dec_prod : v;
+      }
     }
-    __syncthreads();
   }
 }
 
