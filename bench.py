@@ -720,6 +720,35 @@ def run_gpu(args, rank, world, local_rank):
     step_ms = ms / args.steps
     value = job_value(FLOPS_PER_STEP, world, step_ms)
 
+    # per-step distribution (beside the headline): each replay bracketed by its
+    # own events, warm (back to back) and with L2 flushed before every step
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # 256 MiB > 126 MB of L2
+
+    def step_distribution(n, vanilla=False, cold=False):
+        pairs = []
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                replay(i, vanilla)
+            torch.cuda.synchronize(dev)
+            for i in range(n):
+                if cold:
+                    flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                replay(i, vanilla)
+                b.record(stream)
+                pairs.append((a, b))
+            torch.cuda.synchronize(dev)
+        us = sorted(a.elapsed_time(b) * 1e3 for a, b in pairs)
+        q = lambda f: us[min(len(us) - 1, int(round(f * (len(us) - 1))))]
+        return {"median_us": q(0.5), "p10_us": q(0.1), "p90_us": q(0.9), "steps": n}
+
+    n_dist = 200
+    dist_steps = {"averis": {"warm": step_distribution(n_dist), "cold_l2": step_distribution(n_dist, cold=True)},
+                  "vanilla": {"warm": step_distribution(n_dist, True),
+                              "cold_l2": step_distribution(n_dist, True, cold=True)}}
+    del flush
+
     # per-kernel-group timing (same stream, events around n launches each)
     xr = api.NVFP4Tensor(L, M, dev)
     dr = api.NVFP4Tensor(L, N, dev)
@@ -903,6 +932,7 @@ def run_gpu(args, rank, world, local_rank):
         "averis_overhead_vs_vanilla": (ms / ms_van) - 1.0,
         "weight_quant_us": wq_us,
         "roofline": roof,
+        "step_us_distribution": dist_steps,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                    "reasons": clocks["reasons"], "samples_in_region": clocks["samples_in_region"]},
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
