@@ -28,15 +28,15 @@
 //                CTA's barrier, whose producers expect the bytes of both
 //                CTAs; A's scale atoms are each CTA's own and complete on
 //                its own barrier;
-//   warp 9     : in the leading CTA, B's scale copier (tcgen05.cp
-//                cta_group::2: each CTA's atoms into its own tensor
-//                memory);
-//   warps 10..13: A's scales into tensor memory, one warp per lane quarter
+//   warps 9, 10: in the leading CTA, B's scale copiers, alternate stages
+//                (tcgen05.cp cta_group::2: each CTA's atoms into its own
+//                tensor memory);
+//   warps 11..14: A's scales into tensor memory, one warp per lane quarter
 //                in each CTA, by tcgen05.st from registers (the image a
 //                32x128b.warpx4 copy makes).  Tensor memory takes writes at
 //                a limited rate while the MMAs run: splitting them between
 //                the copy engine (B) and the stores (A) spreads the load;
-//   warps 14..21: epilogue in both CTAs, each over its own 128 x 256
+//   warps 15..22: epilogue in both CTAs, each over its own 128 x 256
 //                accumulator: the bias row staged in shared memory,
 //                tcgen05.ld, alpha * acc + bias, bf16, TMA store.
 // The leading CTA's MMA commits signal both CTAs' barriers (multicast
@@ -70,7 +70,8 @@ struct Gemm2Cfg {
   static constexpr int kProducers = 8;                     // two per operand, alternate stages
   static constexpr int kSfWarps = 4;                       // one per lane quarter
   static constexpr int kCopyWarp = 1 + kProducers;
-  static constexpr int kFirstSfWarp = kCopyWarp + 1;
+  static constexpr int kCopyWarps = 2;                     // B's scale copies, alternate stages
+  static constexpr int kFirstSfWarp = kCopyWarp + kCopyWarps;
   static constexpr int kFirstEpiWarp = kFirstSfWarp + kSfWarps;
   static constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
   static constexpr uint32_t kSbo = 8 * 128;                // 8-row swizzle atom of 128-byte rows
@@ -147,8 +148,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
   uint64_t* res_load = acc_empty + 1;           // leading CTA: resident scales landed in both CTAs
   uint64_t* res_cp = res_load + 1;              // both CTAs: resident scales copied
   uint64_t* res_free = res_cp + 1;              // leading CTA: the MMAs of a column block are done
-  uint64_t* drained = res_free + 1;             // [2] leading CTA: MMA and copy threads drained
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 2);
+  uint64_t* drained = res_free + 1;             // [1 + kCopyWarps] leading CTA: MMA and copy threads drained
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1 + Cfg::kCopyWarps);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -181,8 +182,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
     mbar_init(res_load, 1);
     mbar_init(res_cp, 1);
     mbar_init(res_free, 1);
-    mbar_init(&drained[0], 1);
-    mbar_init(&drained[1], 1);
+    for (int d = 0; d <= Cfg::kCopyWarps; ++d) mbar_init(&drained[d], 1);
     fence_mbarrier_init();
   }
   if (warp == 0) {
@@ -264,17 +264,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
         }
       }
     }
-  } else if (warp == Cfg::kCopyWarp) {
+  } else if (warp >= Cfg::kCopyWarp && warp < Cfg::kCopyWarp + Cfg::kCopyWarps) {
     if (lead && lane == 0) {
-      // ---------------- B's scale copier (leading CTA; each copy fills both CTAs) ----------------
-      // Stage ks's copies go to the slots of its stage buffer st: the slot's
-      // previous MMAs completed before the stage was refilled.
-      uint32_t st = 0, ph = 0;
-      int res_uses = 0;
+      // ---------------- B's scale copiers (leading CTA; each copy fills both CTAs) ----------------
+      // Copier cw takes the stages it with it % kCopyWarps == cw, so one
+      // thread's waits and commits run beside the other's copies.  Stage
+      // ks's copies go to the slots of its stage buffer st: the slot's
+      // previous MMAs completed before the stage was refilled.  Copier 0
+      // also copies the resident scales of a new column block.
+      const int cw = warp - Cfg::kCopyWarp;
+      int it = 0, res_uses = 0;
       bool ok = true;
       const uint64_t res_d = smem_desc(smem_u32(sRes), 0, 128, kLayoutSwizzleNone);
       for (int i = 0; i < count && ok; ++i) {
-        if (res_st > 0 && new_block(i)) {
+        if (cw == 0 && res_st > 0 && new_block(i)) {
           if (res_uses >= 1 && !mbar_wait_poll(res_free, static_cast<uint32_t>(res_uses - 1) & 1u, p.status)) break;
           if (!mbar_wait_poll(res_load, static_cast<uint32_t>(res_uses) & 1u, p.status)) break;
           ++res_uses;
@@ -288,7 +291,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
                                         res_d + static_cast<uint64_t>(32 * (g * res_st * Cfg::kKbPerStage + kb)));
           tc_commit_pair_both(res_cp);
         }
-        for (int ks = 0; ks < n_kst; ++ks) {
+        for (int ks = 0; ks < n_kst; ++ks, ++it) {
+          if (it % Cfg::kCopyWarps != cw) continue;
+          const uint32_t st = static_cast<uint32_t>(it % Cfg::kStages);
+          const uint32_t ph = static_cast<uint32_t>(it / Cfg::kStages) & 1u;
           if (!mbar_wait_poll(&full_sfb[st], ph, p.status)) {
             ok = false;
             break;
@@ -305,14 +311,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg::kThreads, 
                                           sfb_d + static_cast<uint64_t>(32 * (g * Cfg::kKbPerStage + kb)));
           }
           tc_commit_pair(&sf_full[st]);
-          if (++st == Cfg::kStages) {
-            st = 0;
-            ph ^= 1u;
-          }
         }
       }
-      tc_commit_pair(&drained[1]);
-      mbar_wait(&drained[1], 0, p.status);
+      tc_commit_pair(&drained[1 + cw]);
+      mbar_wait(&drained[1 + cw], 0, p.status);
     }
   } else if (warp >= Cfg::kFirstSfWarp && warp < Cfg::kFirstEpiWarp) {
     // ---------------- A's scales into tensor memory (both CTAs) ----------------
