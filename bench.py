@@ -530,7 +530,7 @@ def run_reference(args, rank, world):
 # ---------------------------------------------------------------------------
 # measured DRAM traffic (ncu), valid only for the kernel sources it was taken on
 # ---------------------------------------------------------------------------
-KERNEL_SOURCES = ["colreduce.cu", "quant.cu", "quant_common.cuh", "split_fused.cu", "gemm.cu", "gemm2.cu", "gemm3.cu",
+KERNEL_SOURCES = ["colreduce.cu", "quant.cu", "quant_common.cuh", "split_fused.cu", "gemm.cu", "gemm2.cu", "gemm3.cu", "pair.cuh",
                   "device.cuh", "internal.h"]
 TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "traffic_qkv_step.json")
 

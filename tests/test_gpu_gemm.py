@@ -34,8 +34,9 @@ def _gemm(api, a_q, b_q, bias=None, out=torch.float32):
     return Y.float().cpu().numpy().astype(np.float64)
 
 
-# bf16 outputs with K a multiple of 256 run on the CTA-pair kernel, the
-# others on the one-CTA kernel: the probes run at K = 64 and 256 to cover both.
+# bf16 outputs with K a multiple of 256 run on a CTA-pair kernel (the
+# short-contraction one for K <= 1024), the others on the one-CTA kernel: the
+# probes run at K = 64 and 256 to cover both.
 KERNELS = [(torch.float32, 64), (torch.bfloat16, 64), (torch.bfloat16, 256)]
 
 
@@ -142,6 +143,22 @@ def test_random_gemm_bf16_out(api, M, N, K):
     check_bf16_output(Y, ref, gemm_tolerance(a, b, bias, K))
 
 
+@pytest.mark.parametrize("M,N,K", [(1000, 700, 512), (4224, 2112, 768), (8192, 1280, 1024)])
+def test_short_pair_kernel_ragged(api, M, N, K):
+    """The short-contraction pair kernel (bf16 out, K <= 1024): M and N not
+    multiples of the 256 x 256 pair tile (the last row block leaves the second
+    CTA of its pair with no rows, the last column block half empty), and runs
+    of several tiles per pair that change column block (B's resident rows and
+    scales reloaded).  Every output is compared."""
+    rng = np.random.default_rng(M + 3 * N + K)
+    a = _rand_q(rng, M, K, g_dec=0.01)
+    b = _rand_q(rng, N, K, g_dec=0.003)
+    bias = rng.standard_normal(N) * 0.1
+    Y = _gemm(api, a, b, bias, out=torch.bfloat16)
+    ref = oracle.gemm_reference(a, b, bias)
+    check_bf16_output(Y, ref, gemm_tolerance(a, b, bias, K))
+
+
 def test_quantized_operands_from_oracle(api):
     """Operands produced by the oracle's quantizer (realistic scale mix)."""
     rng = np.random.default_rng(4)
@@ -167,11 +184,11 @@ def _gemm_sampled(api, a_q, b_q, cols, bias=None, out=torch.float32):
 def test_resident_b_scales_across_column_blocks_bf16(api, K):
     """Many more tiles than CTAs (or CTA pairs), so a run of tiles changes
     column block (B's resident scales are reloaded) and shares it between
-    tiles.  The pair kernel (K a multiple of 256) keeps all of B's scales
-    resident up to K = 1536 (256, 1280: a last stage of one chunk) and
-    streams them past one resident stage beyond (2048, 2304: a last stage of
-    one chunk); K = 2112 runs the one-CTA kernel (five of nine stages
-    resident, a partial last stage)."""
+    tiles.  K = 256 runs the short-contraction pair kernel (B's rows and
+    scales resident per column block); the pair kernel keeps all of B's
+    scales resident at K = 1280 and 1536 and streams them beyond (2048, 2304:
+    a last stage of one chunk); K = 2112 runs the one-CTA kernel (five of
+    nine stages resident, a partial last stage)."""
     rng = np.random.default_rng(K)
     M, N = 512, 256 * 160
     a = _rand_q(rng, M, K, g_dec=0.01)
