@@ -749,6 +749,19 @@ def run_gpu(args, rank, world, local_rank):
                               "cold_l2": step_distribution(n_dist, True, cold=True)}}
     del flush
 
+    # sustained: the Averis step replayed back to back for about two seconds
+    # (long enough to meet the power cap), SM clocks sampled inside the region
+    n_sus = max(args.steps, int(2.0 / (step_ms * 1e-3)))
+    with torch.cuda.stream(stream):
+        torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clk_sus:
+        t0 = time.monotonic()
+        ms_sus = timed(n_sus)
+        clk_sus.region(t0, time.monotonic())
+    sus_step_ms = ms_sus / n_sus
+    sustained = {"steps": n_sus, "ms_per_step": sus_step_ms,
+                 "tflops": FLOPS_PER_STEP / (sus_step_ms * 1e-3) / 1e12, "clocks": clk_sus.summary()}
+
     # per-kernel-group timing (same stream, events around n launches each)
     xr = api.NVFP4Tensor(L, M, dev)
     dr = api.NVFP4Tensor(L, N, dev)
@@ -933,6 +946,7 @@ def run_gpu(args, rank, world, local_rank):
         "weight_quant_us": wq_us,
         "roofline": roof,
         "step_us_distribution": dist_steps,
+        "sustained": sustained,
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"],
                    "reasons": clocks["reasons"], "samples_in_region": clocks["samples_in_region"]},
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
