@@ -304,3 +304,55 @@ def test_set_wait_limit_validation_on_the_host(lib):
     import torch
     if not torch.cuda.is_available():
         assert f(ctypes.c_void_p(256), 1 << 20, 5, None) == api.AVR_ERR_NO_DEVICE
+
+
+def _prototypes():
+    """{name: (return type, [parameter types])} of every entry point in the
+    header, comments removed, parameter names dropped."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    out = {}
+    for ret, name, params in re.findall(
+            r"^(size_t|avr_status|const char\s*\*)\s*(\w+)\s*\(([^)]*)\)\s*;", text, flags=re.M | re.S):
+        types = []
+        for p in params.split(","):
+            p = " ".join(p.split())
+            if not p or p == "void":
+                continue
+            m = re.match(r"^(.*?[\s*])(\w+)$", p)        # type, then the parameter's name
+            types.append(m.group(1).replace(" ", "") if m else p.replace(" ", ""))
+        out[name] = (ret.replace(" ", ""), types)
+    return out
+
+
+def _c_class(t):
+    """The ctypes class a C parameter or return type must be marshalled as."""
+    if t.endswith("*") or t == "avr_stream":
+        return "ptr"
+    # size_t and uint64_t are one ctypes type (c_ulong) on this ABI
+    return {"int64_t": "i64", "uint64_t": "u64", "uint32_t": "u32", "size_t": "u64", "int": "int",
+            "avr_dtype": "int", "avr_round": "int", "avr_status": "int"}[t]
+
+
+def _ctypes_class(ct):
+    if ct is ctypes.c_void_p or ct is ctypes.c_char_p or (isinstance(ct, type) and issubclass(ct, ctypes._Pointer)):
+        return "ptr"
+    assert ctypes.c_size_t is ctypes.c_uint64
+    return {ctypes.c_int64: "i64", ctypes.c_uint64: "u64", ctypes.c_uint32: "u32", ctypes.c_int: "int"}[ct]
+
+
+def test_binding_signatures_match_the_header():
+    """Every entry point's ctypes signature has the header's arity and, per
+    argument, the same class (pointer, int, int64, uint64 or size_t, uint32):
+    a slip in the argument list would otherwise pass garbage silently."""
+    from quantized_gemm_column_b200 import api
+    protos = _prototypes()
+    assert set(protos) == set(declared_functions())
+    for name, (ret, params) in protos.items():
+        assert name in api._SIGS, name
+        res, args = api._SIGS[name]
+        assert len(args) == len(params), (name, len(args), params)
+        got = [_ctypes_class(a) for a in args]
+        want = [_c_class(p) for p in params]
+        assert got == want, (name, got, want)
+        assert _ctypes_class(res) == ("ptr" if ret == "constchar*" else _c_class(ret)), name
