@@ -356,3 +356,28 @@ def test_binding_signatures_match_the_header():
         want = [_c_class(p) for p in params]
         assert got == want, (name, got, want)
         assert _ctypes_class(res) == ("ptr" if ret == "constchar*" else _c_class(ret)), name
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    """Without the built library the binding raises: nothing falls back to a
+    CPU path or to the oracle."""
+    from quantized_gemm_column_b200 import api
+    monkeypatch.setattr(api, "_LIB", None)
+    monkeypatch.setattr(api._build, "LIB", str(tmp_path / "libaveris.so"))
+    with pytest.raises(api.AverisError) as e:
+        api.load()
+    assert e.value.status == api.AVR_ERR_NO_DEVICE
+    with pytest.raises(api.AverisError):
+        api.averis_workspace_size(256, 128)
+
+
+def test_product_path_never_imports_the_oracle():
+    """The package's sources name no oracle module: only the tests, the smoke
+    check and the benchmark's CPU legs use it."""
+    pkg = os.path.join(ROOT, "quantized_gemm_column_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, flags=re.M), f
+                assert "import oracle" not in text, f
