@@ -381,3 +381,17 @@ def test_product_path_never_imports_the_oracle():
                 text = open(os.path.join(dirpath, f), encoding="utf-8").read()
                 assert not re.search(r"^\s*(import|from)\s+oracle\b", text, flags=re.M), f
                 assert "import oracle" not in text, f
+
+
+def test_oracle_imports_nothing_of_the_cuda_path():
+    """The oracle is independent of the CUDA path: it imports only numpy and
+    the standard library, never the package or its library."""
+    allowed = {"numpy", "math", "dataclasses"}
+    odir = os.path.join(ROOT, "oracle")
+    for f in os.listdir(odir):
+        if not f.endswith(".py"):
+            continue
+        text = open(os.path.join(odir, f), encoding="utf-8").read()
+        for mod in re.findall(r"^\s*(?:import|from)\s+([\w.]+)", text, flags=re.M):
+            assert mod.startswith(".") or mod.split(".")[0] in allowed, (f, mod)
+        assert "quantized_gemm_column_b200" not in text and "libaveris" not in text, f
