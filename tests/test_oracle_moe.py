@@ -108,3 +108,23 @@ def test_moe_chain_is_exact_on_representable_inputs(rounding):
             for k in range(K):
                 ref[i] += Xe[i, k] * Ws[e][k].astype(np.float64)
         assert np.allclose(Y[e], ref, rtol=1e-6, atol=1e-6 * np.abs(ref).max())
+
+
+def test_experts_draw_separate_streams():
+    """Two experts holding the same tokens round them independently: each
+    buffer row has its own place in the stream, so their stochastic codes
+    differ in about half of the elements whose round-up probability is 1/2."""
+    K, n = 128, 64
+    a = np.full((n, K), 1.25, np.float32)
+    a[:, ::16] = 6.0
+    a[1::2] *= -1                                     # +/- row pairs: mu = 0, X_R = X
+    offs, L = oracle.moe_offsets([n, n])
+    X = np.zeros((L, K), np.float32)
+    X[offs[0]:offs[0] + n] = a
+    X[offs[1]:offs[1] + n] = a
+    s = oracle.moe_split_quant(X, [n, n], "sr", seed=2, offset=5)
+    c0, c1 = (oracle.unpack_codes(s[e]["xr_q"].codes)[:n] & 7 for e in (0, 1))
+    assert np.array_equal(s[0]["xr_q"].scales[:n], s[1]["xr_q"].scales[:n])
+    free = np.abs(a) != 6.0
+    differ = np.mean(c0[free] != c1[free])
+    assert 0.35 < differ < 0.65, differ

@@ -14,7 +14,9 @@ case, in every module that holds a reference to it.
 Some readings cannot be pinned on the CPU at all: which stream tag an operand
 draws from, or how the stream's values are laid over a tensor's elements, are
 conventions the pages leave open; any choice passes every CPU pin and only the
-bit-exact device comparison tells them apart.  No case plants such a mistake.
+bit-exact device comparison tells them apart.  What the CPU does pin is that
+the operands draw separate streams (mean and residual, activation and
+gradient, one expert and the next), and the cases that break that are here.
 
 A control case runs the same harness on the unmodified oracle and requires
 every pin to pass, so that a broken harness cannot pass the mutation cases.
@@ -181,6 +183,11 @@ MUTATIONS = [
        "(_as_f32(X) + np.asarray(mu, dtype=np.float32)[None, :])")], []),
     ("residual amax taken of X", A, "column_mean_and_residual_amax",
      [("np.max(np.abs(XR))", "np.max(np.abs(_as_f32(X)))")], []),
+    ("mean quantized from the residual's stream", A, "averis_split_quant",
+     [("mu_q = nvfp4_quantize(mu[None, :], rounding, seed, offset, t_mu)",
+       "mu_q = nvfp4_quantize(mu[None, :], rounding, seed, offset, t_r)")], []),
+    ("gradient split on the activation's streams", A, "averis_split_quant",
+     [("if grad else (TAGS[\"x_r\"], TAGS[\"mu_x\"])", "if False else (TAGS[\"x_r\"], TAGS[\"mu_x\"])")], []),
     ("mean quantized with the residual's tensor scale", A, "averis_split_quant",
      [("mu_q = nvfp4_quantize(mu[None, :], rounding, seed, offset, t_mu)",
        "mu_q = nvfp4_quantize(mu[None, :], rounding, seed, offset, t_mu, amax=A)")], []),
@@ -200,6 +207,8 @@ MUTATIONS = [
     ("expert segments aligned to 64", A, "moe_offsets",
      [("(int(n) + MOE_ALIGN - 1) // MOE_ALIGN * MOE_ALIGN", "(int(n) + 63) // 64 * 64")], []),
     ("expert statistics from the buffer's start", A, "moe_split_quant", [("Xe = X[o:o + n]", "Xe = X[:o + n]")], []),
+    ("every expert's stream starts at the offset", A, "moe_split_quant",
+     [("offset + (o * K) // 16, t_r", "offset, t_r")], []),
     # ---- the monitor ----
     ("energy ratio normalised by the token count", S, "mean_energy_ratio", [("m = X.shape[1]", "m = X.shape[0]")], []),
     ("energy ratio without the square root", S, "mean_energy_ratio",

@@ -192,3 +192,43 @@ def test_nonfinite_rejected():
     X[1, 1] = np.inf
     with pytest.raises(ValueError):
         oracle.averis_split_quant(X)
+
+
+# --------------------------------------------------------------------------
+# separate random streams for the split's operands
+# --------------------------------------------------------------------------
+def _twin_rows(K=256):
+    """X = [2a; 0] with a on the grid of 1.25 steps and a 6 in every block:
+    mu = a and X_R = [a; -a] exactly, and mu and X_R share the tensor amax
+    (6), so mu and row 0 of X_R have the same scales and the same scaled
+    values, each 1.25 (round-up probability 1/2) except the block maxima."""
+    a = np.full(K, 1.25, dtype=np.float32)
+    a[::16] = 6.0
+    return np.stack([2 * a, np.zeros(K, np.float32)]), a
+
+
+def test_mean_and_residual_draw_separate_streams():
+    """With one stream for both, mu_bar and row 0 of X_bar_R would round every
+    element the same way; with separate streams about half of the 1.25s
+    round differently (the stochastic rounding of the two operands must be
+    independent)."""
+    X, a = _twin_rows()
+    mu, XR, mu_q, xr_q = oracle.averis_split_quant(X, "sr", seed=11, offset=3)
+    assert np.array_equal(mu, a) and np.array_equal(XR[0], a)
+    assert np.array_equal(mu_q.scales[0], xr_q.scales[0]) and mu_q.g_dec == xr_q.g_dec
+    c_mu, c_r = F.unpack_codes(mu_q.codes)[0], F.unpack_codes(xr_q.codes)[0]
+    free = a != 6.0
+    assert set(np.unique(c_mu[free])) <= {2, 3} and set(np.unique(c_r[free])) <= {2, 3}
+    differ = np.mean(c_mu[free] != c_r[free])
+    assert 0.35 < differ < 0.65, differ
+
+
+def test_activation_and_gradient_splits_draw_separate_streams():
+    """The forward's and the dgrad's split of the same tensor (same seed and
+    offset) round independently."""
+    X, a = _twin_rows()
+    _, _, _, q_x = oracle.averis_split_quant(X, "sr", seed=11, offset=3, grad=False)
+    _, _, _, q_d = oracle.averis_split_quant(X, "sr", seed=11, offset=3, grad=True)
+    free = np.tile(a != 6.0, (2, 1))
+    differ = np.mean(F.unpack_codes(q_x.codes)[free] != F.unpack_codes(q_d.codes)[free])
+    assert 0.35 < differ < 0.65, differ
